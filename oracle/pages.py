@@ -1,0 +1,204 @@
+"""Page-level model of the two-stream paged KV cache, for bit-exact checks.
+
+Test infrastructure only (see the package docstring).
+
+Physical pool, per transformer block: [max_pages, 2, page_size, H, D]
+([P1] "Physical Memory Layout"). Dimension 1 is read as K (0) / V (1); the two
+streams are told apart by page-id range: patch pages are [0, Np), special pages
+are [Np, max_pages) ([P3] "Constant Memory with Two-Stream Paging": memory is
+max_patch_pages + max_special_pages).
+
+Patch stream ([P1] "Patch Stream (Recyclable)"; [P3] same section): one page
+per frame, page_size == patches per frame. Pages come from a free list; evicted
+pages go back on it. The free list is a LIFO stack that starts as
+[Np-1, ..., 1, 0], so the first pops yield 0, 1, 2, ...
+
+Special stream ([P1] "Special Stream (Append-Only)"): NS tokens per frame,
+packed back to back with no padding; special token j (0-based over the stream)
+lives on page Np + j // page_size at slot j % page_size.
+
+Visible page table ([P1] "Building the Visible Page Table"; [P3] "Visible Page
+Table Attention"): scale pages in frame order, window pages oldest to newest,
+then the pending page if any, then special pages Np .. Np+k-1. Only the last
+page may be partial; last_page_len is the fill of the last special page.
+
+get_cache_stats keys ([P3] "Monitoring Cache Statistics"): frame_count,
+scale_pages, live_pages, free_pages, special_tokens.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+class OracleError(Exception):
+    def __init__(self, code: str, msg: str = ""):
+        super().__init__(f"{code}: {msg}")
+        self.code = code
+
+
+class PageModel:
+    def __init__(self, S: int, W: int, page_size: int, max_pages: int,
+                 NS: int = 6, patch_pages: int | None = None):
+        self.S, self.W, self.ps, self.NS = S, W, page_size, NS
+        self.Np = patch_pages if patch_pages else S + W + 1
+        if self.Np < 1 or max_pages < self.Np + (1 if NS > 0 else 0):
+            raise OracleError("CAPACITY", "pool too small")
+        self.max_pages = max_pages
+        self.reset()
+
+    def reset(self) -> None:
+        self.free = list(range(self.Np - 1, -1, -1))
+        self.scale: list[tuple[int, int]] = []    # (frame, page)
+        self.window: list[tuple[int, int]] = []   # (frame, page), oldest first
+        self.pending: tuple[int, int] | None = None
+        self.sp_len = 0
+        self.sp_owner: list[tuple[int, int]] = []  # (frame, slot) of special token j
+        self.committed = 0
+        self.defer = False
+
+    @property
+    def special_capacity(self) -> int:
+        return (self.max_pages - self.Np) * self.ps
+
+    # -- operations -------------------------------------------------------
+    def append(self, f: int) -> tuple[int, int]:
+        """New frame f: returns (patch page, first special slot index)."""
+        if self.pending is not None:
+            raise OracleError("ORDER", "pending frame")
+        if not self.free:
+            raise OracleError("CAPACITY", "no free patch page")
+        if self.sp_len + self.NS > self.special_capacity:
+            raise OracleError("CAPACITY", "special stream full")
+        page = self.free.pop()
+        sp0 = self.sp_len
+        self.sp_len += self.NS
+        self.sp_owner.extend((f, i) for i in range(self.NS))
+        if self.defer:
+            self.pending = (f, page)
+        else:
+            self._commit(f, page)
+        return page, sp0
+
+    def _commit(self, f: int, page: int) -> None:
+        if len(self.scale) < self.S:
+            self.scale.append((f, page))
+        else:
+            self.window.append((f, page))
+        self.committed += 1
+
+    def evict(self) -> list[int]:
+        """Frees window pages beyond W, oldest first; returns the freed frames."""
+        if self.defer:
+            return []
+        freed = []
+        while len(self.window) > self.W:
+            f, p = self.window.pop(0)
+            self.free.append(p)
+            freed.append(f)
+        return freed
+
+    def set_defer(self, on: bool) -> None:
+        if not on and self.pending is not None:
+            raise OracleError("ORDER", "pending frame")
+        self.defer = bool(on)
+
+    def commit(self) -> None:
+        if self.pending is None:
+            raise OracleError("NO_PENDING")
+        f, p = self.pending
+        self.pending = None
+        self.defer = False
+        self._commit(f, p)
+        self.evict()
+
+    def rollback(self) -> None:
+        if self.pending is None:
+            raise OracleError("NO_PENDING")
+        _, p = self.pending
+        self.pending = None
+        self.defer = False
+        self.free.append(p)
+        self.sp_len -= self.NS
+        del self.sp_owner[self.sp_len:]
+
+    # -- queries ----------------------------------------------------------
+    def patch_pages_visible(self) -> list[tuple[int, int]]:
+        out = self.scale + self.window
+        if self.pending is not None:
+            out = out + [self.pending]
+        return out
+
+    def page_table(self) -> tuple[list[int], int]:
+        """(kv_indices, last_page_len) of the visible page table."""
+        if self.committed == 0 and self.pending is None:
+            raise OracleError("EMPTY")
+        patch = [p for _, p in self.patch_pages_visible()]
+        k = -(-self.sp_len // self.ps)
+        special = [self.Np + i for i in range(k)]
+        last = self.sp_len - self.ps * (k - 1) if k else self.ps
+        return patch + special, last
+
+    def visible_token_count(self) -> int:
+        return len(self.patch_pages_visible()) * self.ps + self.sp_len
+
+    def stats(self) -> dict:
+        pend = 1 if self.pending is not None else 0
+        return {
+            "frame_count": self.committed + pend,
+            "scale_pages": len(self.scale),
+            "live_pages": len(self.window) + pend,
+            "free_pages": len(self.free),
+            "special_tokens": self.sp_len,
+        }
+
+    def special_location(self, j: int) -> tuple[int, int]:
+        return self.Np + j // self.ps, j % self.ps
+
+    def visible_tokens(self) -> set:
+        """Visible tokens in the frame simulator's ('p', frame, t) / ('s', frame,
+        slot) form, read back through the page table: each listed page and
+        slot is mapped to the frame that wrote it."""
+        table, last = self.page_table()
+        owner = {p: f for f, p in self.patch_pages_visible()}
+        out = set()
+        for n, p in enumerate(table):
+            cnt = last if n == len(table) - 1 else self.ps
+            for t in range(cnt):
+                if p < self.Np:
+                    out.add(("p", owner[p], t))
+                else:
+                    out.add(("s",) + self.sp_owner[(p - self.Np) * self.ps + t])
+        return out
+
+    def snapshot(self):
+        return (tuple(self.free), tuple(self.scale), tuple(self.window), self.pending,
+                self.sp_len, tuple(self.sp_owner), self.committed, self.defer)
+
+
+class PoolImage:
+    """Expected raw contents of one block's pool: [max_pages, 2, ps, H, D] of
+    16-bit bit patterns. `write` mirrors what an append stores."""
+
+    def __init__(self, model: PageModel, H: int, D: int):
+        self.m = model
+        self.bits = np.zeros((model.max_pages, 2, model.ps, H, D), dtype=np.uint16)
+
+    def write(self, page: int, sp0: int, k_bits: np.ndarray, v_bits: np.ndarray) -> None:
+        """k_bits, v_bits: [NS + P, H, D] uint16. Tokens 0..NS-1 are the frame's
+        special tokens, NS.. its patch tokens."""
+        NS, ps = self.m.NS, self.m.ps
+        for kv, x in ((0, k_bits), (1, v_bits)):
+            self.bits[page, kv, :ps] = x[NS:NS + ps]
+            for i in range(NS):
+                pg, slot = self.m.special_location(sp0 + i)
+                self.bits[pg, kv, slot] = x[i]
+
+    def gather(self, kv_indices, last_page_len):
+        """Visible K and V rows in page-table order: two [L, H, D] uint16 arrays."""
+        ps = self.m.ps
+        ks, vs = [], []
+        for n, p in enumerate(kv_indices):
+            cnt = last_page_len if n == len(kv_indices) - 1 else ps
+            ks.append(self.bits[p, 0, :cnt])
+            vs.append(self.bits[p, 1, :cnt])
+        return np.concatenate(ks), np.concatenate(vs)

@@ -1,0 +1,224 @@
+"""Pins for the oracle's cache-state models (no GPU).
+
+The page-level model and the frame-list simulator are pinned against the
+values the pages print, against closed forms of the retention rule, and
+against each other on random operation sequences.
+"""
+import json
+import math
+import os
+
+import pytest
+from hypothesis import given, settings, strategies as st
+
+from oracle import FrameListSim, PageModel, OracleError
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def load(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def test_stats_example_12_frames():
+    g = load("cache_stats_12_frames.json")
+    c = g["config"]
+    m = PageModel(c["scale_frames"], c["sliding_window"], c["page_size"],
+                  max_pages=g["patch_pages"] + 2, NS=c["num_special"],
+                  patch_pages=g["patch_pages"])
+    for f in range(c["frames"]):
+        m.append(f)
+        m.evict()
+    assert m.stats() == g["expected"]
+
+
+def test_interval_keyframes_200_frames():
+    g = load("keyframe_interval_200.json")
+    n, k = g["frames"], g["keyframe_interval"]
+    S, W, NS = 8, g["sliding_window"], g["special_tokens_per_frame"]
+    m = PageModel(S, W, 256, max_pages=S + W + 1 + 4, NS=NS)
+    sim = FrameListSim(S, W, NS)
+    for t in range(n):
+        key = (t % k) == 0
+        for model in (m, sim):
+            if key:
+                model.append(t)
+                model.evict()
+            else:
+                model.set_defer(True)
+                model.append(t)
+                model.evict()
+                model.rollback()
+    assert m.committed == g["expected_keyframes"]
+    assert len(sim.C) == g["expected_keyframes"]
+    assert m.sp_len == NS * g["expected_keyframes"]
+    assert len(sim.SP) == NS * g["expected_keyframes"]
+
+
+@pytest.mark.parametrize("ps,n,pages,lpl", [
+    (16, 12, 5, 8),      # 72 special tokens on 16-token pages: 4 full + 8
+    (256, 320, 8, 128),  # 1920 tokens on 256-token pages: 7 full + 128
+    (999, 1000, 7, 6),   # 6000 tokens on 999-token pages: 6 full + 6
+])
+def test_special_stream_worked_sizes(ps, n, pages, lpl):
+    m = PageModel(8, 64, ps, max_pages=73 + pages, NS=6)
+    for f in range(n):
+        m.append(f)
+        m.evict()
+    table, last = m.page_table()
+    special = [p for p in table if p >= m.Np]
+    assert len(special) == pages
+    assert last == lpl
+    assert m.sp_len == 6 * n
+
+
+@pytest.mark.parametrize("ps", [16, 17, 256, 999])
+def test_special_stream_grows_six_per_frame(ps):
+    m = PageModel(2, 4, ps, max_pages=7 + 64, NS=6)
+    for n in range(1, 120):
+        before = m.sp_len
+        m.append(n)
+        m.evict()
+        assert m.sp_len - before == 6
+        table, last = m.page_table()
+        # continuous packing: 6n tokens fill ceil(6n/ps) pages, the last one
+        # holding the remainder (a full page when 6n is a multiple of ps)
+        assert len([p for p in table if p >= m.Np]) == math.ceil(6 * n / ps)
+        assert last == ((6 * n - 1) % ps) + 1
+
+
+@pytest.mark.parametrize("S,W", [(8, 64), (2, 4), (0, 3), (3, 0), (1, 1)])
+def test_retained_frames_closed_form(S, W):
+    """After n keyframes: the first min(n, S) frames plus the latest
+    min(n - S, W) others are resident, i.e. min(n, S + W) frames."""
+    sim = FrameListSim(S, W, 6)
+    m = PageModel(S, W, 16, max_pages=S + W + 1 + 200, NS=6)
+    for n in range(1, 200):
+        f = n - 1
+        sim.append(f)
+        sim.evict()
+        m.append(f)
+        m.evict()
+        want = list(range(min(n, S))) + list(range(max(S, n - W), n))
+        assert sim.patch_frames() == want
+        assert [f for f, _ in m.patch_pages_visible()] == want
+        assert len(want) == min(n, S + W)
+
+
+def test_free_list_pops_in_order_and_reuses_evicted_page():
+    m = PageModel(2, 3, 16, max_pages=7, NS=1)
+    pages = [m.append(f)[0] for f in range(3)]
+    assert pages == [0, 1, 2]
+    for f in range(3, 6):
+        page, _ = m.append(f)
+        m.evict()
+        assert page == f
+    # window now holds frames 3,4,5 (W=3); frame 2 was evicted -> page 2 freed
+    page, _ = m.append(6)
+    assert page == 2
+
+
+def test_capacity_errors():
+    with pytest.raises(OracleError) as e:
+        PageModel(2, 2, 16, max_pages=5, NS=6)
+    assert e.value.code == "CAPACITY"
+    m = PageModel(1, 1, 16, max_pages=4, NS=6)   # 1 special page = 16 tokens
+    m.append(0); m.evict()
+    m.append(1); m.evict()
+    with pytest.raises(OracleError) as e:
+        m.append(2)
+    assert e.value.code == "CAPACITY"
+    with pytest.raises(OracleError) as e:
+        PageModel(1, 1, 16, max_pages=4).page_table()
+    assert e.value.code == "EMPTY"
+
+
+def _invariants(m: PageModel):
+    used = [p for _, p in m.scale] + [p for _, p in m.window]
+    if m.pending is not None:
+        used.append(m.pending[1])
+    assert len(used) + len(m.free) == m.Np
+    assert sorted(used + m.free) == list(range(m.Np))
+    assert len(m.scale) <= m.S
+    if not m.defer:
+        assert len(m.window) <= m.W
+    assert len(m.sp_owner) == m.sp_len
+
+
+OPS = st.lists(st.sampled_from(["key", "key", "key", "defer_keep", "defer_drop",
+                                "evict", "bad_commit", "bad_rollback"]),
+               min_size=1, max_size=60)
+
+
+@settings(max_examples=150, deadline=None)
+@given(ops=OPS, S=st.integers(0, 3), W=st.integers(0, 4), ps=st.sampled_from([1, 5, 16]))
+def test_page_model_matches_frame_list(ops, S, W, ps):
+    NS = 6
+    m = PageModel(S, W, ps, max_pages=S + W + 1 + (NS * 64) // ps + 2, NS=NS)
+    sim = FrameListSim(S, W, NS)
+    f = 0
+    for op in ops:
+        if op == "evict":
+            m.evict(); sim.evict()
+        elif op == "key":
+            m.set_defer(False); sim.set_defer(False)
+            m.append(f); sim.append(f)
+            m.evict(); sim.evict()
+            f += 1
+        elif op in ("defer_keep", "defer_drop"):
+            m.set_defer(True); sim.set_defer(True)
+            m.append(f); sim.append(f)
+            m.evict(); sim.evict()
+            assert m.visible_tokens() == sim.visible_tokens(ps)
+            _invariants(m)
+            if op == "defer_keep":
+                m.commit(); sim.commit()
+            else:
+                m.rollback(); sim.rollback()
+            f += 1
+        elif op == "bad_commit":
+            with pytest.raises(OracleError):
+                m.commit()
+            with pytest.raises(ValueError):
+                sim.commit()
+        elif op == "bad_rollback":
+            with pytest.raises(OracleError):
+                m.rollback()
+            with pytest.raises(ValueError):
+                sim.rollback()
+        _invariants(m)
+        if m.committed or m.pending is not None:
+            assert m.visible_tokens() == sim.visible_tokens(ps)
+            assert m.visible_token_count() == len(sim.visible_tokens(ps))
+
+
+@settings(max_examples=100, deadline=None)
+@given(n=st.integers(0, 90), S=st.integers(0, 4), W=st.integers(0, 5))
+def test_rollback_restores_pre_append_state(n, S, W):
+    m = PageModel(S, W, 7, max_pages=S + W + 1 + 100, NS=6)
+    sim = FrameListSim(S, W, 6)
+    for f in range(n):
+        m.append(f); m.evict()
+        sim.append(f); sim.evict()
+    before_m, before_s = m.snapshot(), sim.snapshot()
+    for model in (m, sim):
+        model.set_defer(True)
+        model.append(n)
+        model.evict()
+        model.rollback()
+    assert m.snapshot() == before_m
+    assert sim.snapshot() == before_s
+
+
+def test_deferred_frame_is_visible_on_top_of_full_window():
+    S, W = 2, 3
+    m = PageModel(S, W, 16, max_pages=S + W + 1 + 10, NS=6)
+    for f in range(10):
+        m.append(f); m.evict()
+    m.set_defer(True)
+    m.append(10)
+    m.evict()                                  # no-op while deferred
+    assert [f for f, _ in m.patch_pages_visible()] == [0, 1, 7, 8, 9, 10]
+    m.commit()                                 # commit runs the eviction
+    assert [f for f, _ in m.patch_pages_visible()] == [0, 1, 8, 9, 10]
