@@ -1,0 +1,415 @@
+"""Benchmark: frames/s of the 24-block per-frame paged-KV prefill step on a
+224x224, 320-frame stream (H=16, D=64, 256 patch + 6 special tokens, page 256,
+8 scale frames, window 64), plus attention TFLOP/s and its roofline fraction.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 1]
+    python bench.py --impl reference ...   # the CPU oracle, timed on host cores
+
+One step = the whole stream: reset, then for each of the 320 frames one plan
+and 24 x (append_frame + run) through the C-ABI, with evict_frames after each
+append. Inputs come from a ring of 16 seeded frame sets already in HBM; the
+24 block pools (1.9 GB) exceed L2, so every call reads its K/V from HBM.
+With --gpus N (torchrun) each rank runs an independent replica stream (the
+path does not shard); value = frames of all ranks / max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workload  # noqa: E402
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+def call_flops(T, lkv, H, D):
+    """Tensor FLOPs of one attention call: Q K^T and P V, 2 per MAC."""
+    return 4.0 * T * lkv * H * D
+
+
+def call_kv_bytes(lkv, H, D, elt=2):
+    """Algorithmic HBM bytes of one call: the visible K and V rows, read once."""
+    return 2.0 * lkv * H * D * elt
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}",
+                 "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.15)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                smax.append(float(f[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------ GPU arm
+class StreamRunner:
+    """One replica of the workload's stream on the current GPU."""
+
+    def __init__(self, wl, seed, ring=16):
+        import torch
+        import paged_kv_cache_frame_b200 as pkv
+        from paged_kv_cache_frame_b200 import capi
+        self.torch, self.pkv, self.capi = torch, pkv, capi
+        self.L = capi.lib()
+        self.wl, self.ring_n = wl, ring
+        self.stream = torch.cuda.current_stream()
+        self.sp = self.stream.cuda_stream
+        self.cache = pkv.PagedKVCache(wl.max_pages, wl.page_size, wl.H, wl.D, wl.S, wl.W,
+                                      num_blocks=wl.blocks, num_special=wl.NS, dtype=wl.dtype)
+        self.cache.allocate_pools("cuda")
+        self.h = self.cache.handle
+        self.ws = torch.empty(pkv.workspace_bytes([self.cache]), dtype=torch.uint8, device="cuda")
+        self.ring = workload.qkv_ring_cuda(wl, seed, ring)            # [R, B, 3, T, H, D]
+        self.out = torch.empty((wl.blocks, wl.T, wl.H, wl.D), dtype=wl.torch_dtype(), device="cuda")
+        self.keep = workload.keyframe_mask(wl, seed)
+        self.defer = wl.keyframes != "all"
+        elt = self.ring.element_size()
+        self.ptr = [[[self.ring[r, b, i].data_ptr() for i in range(3)] for b in range(wl.blocks)]
+                    for r in range(ring)]
+        self.optr = [self.out[b].data_ptr() for b in range(wl.blocks)]
+        self.ws_ptr, self.ws_bytes = self.ws.data_ptr(), self.ws.numel()
+        self.stats = []          # per frame: (lkv, splits)
+        self.launches = 0
+        self._elt = elt
+
+    def _chk(self, rc, what):
+        if rc != 0:
+            raise self.capi.KVError(rc, what, self.L.kv_last_error().decode())
+
+    def one_pass(self, events=None, host=None):
+        """One pass over the stream. events: list to receive (start, end)
+        event pairs around every kv_run. host: (pinned ring, pinned out, dev
+        staging) for the end-to-end variant that copies inputs in and outputs
+        out every frame."""
+        torch, L, wl, h, sp = self.torch, self.L, self.wl, self.h, self.sp
+        self._chk(L.kv_reset(h), "kv_reset")
+        plan = ctypes.c_void_p()
+        cache_arr = (ctypes.c_void_p * 1)(h)
+        self.stats = []
+        launches = 0
+        for f in range(wl.frames):
+            r = f % self.ring_n
+            if host is not None:
+                hring, hout, dstage = host
+                dstage.copy_(hring[r], non_blocking=True)
+                ptr = [[dstage[b, i].data_ptr() for i in range(3)] for b in range(wl.blocks)]
+            else:
+                ptr = self.ptr[r]
+            if self.defer:
+                self._chk(L.kv_defer_eviction(h, 1), "defer")
+            for b in range(wl.blocks):
+                q, k, v = ptr[b]
+                self._chk(L.kv_append_frame(h, b, k, v, sp), "append")
+                launches += 1
+                if b == 0:
+                    self._chk(L.kv_evict_frames(h), "evict")
+                    if plan.value:
+                        L.kv_plan_free(plan)
+                    self._chk(L.kv_plan(ctypes.byref(plan), cache_arr, 1, 0, self.ws_ptr, self.ws_bytes, sp),
+                              "plan")
+                    st = self.capi.kv_plan_stats()
+                    L.kv_plan_get_stats(plan, ctypes.byref(st))
+                    launches += 1
+                    self.stats.append((st.visible_tokens, st.n_split_units))
+                if events is not None:
+                    e0 = torch.cuda.Event(enable_timing=True)
+                    e1 = torch.cuda.Event(enable_timing=True)
+                    e0.record(self.stream)
+                self._chk(L.kv_run(plan, b, q, self.optr[b], sp), "run")
+                launches += 1 + (1 if self.stats[-1][1] else 0)
+                if events is not None:
+                    e1.record(self.stream)
+                    events.append((e0, e1))
+            if self.defer:
+                if self.keep[f]:
+                    self._chk(L.kv_commit_frame(h), "commit")
+                else:
+                    self._chk(L.kv_rollback_last_frame(h), "rollback")
+            if host is not None:
+                hout[r].copy_(self.out, non_blocking=True)
+        if plan.value:
+            L.kv_plan_free(plan)
+        self.launches = launches
+        return launches
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    from paged_kv_cache_frame_b200 import build
+    build.build()
+    wl = workload.WORKLOADS[args.workload]
+    runner = StreamRunner(wl, seed=args.seed + 1000 * rank)
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        runner.one_pass()
+    torch.cuda.synchronize()
+
+    # ---- timed region: K passes over the stream, inputs resident in HBM
+    events = []
+    barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    with clocks:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record()
+        launches = 0
+        for _ in range(args.steps):
+            launches += runner.one_pass(events=events)
+        t1.record()
+        torch.cuda.synchronize()
+    barrier()
+    ms = t0.elapsed_time(t1)
+    ms_t = torch.tensor([ms], device="cuda")
+    if world > 1:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+    frames_total = args.steps * wl.frames * world
+    value = frames_total / (ms_max / 1e3)
+
+    # per-call attention time (run = attention + merge) against the roofline
+    run_ms = [a.elapsed_time(b) for a, b in events]
+    per_pass = len(run_ms) // args.steps
+    lkvs = [s[0] for s in runner.stats]                 # per frame of the last pass
+    flops = sum(call_flops(wl.T, l, wl.H, wl.D) for l in lkvs) * wl.blocks
+    kvbytes = sum(call_kv_bytes(l, wl.H, wl.D) for l in lkvs) * wl.blocks
+    run_s = sum(run_ms[-per_pass:]) / 1e3
+    pk, pk_kind = peaks()
+    tflops = flops / run_s / 1e12
+    gbs = kvbytes / run_s / 1e9
+    t_roof = sum(max(call_flops(wl.T, l, wl.H, wl.D) / (pk["bf16_tflops"] * 1e12),
+                     call_kv_bytes(l, wl.H, wl.D) / (pk["hbm_gbs"] * 1e9)) for l in lkvs) * wl.blocks
+    roof_frac = t_roof / run_s
+
+    # ---- end to end: host (pinned) inputs copied in, outputs copied out, every frame
+    e2e = None
+    if not args.no_e2e:
+        hring = runner.ring.cpu().pin_memory()
+        hout = torch.empty((runner.ring_n,) + tuple(runner.out.shape), dtype=runner.out.dtype).pin_memory()
+        dstage = torch.empty_like(runner.ring[0])
+        runner.one_pass(host=(hring, hout, dstage))
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(args.steps):
+            runner.one_pass(host=(hring, hout, dstage))
+        b.record()
+        torch.cuda.synchronize()
+        barrier()
+        ems = torch.tensor([a.elapsed_time(b)], device="cuda")
+        if world > 1:
+            dist.all_reduce(ems, op=dist.ReduceOp.MAX)
+        e2e = {"value": frames_total / (float(ems.item()) / 1e3), "unit": "frames/s",
+               "h2d_bytes_per_step": int(dstage.numel() * dstage.element_size() * wl.frames),
+               "d2h_bytes_per_step": int(runner.out.numel() * runner.out.element_size() * wl.frames)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, args.seed, budget_s=args.cpu_budget)
+
+    if rank == 0:
+        line = {
+            "metric": "frames/s (24-block stack) at 224x224, 320 frames",
+            "value": round(value, 2), "unit": "frames/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+            "data": "synthetic (seeded N(0,1) Q/K/V, ring of 16 frame sets in HBM)",
+            "config": {"workload": wl.name, "frames": wl.frames, "blocks": wl.blocks, "H": wl.H,
+                       "D": wl.D, "tokens_per_frame": wl.T, "page_size": wl.page_size,
+                       "scale_frames": wl.S, "window": wl.W, "keyframes": wl.keyframes,
+                       "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (24 block pools, 1.9 GB, read every frame)"},
+            "attention": {"tflops": round(tflops, 2), "kv_gbs": round(gbs, 1),
+                          "roofline_frac": round(roof_frac, 4),
+                          "roofline_ms_per_pass": round(t_roof * 1e3, 3),
+                          "run_ms_per_pass": round(run_s * 1e3, 3)},
+            "roofline": {"bound": "tensor", "achieved": round(tflops, 2),
+                         "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": round(tflops / pk["bf16_tflops"], 4), "traffic": None,
+                         "peak_kind": f"{pk_kind} bf16 dense burst",
+                         "kernel": "paged_prefill_attn + splitkv_merge (kv_run), event-timed per call"},
+            "gpu_launches": launches,
+            "clocks": clocks.summary(),
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------ oracle arm
+def cpu_baseline(wl, seed, budget_s=20.0, frames_sample=(0, 71, 159, 319), rows=48):
+    """Times the CPU oracle (float64 dense attention) on a bounded sample of
+    the workload and extrapolates frames/s by FLOPs."""
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from oracle.stream import StreamOracle, bits16
+    fr_cache = {}
+
+    def fetch(f):
+        if f not in fr_cache:
+            fr_cache.clear()
+            fr_cache[f] = tuple(bits16(x) for x in workload.frame_qkv(wl, seed, f, 0))
+        return fr_cache[f]
+
+    so = StreamOracle(wl.S, wl.W, wl.NS, wl.P, wl.dtype, fetch)
+    rng = np.random.default_rng(seed)
+    sel = sorted(rng.choice(wl.T, size=min(rows, wl.T), replace=False).tolist())
+    t_att, fl = 0.0, 0.0
+    done = []
+    for f in range(max(frames_sample) + 1):
+        so.begin_frame(f)
+        if f in frames_sample:
+            t = time.perf_counter()
+            so.expected(sel)
+            dt = time.perf_counter() - t
+            lkv = len(so.sim.patch_frames()) * wl.P + len(so.sim.SP)
+            t_att += dt
+            fl += call_flops(len(sel), lkv, wl.H, wl.D)
+            done.append(f)
+            if t_att > budget_s:
+                break
+    gflops = fl / t_att / 1e9
+    # whole-workload FLOPs: every frame, every block
+    sim_l = [min(n, wl.S + wl.W) * wl.P + wl.NS * n for n in range(1, wl.frames + 1)]
+    total = sum(call_flops(wl.T, l, wl.H, wl.D) for l in sim_l) * wl.blocks
+    fps = wl.frames / (total / (gflops * 1e9))
+    threads = 1   # numpy einsum without BLAS runs on one thread
+    return {"value": fps, "unit": "frames/s", "cores": threads, "kind": "oracle",
+            "gflops": round(gflops, 3),
+            "sample": f"float64 oracle attention of block 0 at frames {[d + 1 for d in done]} for "
+                      f"{len(sel)} of {wl.T} query rows ({t_att:.1f} s); frames/s extrapolated by "
+                      f"the workload's {total / 1e12:.1f} TFLOP"}
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = workload.WORKLOADS[args.workload]
+    budget = max(5.0, 150.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        cpu_baseline(wl, args.seed, budget_s=budget / 4, frames_sample=(0,), rows=8)
+    t = time.perf_counter()
+    vals = []
+    for _ in range(args.steps):
+        vals.append(cpu_baseline(wl, args.seed, budget_s=budget, frames_sample=(71, 319), rows=16))
+    el = time.perf_counter() - t
+    v = statistics.median(x["value"] for x in vals)
+    line = {
+        "impl": "reference", "metric": "frames/s (24-block stack) at 224x224, 320 frames",
+        "value": v, "unit": "frames/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(el * 1e3 / max(1, args.steps), 1), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "frames": wl.frames, "blocks": wl.blocks},
+        "cpu_baseline": {"value": v, "unit": "frames/s", "cores": 1, "kind": "oracle",
+                         "sample": vals[-1]["sample"]},
+        "e2e": {"value": v, "unit": "frames/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", type=int, default=1, choices=[1, 2, 3, 4])
+    ap.add_argument("--seed", type=int, default=1)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

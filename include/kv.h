@@ -1,0 +1,254 @@
+/*
+ * paged_kv_cache_frame_b200 -- C-ABI for per-frame paged-KV prefill attention
+ * on NVIDIA B200 (sm_100a).
+ *
+ * The operation, from the LingBot-Map pages:
+ *   [P1] "How the Paged KV Cache Attention Mechanism Enables Long Sequence
+ *        Inference in LingBot-Map"
+ *   [P2] "KV Cache Mechanism in LingBot-Map for Streaming Inference: A Deep Dive"
+ *   [P3] "FlashInfer Paged KV Cache Performance Benefits in LingBot-Map:
+ *        Technical Implementation and Benchmarks"
+ *   [P4] "How LingBot-Map Achieves ~20 FPS Inference with Its KV Cache"
+ *
+ * Each video frame brings T = NS + P tokens (NS special tokens: camera,
+ * register, scale; P patch tokens). Per transformer block the frame's K/V are
+ * appended to a paged pool and the frame's T queries attend, with no mask,
+ * over every visible token: the S scale frames, the latest W window frames
+ * (the current one included) and the whole append-only special stream.
+ *
+ * Conventions for every call:
+ *   - Return value: KV_OK (0) or a negative KV_ERR_* code. Nothing aborts;
+ *     kv_last_error() gives a one-line detail of the last failure on the
+ *     calling thread.
+ *   - Device buffers (pool, q, k, v, out, workspace) belong to the caller. The
+ *     library never allocates device memory. Host state (kv_cache_t,
+ *     kv_plan_t) belongs to the library and is released by kv_destroy /
+ *     kv_plan_free.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Device work is
+ *     enqueued asynchronously on it; errors raised later inside a kernel are
+ *     reported by kv_check_device.
+ *   - Token order inside a frame, for q, k, v and out alike: tokens 0..NS-1
+ *     are the special tokens, NS..T-1 the patch tokens. Tensors [T, H, D] are
+ *     contiguous, 16-byte aligned, in the cache's dtype.
+ *   - Frame step rule. The first kv_append_frame of a frame step (any block)
+ *     advances the page state: it takes a patch page and NS special slots for
+ *     the new frame. Every other block must then be appended exactly once in
+ *     the same step before its kv_run. A step is complete when all blocks are
+ *     appended; the next append opens a new step. A pending (deferred) frame
+ *     must be committed or rolled back before the next step.
+ *   - Not thread-safe: one host thread drives a cache and its plans.
+ */
+#ifndef PAGED_KV_CACHE_FRAME_B200_KV_H
+#define PAGED_KV_CACHE_FRAME_B200_KV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  KV_OK = 0,
+  KV_ERR_ARG = -1,          /* null/out-of-range argument, misaligned pointer, bad shape */
+  KV_ERR_CAPACITY = -2,     /* pool too small, no free patch page, special stream full,
+                               workspace too small, too many streams in one plan */
+  KV_ERR_ORDER = -3,        /* call out of order (frame step rule above) */
+  KV_ERR_NO_PENDING = -4,   /* commit or rollback without a deferred frame */
+  KV_ERR_NOT_APPENDED = -5, /* kv_run for a block not appended in the current step */
+  KV_ERR_EMPTY = -6,        /* kv_plan before the first frame */
+  KV_ERR_CUDA = -7,         /* a CUDA runtime or driver call failed */
+  KV_ERR_DEVICE_CHECK = -8, /* a kernel set the device error word (bounded wait expired
+                               or an index check failed) */
+  KV_ERR_UNSUPPORTED = -9,  /* no kernel for this head_dim/dtype (head_dim must be 64 or 128) */
+  KV_ERR_STALE_PLAN = -10   /* the cache state changed after the plan was built */
+};
+
+enum { KV_BF16 = 0, KV_FP16 = 1 };
+
+/* Upper bound on the streams (requests) batched in one plan. */
+#define KV_MAX_STREAMS 32
+
+typedef struct kv_cache kv_cache_t; /* one video stream's cache, all blocks */
+typedef struct kv_plan kv_plan_t;   /* one frame step's execution plan */
+
+/* get_cache_stats ([P3] "Monitoring Cache Statistics").
+ *   frame_count    frames appended since init/reset and not rolled back
+ *                  (a pending frame counts)
+ *   scale_pages    resident scale-frame patch pages (<= scale_frames)
+ *   live_pages     resident window patch pages, a pending frame's page included
+ *   free_pages     patch pages on the free list
+ *   special_tokens tokens in the special stream (NS per frame_count)
+ * scale_pages + live_pages + free_pages == patch pages, always. */
+typedef struct kv_stats {
+  int frame_count;
+  int scale_pages;
+  int live_pages;
+  int free_pages;
+  int special_tokens;
+} kv_stats;
+
+/* Execution-plan summary, for tests and benchmarks. */
+typedef struct kv_plan_stats {
+  int n_streams;      /* requests in the plan */
+  int n_ctas;         /* CTAs of the attention launch (work units) */
+  int n_split_units;  /* (stream, head, q-tile) units split across CTAs */
+  int n_kv_tiles;     /* 128-token K/V tiles summed over streams */
+  int tiles_per_cta;  /* largest number of K/V tiles one CTA processes */
+  long long visible_tokens; /* visible tokens summed over streams */
+} kv_plan_stats;
+
+/* kv_init -- create one stream's cache ([P1] "Implementation Example": the
+ * FlashInferKVCacheManager constructor; [P2] "Configuration Parameters").
+ *   max_pages     pages per block pool: patch pages + special pages
+ *   page_size     tokens per page; must equal the patch tokens per frame
+ *                 ([P1] "Patch Stream (Recyclable)": one page per frame)
+ *   num_heads, head_dim   H, D of K/V/Q (D = 64 or 128 for kv_run)
+ *   scale_frames  S: the first S committed frames stay resident for good
+ *   window        W: at most W non-scale frames stay resident
+ *   num_blocks    transformer blocks (one pool each)
+ *   num_special   NS special tokens per frame (6 on the pages), >= 0
+ *   dtype         KV_BF16 or KV_FP16
+ *   patch_pages   size of the recyclable patch pool; 0 = S + W + 1 (append takes
+ *                 a page before eviction returns one). Pages [0, patch_pages) are
+ *                 patch pages, [patch_pages, max_pages) special pages.
+ * Errors: KV_ERR_ARG (bad value), KV_ERR_CAPACITY (max_pages < patch_pages + 1
+ * when num_special > 0). No CUDA call is made. */
+int kv_init(kv_cache_t** out, int max_pages, int page_size, int num_heads, int head_dim,
+            int scale_frames, int window, int num_blocks, int num_special, int dtype,
+            int patch_pages);
+
+/* kv_destroy -- free the host state. Pools are not touched. NULL is ignored. */
+void kv_destroy(kv_cache_t* c);
+
+/* kv_reset -- clean_kv_cache ([P2] "Manual Cache Control"): back to the state
+ * kv_init left, keeping the bound pools (their contents are not cleared). */
+int kv_reset(kv_cache_t* c);
+
+/* kv_pool_bytes -- bytes of one block's pool
+ * [max_pages, 2, page_size, H, D] ([P1] "Physical Memory Layout"). Dimension 1
+ * is K (0) / V (1); the two streams are told apart by page-id range. */
+size_t kv_pool_bytes(const kv_cache_t* c);
+
+/* kv_bind_pool -- lend block `block` a device pool of kv_pool_bytes() bytes,
+ * 16-byte aligned, owned by the caller and kept alive while the cache uses it.
+ * The pool is zero-filled on `stream` (so that masked rows a kernel reads
+ * past a page's end are finite) and a TMA descriptor for it is built on the
+ * host. Errors: KV_ERR_ARG, KV_ERR_CUDA. */
+int kv_bind_pool(kv_cache_t* c, int block, void* pool, void* stream);
+
+/* kv_append_frame -- append_frame(block_idx, k, v) ([P1] "Appending New
+ * Frames"). k, v: device [T, H, D]. Special tokens 0..NS-1 go to the special
+ * stream at its current length (packed continuously, possibly across two
+ * pages); patch tokens NS..T-1 fill the frame's patch page, taken from the
+ * free list by the first append of the step. Launches one scatter kernel
+ * with 16-byte stores on `stream`.
+ * If k and v are both NULL only the page state advances and the block is
+ * marked appended; nothing is written (for callers that fill the pool
+ * themselves, and host-side tests).
+ * Errors: KV_ERR_ARG, KV_ERR_ORDER (block appended twice in a step, or a
+ * pending frame from an earlier step), KV_ERR_CAPACITY (no free patch page or
+ * special stream full; the state is left unchanged), KV_ERR_CUDA. */
+int kv_append_frame(kv_cache_t* c, int block, const void* k, const void* v, void* stream);
+
+/* kv_evict_frames -- evict_frames ([P1] "Evicting Stale Frames"; [P2]
+ * "Sliding-Window Eviction Strategy"): while more than W window pages are
+ * resident, push the oldest on the free list. Scale and special pages are
+ * never touched. No-op while eviction is deferred. Idempotent. Host only. */
+int kv_evict_frames(kv_cache_t* c);
+
+/* kv_defer_eviction -- _set_defer_eviction ([P2] "Flow-Based Keyframe
+ * Selection"): with on != 0 the next appended frame stays pending (visible,
+ * not committed) and eviction is suspended until kv_commit_frame or
+ * kv_rollback_last_frame. Turning it off while a frame is pending is
+ * KV_ERR_ORDER. */
+int kv_defer_eviction(kv_cache_t* c, int on);
+
+/* kv_commit_frame -- execute_deferred_eviction ([P2] "Flow-Based Keyframe
+ * Selection"): the pending frame becomes a normal frame, eviction runs, defer
+ * is switched off. Errors: KV_ERR_NO_PENDING; KV_ERR_ORDER if its step has
+ * not appended every block. */
+int kv_commit_frame(kv_cache_t* c);
+
+/* kv_rollback_last_frame -- rollback_last_frame ([P2] "Flow-Based Keyframe
+ * Selection"; [P4] "Deferred Eviction and Rollback Mechanism"): discard the
+ * pending frame: its patch page goes back on the free list, the special stream
+ * shrinks by NS, defer is switched off and the step is closed. The page state
+ * then equals the state before the frame's append. Pool bytes are not
+ * touched. Errors: KV_ERR_NO_PENDING. */
+int kv_rollback_last_frame(kv_cache_t* c);
+
+/* kv_get_stats -- get_cache_stats ([P3] "Monitoring Cache Statistics"). */
+int kv_get_stats(const kv_cache_t* c, kv_stats* out);
+
+/* kv_get_free_list -- the free list bottom to top (the next page handed out is
+ * ids[n-1]). Writes at most `cap` ids; *n gets the full length. */
+int kv_get_free_list(const kv_cache_t* c, int* ids, int cap, int* n);
+
+/* kv_workspace_bytes -- device workspace kv_plan needs for these caches
+ * (plan tables, split-KV partials, the device error word). 0 on bad input. */
+size_t kv_workspace_bytes(kv_cache_t* const* caches, int n_streams);
+
+/* kv_plan -- plan() once per frame step ([P1] "FlashInfer Kernel Execution";
+ * [P3] "Visible Page Table Attention"). For each cache, build the visible page
+ * table ([P1] "Building the Visible Page Table"): scale pages in frame order,
+ * window pages oldest to newest, the pending page, then the special pages,
+ * and paged_kv_last_page_len = fill of the last special page (1..page_size).
+ * Split the 128-token K/V tiles over CTAs (tiles_per_split = 0: automatic
+ * schedule for the SM count; > 0: at most that many tiles per CTA, which
+ * forces split-KV for tests) and copy the tables into `workspace` on
+ * `stream` (kernel launches whose parameters carry the tables: asynchronous,
+ * no host staging buffer). Stream i's queries are rows
+ * [sum_{j<i} T, sum_{j<=i} T) of kv_run's q.
+ * workspace == NULL builds a host-only plan (kv_get_page_table works, kv_run
+ * does not). All caches must share page_size, H, D, NS, num_blocks and dtype.
+ * The plan stays valid, for every block, until a cache's page state changes.
+ * Errors: KV_ERR_ARG, KV_ERR_EMPTY (a cache with no frame), KV_ERR_CAPACITY
+ * (workspace smaller than kv_workspace_bytes, > KV_MAX_STREAMS), KV_ERR_CUDA. */
+int kv_plan(kv_plan_t** out, kv_cache_t* const* caches, int n_streams, int tiles_per_split,
+            void* workspace, size_t workspace_bytes, void* stream);
+
+/* kv_run -- run() for one block ([P1] "FlashInfer Kernel Execution"; [P3]
+ * "Custom CUDA Kernel Implementation"): for every stream r, head h and query
+ * row i of the frame,
+ *     out[i, h] = sum_j softmax_j(q[i, h] . k_j[h] / sqrt(D)) v_j[h]
+ * over the visible tokens j of block `block`'s pool, no mask. q, out: device
+ * [sum T, H, D] in the cache dtype; fp32 accumulation; out rounded to nearest
+ * even. Launches the attention kernel and, when the plan splits a unit, the
+ * split-KV merge kernel on `stream`.
+ * Errors: KV_ERR_ARG, KV_ERR_STALE_PLAN, KV_ERR_NOT_APPENDED, KV_ERR_CUDA. */
+int kv_run(const kv_plan_t* plan, int block, const void* q, void* out, void* stream);
+
+/* kv_plan_free -- release a plan's host state. NULL is ignored. */
+void kv_plan_free(kv_plan_t* plan);
+
+/* kv_get_page_table -- host copy of stream `stream_idx`'s visible page table:
+ * up to `cap` page ids into `indices`, the full count into *n, and
+ * paged_kv_last_page_len into *last_page_len. */
+int kv_get_page_table(const kv_plan_t* plan, int stream_idx, int* indices, int cap, int* n,
+                      int* last_page_len);
+
+/* kv_get_kv_tiles -- host copy of stream `stream_idx`'s K/V tile list, in
+ * visible-table order. Tile t reads pool K rows [row[t], row[t] + 128) of the
+ * [max_pages * 2 * page_size]-row space (its V rows start page_size later);
+ * columns [lo[t], hi[t]) of the tile are visible tokens, the rest are masked.
+ * Writes at most `cap` entries per array; *n gets the full count. */
+int kv_get_kv_tiles(const kv_plan_t* plan, int stream_idx, int* row, int* lo, int* hi, int cap, int* n);
+
+/* kv_plan_get_stats -- summary of the plan's schedule. */
+int kv_plan_get_stats(const kv_plan_t* plan, kv_plan_stats* out);
+
+/* kv_check_device -- synchronise `stream` and read the plan's device error
+ * word. KV_OK, KV_ERR_DEVICE_CHECK (bit set by a kernel) or KV_ERR_CUDA. */
+int kv_check_device(const kv_plan_t* plan, void* stream);
+
+/* kv_strerror -- static text for a status code. */
+const char* kv_strerror(int status);
+
+/* kv_last_error -- detail of the last failing call on this thread ("" if none). */
+const char* kv_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PAGED_KV_CACHE_FRAME_B200_KV_H */

@@ -40,7 +40,9 @@ class StreamOracle:
     def begin_frame(self, f: int, defer: bool = False) -> None:
         """Append frame f (deferred: pending until `end_frame`) and evict."""
         q, k, v = self.fetch(f)
-        k64, v64 = decode(k, self.dtype), decode(v, self.dtype)
+        # bf16/fp16 values are exact in float32; the arithmetic below is float64
+        k64 = decode(k, self.dtype).astype(np.float32)
+        v64 = decode(v, self.dtype).astype(np.float32)
         self.q = decode(q, self.dtype)
         self.sim.set_defer(defer)
         self.sim.append(f)
@@ -80,7 +82,12 @@ class StreamOracle:
         return np.concatenate(ks), np.concatenate(vs)
 
     def expected(self, rows=None) -> np.ndarray:
-        """Attention output [len(rows), H, D] for the current frame's query rows."""
+        """Attention output [len(rows), H, D] for the current frame's query rows,
+        computed head by head in float64."""
         k, v = self.visible_kv()
         q = self.q if rows is None else self.q[np.asarray(rows)]
-        return dense(q, k, v)
+        out = np.empty(q.shape)
+        for h in range(q.shape[1]):
+            out[:, h:h + 1] = dense(q[:, h:h + 1], k[:, h:h + 1].astype(np.float64),
+                                    v[:, h:h + 1].astype(np.float64))
+        return out

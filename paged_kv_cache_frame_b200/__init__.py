@@ -1,0 +1,288 @@
+"""Per-frame paged-KV prefill attention for streaming video on B200 (sm_100a).
+
+Python binding of the C-ABI in include/kv.h. The functions below carry the
+C names and only marshal arguments (torch tensors -> device pointers, torch
+streams -> cudaStream_t); every step of the path runs in libpkv.so.
+
+    cache = PagedKVCache(max_pages, page_size, H, D, scale_frames, window, num_blocks)
+    cache.allocate_pools("cuda")               # torch owns the memory, library borrows it
+    for frame in stream:
+        for b in range(num_blocks):
+            cache.append_frame(b, k[b], v[b])
+            cache.evict_frames()
+            if b == 0:
+                plan = Plan([cache], workspace)    # once per frame step
+            out[b] = plan.run(b, q[b])             # every block
+
+Token order inside a frame: tokens 0..NS-1 are the special tokens, NS..T-1
+the patch tokens, for q, k, v and out alike.
+"""
+from __future__ import annotations
+
+import ctypes
+
+from . import capi
+from .capi import KVError, KV_BF16, KV_FP16, KV_MAX_STREAMS
+
+__all__ = [
+    "PagedKVCache", "Plan", "KVError", "workspace_bytes", "KV_BF16", "KV_FP16", "KV_MAX_STREAMS",
+    "kv_init", "kv_destroy", "kv_reset", "kv_pool_bytes", "kv_bind_pool", "kv_append_frame",
+    "kv_evict_frames", "kv_defer_eviction", "kv_commit_frame", "kv_rollback_last_frame",
+    "kv_get_stats", "kv_get_free_list", "kv_workspace_bytes", "kv_plan", "kv_run",
+    "kv_plan_free", "kv_get_page_table", "kv_get_kv_tiles", "kv_plan_get_stats",
+    "kv_check_device", "kv_strerror", "kv_last_error",
+]
+
+
+def _ptr(x) -> int | None:
+    """Device (or host) address of a tensor, or an int address, or None."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(s) -> int | None:
+    if s is None:
+        import torch
+        if torch.cuda.is_available() and torch.cuda.is_initialized():
+            return torch.cuda.current_stream().cuda_stream
+        return None
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+# ---------------------------------------------------------------- C names
+def kv_init(max_pages, page_size, num_heads, head_dim, scale_frames, window, num_blocks,
+            num_special=6, dtype=KV_BF16, patch_pages=0) -> int:
+    h = ctypes.c_void_p()
+    capi.check(capi.lib().kv_init(ctypes.byref(h), max_pages, page_size, num_heads, head_dim,
+                                  scale_frames, window, num_blocks, num_special, dtype,
+                                  patch_pages), "kv_init")
+    return h.value
+
+
+def kv_destroy(c) -> None:
+    capi.lib().kv_destroy(c)
+
+
+def kv_reset(c) -> None:
+    capi.check(capi.lib().kv_reset(c), "kv_reset")
+
+
+def kv_pool_bytes(c) -> int:
+    return capi.lib().kv_pool_bytes(c)
+
+
+def kv_bind_pool(c, block, pool, stream=None) -> None:
+    capi.check(capi.lib().kv_bind_pool(c, block, _ptr(pool), _stream(stream)), "kv_bind_pool")
+
+
+def kv_append_frame(c, block, k, v, stream=None) -> None:
+    capi.check(capi.lib().kv_append_frame(c, block, _ptr(k), _ptr(v), _stream(stream)),
+               "kv_append_frame")
+
+
+def kv_evict_frames(c) -> None:
+    capi.check(capi.lib().kv_evict_frames(c), "kv_evict_frames")
+
+
+def kv_defer_eviction(c, on) -> None:
+    capi.check(capi.lib().kv_defer_eviction(c, 1 if on else 0), "kv_defer_eviction")
+
+
+def kv_commit_frame(c) -> None:
+    capi.check(capi.lib().kv_commit_frame(c), "kv_commit_frame")
+
+
+def kv_rollback_last_frame(c) -> None:
+    capi.check(capi.lib().kv_rollback_last_frame(c), "kv_rollback_last_frame")
+
+
+def kv_get_stats(c) -> dict:
+    s = capi.kv_stats()
+    capi.check(capi.lib().kv_get_stats(c, ctypes.byref(s)), "kv_get_stats")
+    return {f: getattr(s, f) for f, _ in s._fields_}
+
+
+def kv_get_free_list(c) -> list[int]:
+    n = ctypes.c_int()
+    capi.check(capi.lib().kv_get_free_list(c, None, 0, ctypes.byref(n)), "kv_get_free_list")
+    buf = (ctypes.c_int * max(1, n.value))()
+    capi.check(capi.lib().kv_get_free_list(c, buf, n.value, ctypes.byref(n)), "kv_get_free_list")
+    return list(buf[: n.value])
+
+
+def _handles(caches):
+    arr = (ctypes.c_void_p * len(caches))()
+    for i, c in enumerate(caches):
+        arr[i] = c
+    return arr
+
+
+def kv_workspace_bytes(caches) -> int:
+    return capi.lib().kv_workspace_bytes(_handles(caches), len(caches))
+
+
+def kv_plan(caches, tiles_per_split=0, workspace=None, workspace_bytes=0, stream=None) -> int:
+    h = ctypes.c_void_p()
+    if workspace is not None and not isinstance(workspace, int):
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    capi.check(capi.lib().kv_plan(ctypes.byref(h), _handles(caches), len(caches), tiles_per_split,
+                                  _ptr(workspace), workspace_bytes,
+                                  _stream(stream) if workspace is not None else None), "kv_plan")
+    return h.value
+
+
+def kv_run(plan, block, q, out, stream=None) -> None:
+    capi.check(capi.lib().kv_run(plan, block, _ptr(q), _ptr(out), _stream(stream)), "kv_run")
+
+
+def kv_plan_free(plan) -> None:
+    capi.lib().kv_plan_free(plan)
+
+
+def kv_get_page_table(plan, stream_idx=0):
+    n, lpl = ctypes.c_int(), ctypes.c_int()
+    capi.check(capi.lib().kv_get_page_table(plan, stream_idx, None, 0, ctypes.byref(n),
+                                            ctypes.byref(lpl)), "kv_get_page_table")
+    buf = (ctypes.c_int * max(1, n.value))()
+    capi.check(capi.lib().kv_get_page_table(plan, stream_idx, buf, n.value, ctypes.byref(n),
+                                            ctypes.byref(lpl)), "kv_get_page_table")
+    return list(buf[: n.value]), lpl.value
+
+
+def kv_get_kv_tiles(plan, stream_idx=0):
+    n = ctypes.c_int()
+    capi.check(capi.lib().kv_get_kv_tiles(plan, stream_idx, None, None, None, 0, ctypes.byref(n)),
+               "kv_get_kv_tiles")
+    m = max(1, n.value)
+    row, lo, hi = (ctypes.c_int * m)(), (ctypes.c_int * m)(), (ctypes.c_int * m)()
+    capi.check(capi.lib().kv_get_kv_tiles(plan, stream_idx, row, lo, hi, n.value, ctypes.byref(n)),
+               "kv_get_kv_tiles")
+    return [(row[i], lo[i], hi[i]) for i in range(n.value)]
+
+
+def kv_plan_get_stats(plan) -> dict:
+    s = capi.kv_plan_stats()
+    capi.check(capi.lib().kv_plan_get_stats(plan, ctypes.byref(s)), "kv_plan_get_stats")
+    return {f: getattr(s, f) for f, _ in s._fields_}
+
+
+def kv_check_device(plan, stream=None) -> None:
+    capi.check(capi.lib().kv_check_device(plan, _stream(stream)), "kv_check_device")
+
+
+def kv_strerror(status) -> str:
+    return capi.strerror(status)
+
+
+def kv_last_error() -> str:
+    return capi.lib().kv_last_error().decode()
+
+
+def workspace_bytes(caches) -> int:
+    return kv_workspace_bytes([c.handle for c in caches])
+
+
+# ---------------------------------------------------------------- objects
+class PagedKVCache:
+    """One video stream's paged cache (all transformer blocks)."""
+
+    def __init__(self, max_pages, page_size, num_heads, head_dim, scale_frames=8, window=64,
+                 num_blocks=1, num_special=6, dtype="bf16", patch_pages=0):
+        self.dtype = dtype
+        code = KV_FP16 if dtype in ("fp16", "float16") or str(dtype) == "torch.float16" else KV_BF16
+        self.handle = kv_init(max_pages, page_size, num_heads, head_dim, scale_frames, window,
+                              num_blocks, num_special, code, patch_pages)
+        self.max_pages, self.page_size = max_pages, page_size
+        self.H, self.D, self.num_blocks, self.NS = num_heads, head_dim, num_blocks, num_special
+        self.T = page_size + num_special
+        self.pools = [None] * num_blocks
+
+    def __del__(self):
+        h = getattr(self, "handle", None)
+        if h:
+            kv_destroy(h)
+            self.handle = None
+
+    def pool_bytes(self) -> int:
+        return kv_pool_bytes(self.handle)
+
+    def bind_pool(self, block, pool, stream=None):
+        kv_bind_pool(self.handle, block, pool, stream)
+        self.pools[block] = pool
+
+    def allocate_pools(self, device="cuda", stream=None):
+        """Allocate each block's pool [max_pages, 2, page_size, H, D] with torch and bind it."""
+        import torch
+        dt = torch.float16 if self.dtype in ("fp16", "float16") else torch.bfloat16
+        for b in range(self.num_blocks):
+            pool = torch.empty((self.max_pages, 2, self.page_size, self.H, self.D), dtype=dt,
+                               device=device)
+            self.bind_pool(b, pool, stream)
+        return self.pools
+
+    def append_frame(self, block, k, v, stream=None):
+        kv_append_frame(self.handle, block, k, v, stream)
+
+    def evict_frames(self):
+        kv_evict_frames(self.handle)
+
+    def defer_eviction(self, on=True):
+        kv_defer_eviction(self.handle, on)
+
+    def commit_frame(self):
+        kv_commit_frame(self.handle)
+
+    def rollback_last_frame(self):
+        kv_rollback_last_frame(self.handle)
+
+    def get_stats(self) -> dict:
+        return kv_get_stats(self.handle)
+
+    def free_list(self) -> list[int]:
+        return kv_get_free_list(self.handle)
+
+    def reset(self):
+        kv_reset(self.handle)
+
+
+class Plan:
+    """One frame step's plan over a batch of caches; run() per block."""
+
+    def __init__(self, caches, workspace=None, tiles_per_split=0, stream=None):
+        self.caches = list(caches)
+        self.workspace = workspace
+        self.handle = kv_plan([c.handle for c in self.caches], tiles_per_split, workspace,
+                              stream=stream)
+        c0 = self.caches[0]
+        self.rows = sum(c.T for c in self.caches)
+        self.H, self.D, self.dtype = c0.H, c0.D, c0.dtype
+
+    def __del__(self):
+        h = getattr(self, "handle", None)
+        if h:
+            kv_plan_free(h)
+            self.handle = None
+
+    def run(self, block, q, out=None, stream=None):
+        if out is None:
+            import torch
+            out = torch.empty_like(q)
+        kv_run(self.handle, block, q, out, stream)
+        return out
+
+    def page_table(self, stream_idx=0):
+        return kv_get_page_table(self.handle, stream_idx)
+
+    def kv_tiles(self, stream_idx=0):
+        return kv_get_kv_tiles(self.handle, stream_idx)
+
+    def stats(self) -> dict:
+        return kv_plan_get_stats(self.handle)
+
+    def check_device(self, stream=None):
+        kv_check_device(self.handle, stream)

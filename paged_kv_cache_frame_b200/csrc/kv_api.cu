@@ -1,0 +1,405 @@
+// C-ABI of the paged KV cache (declared in include/kv.h): argument checks,
+// host page state, plan upload, TMA descriptors and kernel launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "../../include/kv.h"
+#include "kernels.h"
+#include "kv_state.h"
+
+struct kv_cache {
+  pkv::PageState st;
+  std::vector<void*> pools;
+  std::vector<CUtensorMap> maps;
+  std::vector<uint8_t> bound;
+};
+
+struct kv_plan {
+  std::vector<kv_cache*> caches;
+  std::vector<uint64_t> epochs;
+  pkv::HostPlan hp;
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+  int H = 0, D = 0, dtype = 0, total_T = 0;
+};
+
+namespace {
+
+thread_local std::string g_last;
+
+int fail(int code, const std::string& why) {
+  g_last = why;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* where) {
+  g_last = std::string(where) + ": " + cudaGetErrorString(e);
+  return KV_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 3-D view [rows][H][D] of a row-major [rows, H, D] tensor; boxes of
+// 128 rows x 1 head x 64 columns with 128-byte swizzle (the UMMA K-major /
+// MN-major canonical layout).
+int encode_rows_map(CUtensorMap* m, const void* base, int H, int D, long long rows, int dtype) {
+  auto fn = encode_fn();
+  if (!fn) return fail(KV_ERR_CUDA, "cuTensorMapEncodeTiled unavailable (no CUDA driver)");
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)pkv::kTile};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, dtype == KV_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(KV_ERR_CUDA, "cuTensorMapEncodeTiled failed: " + std::to_string((int)r));
+  return KV_OK;
+}
+
+int device_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* kv_strerror(int status) {
+  switch (status) {
+    case KV_OK: return "ok";
+    case KV_ERR_ARG: return "invalid argument";
+    case KV_ERR_CAPACITY: return "capacity exceeded";
+    case KV_ERR_ORDER: return "call out of order";
+    case KV_ERR_NO_PENDING: return "no pending (deferred) frame";
+    case KV_ERR_NOT_APPENDED: return "block not appended in this frame step";
+    case KV_ERR_EMPTY: return "cache holds no frame";
+    case KV_ERR_CUDA: return "CUDA error";
+    case KV_ERR_DEVICE_CHECK: return "device-side check failed";
+    case KV_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case KV_ERR_STALE_PLAN: return "plan is stale (cache state changed)";
+    default: return "unknown status";
+  }
+}
+
+const char* kv_last_error(void) { return g_last.c_str(); }
+
+int kv_init(kv_cache_t** out, int max_pages, int page_size, int num_heads, int head_dim, int scale_frames,
+            int window, int num_blocks, int num_special, int dtype, int patch_pages) {
+  if (!out) return fail(KV_ERR_ARG, "kv_init: out is NULL");
+  *out = nullptr;
+  if (head_dim % 8 != 0) return fail(KV_ERR_ARG, "kv_init: head_dim must be a multiple of 8");
+  pkv::Config c{max_pages, page_size, num_heads, head_dim, scale_frames, window, num_blocks, num_special, dtype,
+                patch_pages > 0 ? patch_pages : scale_frames + window + 1};
+  if (patch_pages < 0) return fail(KV_ERR_ARG, "kv_init: patch_pages < 0");
+  kv_cache* k = new kv_cache();
+  std::string why;
+  const int rc = k->st.init(c, &why);
+  if (rc != KV_OK) {
+    delete k;
+    return fail(rc, why);
+  }
+  k->pools.assign(num_blocks, nullptr);
+  k->maps.assign(num_blocks, CUtensorMap{});
+  k->bound.assign(num_blocks, 0);
+  *out = k;
+  return KV_OK;
+}
+
+void kv_destroy(kv_cache_t* c) { delete c; }
+
+int kv_reset(kv_cache_t* c) {
+  if (!c) return fail(KV_ERR_ARG, "kv_reset: NULL cache");
+  c->st.reset();
+  return KV_OK;
+}
+
+size_t kv_pool_bytes(const kv_cache_t* c) {
+  if (!c) return 0;
+  const pkv::Config& g = c->st.cfg;
+  return (size_t)g.max_pages * 2 * g.page_size * g.H * g.D * 2;
+}
+
+int kv_bind_pool(kv_cache_t* c, int block, void* pool, void* stream) {
+  if (!c || !pool) return fail(KV_ERR_ARG, "kv_bind_pool: NULL argument");
+  if (block < 0 || block >= c->st.cfg.B) return fail(KV_ERR_ARG, "kv_bind_pool: block out of range");
+  if (!aligned16(pool)) return fail(KV_ERR_ARG, "kv_bind_pool: pool not 16-byte aligned");
+  const pkv::Config& g = c->st.cfg;
+  cudaError_t e = cudaMemsetAsync(pool, 0, kv_pool_bytes(c), (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "kv_bind_pool: memset");
+  if (g.D % 64 == 0) {
+    const int rc = encode_rows_map(&c->maps[block], pool, g.H, g.D, (long long)g.max_pages * 2 * g.page_size,
+                                   g.dtype);
+    if (rc != KV_OK) return rc;
+  }
+  c->pools[block] = pool;
+  c->bound[block] = 1;
+  return KV_OK;
+}
+
+int kv_append_frame(kv_cache_t* c, int block, const void* k, const void* v, void* stream) {
+  if (!c) return fail(KV_ERR_ARG, "kv_append_frame: NULL cache");
+  if ((k == nullptr) != (v == nullptr)) return fail(KV_ERR_ARG, "kv_append_frame: k and v must both be set or both NULL");
+  const pkv::Config& g = c->st.cfg;
+  if (block < 0 || block >= g.B) return fail(KV_ERR_ARG, "kv_append_frame: block out of range");
+  if (k) {
+    if (!c->bound[block]) return fail(KV_ERR_ARG, "kv_append_frame: no pool bound for this block");
+    if (!aligned16(k) || !aligned16(v)) return fail(KV_ERR_ARG, "kv_append_frame: k/v not 16-byte aligned");
+  }
+  int page = -1, sp0 = 0;
+  std::string why;
+  const int rc = c->st.append(block, &page, &sp0, &why);
+  if (rc != KV_OK) return fail(rc, why);
+  if (!k) return KV_OK;
+  pkv::AppendArgs a;
+  a.k = k;
+  a.v = v;
+  a.pool = c->pools[block];
+  a.T = g.page_size + g.NS;
+  a.NS = g.NS;
+  a.page_size = g.page_size;
+  a.Np = g.Np;
+  a.max_pages = g.max_pages;
+  a.row_vecs = g.H * g.D * 2 / 16;
+  a.patch_page = page;
+  a.sp0 = sp0;
+  cudaError_t e = pkv::launch_append(a, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "kv_append_frame: scatter launch");
+  return KV_OK;
+}
+
+int kv_evict_frames(kv_cache_t* c) {
+  if (!c) return fail(KV_ERR_ARG, "kv_evict_frames: NULL cache");
+  return c->st.evict();
+}
+
+int kv_defer_eviction(kv_cache_t* c, int on) {
+  if (!c) return fail(KV_ERR_ARG, "kv_defer_eviction: NULL cache");
+  std::string why;
+  const int rc = c->st.set_defer(on, &why);
+  return rc == KV_OK ? rc : fail(rc, why);
+}
+
+int kv_commit_frame(kv_cache_t* c) {
+  if (!c) return fail(KV_ERR_ARG, "kv_commit_frame: NULL cache");
+  std::string why;
+  const int rc = c->st.commit(&why);
+  return rc == KV_OK ? rc : fail(rc, why);
+}
+
+int kv_rollback_last_frame(kv_cache_t* c) {
+  if (!c) return fail(KV_ERR_ARG, "kv_rollback_last_frame: NULL cache");
+  std::string why;
+  const int rc = c->st.rollback(&why);
+  return rc == KV_OK ? rc : fail(rc, why);
+}
+
+int kv_get_stats(const kv_cache_t* c, kv_stats* out) {
+  if (!c || !out) return fail(KV_ERR_ARG, "kv_get_stats: NULL argument");
+  const pkv::PageState& s = c->st;
+  const int pend = s.has_pending ? 1 : 0;
+  out->frame_count = s.committed + pend;
+  out->scale_pages = (int)s.scale_.size();
+  out->live_pages = (int)s.window_.size() + pend;
+  out->free_pages = (int)s.free_.size();
+  out->special_tokens = s.sp_len;
+  return KV_OK;
+}
+
+int kv_get_free_list(const kv_cache_t* c, int* ids, int cap, int* n) {
+  if (!c || !n || cap < 0 || (cap > 0 && !ids)) return fail(KV_ERR_ARG, "kv_get_free_list: bad argument");
+  const auto& f = c->st.free_;
+  *n = (int)f.size();
+  for (int i = 0; i < (int)f.size() && i < cap; ++i) ids[i] = f[i];
+  return KV_OK;
+}
+
+static int check_batch(kv_cache_t* const* caches, int n, std::vector<const pkv::PageState*>* st) {
+  if (!caches || n < 1) return fail(KV_ERR_ARG, "plan: no caches");
+  if (n > KV_MAX_STREAMS) return fail(KV_ERR_CAPACITY, "plan: more than KV_MAX_STREAMS streams");
+  for (int i = 0; i < n; ++i) {
+    if (!caches[i]) return fail(KV_ERR_ARG, "plan: NULL cache");
+    const pkv::Config& a = caches[0]->st.cfg;
+    const pkv::Config& b = caches[i]->st.cfg;
+    if (a.page_size != b.page_size || a.H != b.H || a.D != b.D || a.NS != b.NS || a.B != b.B || a.dtype != b.dtype)
+      return fail(KV_ERR_ARG, "plan: caches differ in page_size/H/D/NS/num_blocks/dtype");
+    st->push_back(&caches[i]->st);
+  }
+  return KV_OK;
+}
+
+size_t kv_workspace_bytes(kv_cache_t* const* caches, int n_streams) {
+  std::vector<const pkv::PageState*> st;
+  if (check_batch(caches, n_streams, &st) != KV_OK) return 0;
+  return pkv::workspace_layout(st).total;
+}
+
+int kv_plan(kv_plan_t** out, kv_cache_t* const* caches, int n_streams, int tiles_per_split, void* workspace,
+            size_t workspace_bytes, void* stream) {
+  if (!out) return fail(KV_ERR_ARG, "kv_plan: out is NULL");
+  *out = nullptr;
+  if (tiles_per_split < 0) return fail(KV_ERR_ARG, "kv_plan: tiles_per_split < 0");
+  std::vector<const pkv::PageState*> st;
+  int rc = check_batch(caches, n_streams, &st);
+  if (rc != KV_OK) return rc;
+  const pkv::Config& g = st[0]->cfg;
+  if (workspace) {
+    if (!aligned16(workspace)) return fail(KV_ERR_ARG, "kv_plan: workspace not 16-byte aligned");
+    if (workspace_bytes < pkv::workspace_layout(st).total)
+      return fail(KV_ERR_CAPACITY, "kv_plan: workspace smaller than kv_workspace_bytes()");
+  }
+  pkv::PlanInputs in;
+  in.num_sms = workspace ? device_sms() : 148;
+  in.ctas_per_sm = pkv::attention_ctas_per_sm(g.D);
+  in.tiles_per_split = tiles_per_split;
+  kv_plan_t* p = new kv_plan_t();
+  std::string why;
+  rc = pkv::build_plan(st, in, &p->hp, &why);
+  if (rc != KV_OK) {
+    delete p;
+    return fail(rc, why);
+  }
+  for (int i = 0; i < n_streams; ++i) {
+    p->caches.push_back(caches[i]);
+    p->epochs.push_back(caches[i]->st.epoch);
+    p->total_T += g.page_size + g.NS;
+  }
+  p->H = g.H;
+  p->D = g.D;
+  p->dtype = g.dtype;
+  p->ws = workspace;
+  p->ws_bytes = workspace_bytes;
+  if (workspace) {
+    cudaError_t e = pkv::upload_plan(workspace, p->hp.image.data(), p->hp.image.size(), (cudaStream_t)stream);
+    if (e != cudaSuccess) {
+      delete p;
+      return cuda_fail(e, "kv_plan: upload");
+    }
+  }
+  *out = p;
+  return KV_OK;
+}
+
+void kv_plan_free(kv_plan_t* plan) { delete plan; }
+
+int kv_run(const kv_plan_t* p, int block, const void* q, void* out, void* stream) {
+  if (!p || !q || !out) return fail(KV_ERR_ARG, "kv_run: NULL argument");
+  if (!p->ws) return fail(KV_ERR_ARG, "kv_run: host-only plan (built without a workspace)");
+  if (p->D != 64 && p->D != 128) return fail(KV_ERR_UNSUPPORTED, "kv_run: head_dim must be 64 or 128");
+  if (!aligned16(q) || !aligned16(out)) return fail(KV_ERR_ARG, "kv_run: q/out not 16-byte aligned");
+  const int B = p->caches[0]->st.cfg.B;
+  if (block < 0 || block >= B) return fail(KV_ERR_ARG, "kv_run: block out of range");
+  pkv::AttnMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  for (size_t r = 0; r < p->caches.size(); ++r) {
+    const kv_cache* c = p->caches[r];
+    if (c->st.epoch != p->epochs[r]) return fail(KV_ERR_STALE_PLAN, "kv_run: cache state changed after kv_plan");
+    if (!c->st.is_appended(block)) return fail(KV_ERR_NOT_APPENDED, "kv_run: block not appended in this step");
+    if (!c->bound[block]) return fail(KV_ERR_ARG, "kv_run: no pool bound for this block");
+    maps.kv[r] = c->maps[block];
+  }
+  int rc = encode_rows_map(&maps.q, q, p->H, p->D, p->total_T, p->dtype);
+  if (rc != KV_OK) return rc;
+  uint8_t* ws = static_cast<uint8_t*>(p->ws);
+  const pkv::KvPlanHeader& hd = p->hp.header;
+  pkv::AttnArgs a;
+  a.reqs = reinterpret_cast<const pkv::KvReq*>(ws + hd.off_reqs);
+  a.units = reinterpret_cast<const pkv::KvUnit*>(ws + hd.off_units);
+  a.tiles = reinterpret_cast<const pkv::KvTile*>(ws + hd.off_tiles);
+  a.part_o = reinterpret_cast<float*>(ws + hd.off_part_o);
+  a.part_lse = reinterpret_cast<float*>(ws + hd.off_part_lse);
+  a.out = out;
+  a.err = reinterpret_cast<uint32_t*>(ws);
+  a.H = p->H;
+  a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)p->D));
+  cudaError_t e = pkv::launch_attention(maps, a, p->D, p->dtype == KV_FP16, hd.n_units, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "kv_run: attention launch");
+  if (hd.n_merge > 0) {
+    pkv::MergeArgs m;
+    m.reqs = a.reqs;
+    m.items = reinterpret_cast<const pkv::KvMergeItem*>(ws + hd.off_merge);
+    m.part_o = a.part_o;
+    m.part_lse = a.part_lse;
+    m.out = out;
+    m.H = p->H;
+    m.n_items = hd.n_merge;
+    e = pkv::launch_merge(m, p->D, p->dtype == KV_FP16, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "kv_run: merge launch");
+  }
+  return KV_OK;
+}
+
+int kv_get_page_table(const kv_plan_t* p, int stream_idx, int* indices, int cap, int* n, int* last_page_len) {
+  if (!p || !n || !last_page_len || cap < 0 || (cap > 0 && !indices))
+    return fail(KV_ERR_ARG, "kv_get_page_table: bad argument");
+  if (stream_idx < 0 || stream_idx >= (int)p->hp.tables.size())
+    return fail(KV_ERR_ARG, "kv_get_page_table: stream out of range");
+  const auto& t = p->hp.tables[stream_idx];
+  *n = (int)t.size();
+  for (int i = 0; i < (int)t.size() && i < cap; ++i) indices[i] = t[i];
+  *last_page_len = p->hp.last_page_len[stream_idx];
+  return KV_OK;
+}
+
+int kv_get_kv_tiles(const kv_plan_t* p, int stream_idx, int* row, int* lo, int* hi, int cap, int* n) {
+  if (!p || !n || cap < 0 || (cap > 0 && (!row || !lo || !hi))) return fail(KV_ERR_ARG, "kv_get_kv_tiles: bad argument");
+  if (stream_idx < 0 || stream_idx >= (int)p->hp.reqs.size()) return fail(KV_ERR_ARG, "kv_get_kv_tiles: stream out of range");
+  int t0 = 0;
+  for (int r = 0; r < stream_idx; ++r) t0 += p->hp.reqs[r].n_tiles;
+  const int nt = p->hp.reqs[stream_idx].n_tiles;
+  *n = nt;
+  for (int i = 0; i < nt && i < cap; ++i) {
+    const pkv::KvTile& t = p->hp.tiles[t0 + i];
+    row[i] = t.row;
+    lo[i] = t.lo;
+    hi[i] = t.hi;
+  }
+  return KV_OK;
+}
+
+int kv_plan_get_stats(const kv_plan_t* p, kv_plan_stats* out) {
+  if (!p || !out) return fail(KV_ERR_ARG, "kv_plan_get_stats: NULL argument");
+  out->n_streams = (int)p->caches.size();
+  out->n_ctas = (int)p->hp.units.size();
+  out->n_split_units = p->hp.n_split_units;
+  out->n_kv_tiles = (int)p->hp.tiles.size();
+  out->tiles_per_cta = p->hp.max_tiles_per_cta;
+  out->visible_tokens = p->hp.visible;
+  return KV_OK;
+}
+
+int kv_check_device(const kv_plan_t* p, void* stream) {
+  if (!p || !p->ws) return fail(KV_ERR_ARG, "kv_check_device: plan without workspace");
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "kv_check_device: synchronize");
+  uint32_t w = 0;
+  e = cudaMemcpy(&w, p->ws, sizeof(w), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "kv_check_device: read error word");
+  if (w) return fail(KV_ERR_DEVICE_CHECK, "kernel error word " + std::to_string(w));
+  return KV_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,383 @@
+// Page state machine and planner (see kv_state.h).
+#include "kv_state.h"
+
+#include <algorithm>
+#include <cstring>
+#include <functional>
+
+#include "../../include/kv.h"
+
+namespace pkv {
+
+namespace {
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+inline int ceil_div(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
+}  // namespace
+
+int PageState::init(const Config& c, std::string* why) {
+  if (c.page_size < 1 || c.H < 1 || c.D < 1 || c.S < 0 || c.W < 0 || c.B < 1 || c.NS < 0 ||
+      c.max_pages < 1 || (c.dtype != KV_BF16 && c.dtype != KV_FP16) || c.Np < 1) {
+    *why = "kv_init: invalid argument";
+    return KV_ERR_ARG;
+  }
+  if ((long long)c.max_pages * 2 * c.page_size > 0x7fffffffLL) {
+    *why = "kv_init: pool row count exceeds int32";
+    return KV_ERR_ARG;
+  }
+  if (c.max_pages < c.Np + (c.NS > 0 ? 1 : 0)) {
+    *why = "kv_init: max_pages must leave at least one special page after the patch pages";
+    return KV_ERR_CAPACITY;
+  }
+  cfg = c;
+  reset();
+  return KV_OK;
+}
+
+void PageState::reset() {
+  free_.clear();
+  for (int p = cfg.Np - 1; p >= 0; --p) free_.push_back(p);
+  scale_.clear();
+  window_.clear();
+  has_pending = false;
+  sp_len = 0;
+  committed = 0;
+  next_frame = 0;
+  defer = false;
+  step_open = false;
+  appended.assign(cfg.B, 0);
+  n_appended = 0;
+  step_page = -1;
+  step_sp0 = 0;
+  ++epoch;
+}
+
+void PageState::commit_frame(const FramePage& fp) {
+  if ((int)scale_.size() < cfg.S)
+    scale_.push_back(fp);
+  else
+    window_.push_back(fp);
+  ++committed;
+}
+
+int PageState::append(int block, int* page, int* sp0, std::string* why) {
+  if (block < 0 || block >= cfg.B) {
+    *why = "append: block out of range";
+    return KV_ERR_ARG;
+  }
+  const bool new_step = !step_open || n_appended == cfg.B;
+  if (new_step) {
+    if (has_pending) {
+      *why = "append: the deferred frame of the previous step must be committed or rolled back";
+      return KV_ERR_ORDER;
+    }
+    if (free_.empty()) {
+      *why = "append: no free patch page (patch_pages too small for S + W)";
+      return KV_ERR_CAPACITY;
+    }
+    if (sp_len + cfg.NS > special_capacity()) {
+      *why = "append: special stream full (raise max_pages)";
+      return KV_ERR_CAPACITY;
+    }
+    const int pg = free_.back();
+    free_.pop_back();
+    step_sp0 = sp_len;
+    sp_len += cfg.NS;
+    step_page = pg;
+    const FramePage fp{next_frame++, pg};
+    if (defer) {
+      has_pending = true;
+      pending_ = fp;
+    } else {
+      commit_frame(fp);
+    }
+    step_open = true;
+    std::fill(appended.begin(), appended.end(), 0);
+    n_appended = 0;
+    ++epoch;
+  } else if (appended[block]) {
+    *why = "append: block already appended in this frame step";
+    return KV_ERR_ORDER;
+  }
+  appended[block] = 1;
+  ++n_appended;
+  *page = step_page;
+  *sp0 = step_sp0;
+  return KV_OK;
+}
+
+int PageState::evict() {
+  if (defer) return KV_OK;
+  bool any = false;
+  while ((int)window_.size() > cfg.W) {
+    free_.push_back(window_.front().page);
+    window_.pop_front();
+    any = true;
+  }
+  if (any) ++epoch;
+  return KV_OK;
+}
+
+int PageState::set_defer(int on, std::string* why) {
+  if (!on && has_pending) {
+    *why = "defer_eviction(0): a frame is pending; commit or roll it back";
+    return KV_ERR_ORDER;
+  }
+  defer = on != 0;
+  return KV_OK;
+}
+
+int PageState::commit(std::string* why) {
+  if (!has_pending) {
+    *why = "commit: no deferred frame";
+    return KV_ERR_NO_PENDING;
+  }
+  if (n_appended != cfg.B) {
+    *why = "commit: not every block of the pending frame has been appended";
+    return KV_ERR_ORDER;
+  }
+  has_pending = false;
+  defer = false;
+  commit_frame(pending_);
+  ++epoch;
+  evict();
+  return KV_OK;
+}
+
+int PageState::rollback(std::string* why) {
+  if (!has_pending) {
+    *why = "rollback: no deferred frame";
+    return KV_ERR_NO_PENDING;
+  }
+  free_.push_back(pending_.page);
+  sp_len -= cfg.NS;
+  --next_frame;
+  has_pending = false;
+  defer = false;
+  step_open = false;
+  std::fill(appended.begin(), appended.end(), 0);
+  n_appended = 0;
+  step_page = -1;
+  ++epoch;
+  return KV_OK;
+}
+
+int PageState::page_table(std::vector<int>* idx, int* last_page_len) const {
+  if (committed == 0 && !has_pending) return KV_ERR_EMPTY;
+  idx->clear();
+  for (const auto& fp : scale_) idx->push_back(fp.page);
+  for (const auto& fp : window_) idx->push_back(fp.page);
+  if (has_pending) idx->push_back(pending_.page);
+  const int ps = cfg.page_size;
+  const int k = ceil_div(sp_len, ps);
+  for (int i = 0; i < k; ++i) idx->push_back(cfg.Np + i);
+  *last_page_len = k ? sp_len - ps * (k - 1) : ps;
+  return KV_OK;
+}
+
+long long PageState::visible_tokens() const {
+  const long long patch = (long long)scale_.size() + (long long)window_.size() + (has_pending ? 1 : 0);
+  return patch * cfg.page_size + sp_len;
+}
+
+void build_tiles(const std::vector<int>& table, int last_page_len, int page_size,
+                 std::vector<KvTile>* tiles) {
+  const int n = (int)table.size();
+  for (int i = 0; i < n; ++i) {
+    const int count = (i == n - 1) ? last_page_len : page_size;
+    const int base = table[i] * 2 * page_size;
+    for (int t0 = 0; t0 < count; t0 += kTile) {
+      const int nn = std::min(kTile, count - t0);
+      KvTile t;
+      if (nn == kTile) {
+        t.row = base + t0; t.lo = 0; t.hi = kTile;
+      } else if (count >= kTile) {
+        // ragged end of a long page: anchor the box at the page's last valid
+        // row so no row outside the page is read; the first rows repeat the
+        // previous tile and are masked
+        t.row = base + count - kTile; t.lo = (int16_t)(kTile - nn); t.hi = kTile;
+      } else {
+        // a page shorter than one tile: the box runs past it, rows >= count masked
+        t.row = base; t.lo = 0; t.hi = (int16_t)nn;
+      }
+      tiles->push_back(t);
+    }
+  }
+}
+
+static size_t header_bytes() { return align_up(sizeof(KvPlanHeader), 256); }
+
+WorkspaceLayout workspace_layout(const std::vector<const PageState*>& st) {
+  WorkspaceLayout L{};
+  size_t units_base = 0, tiles_cap = 0;
+  int D = 0;
+  for (const PageState* s : st) {
+    const Config& c = s->cfg;
+    const int T = c.page_size + c.NS;
+    units_base += (size_t)c.H * ceil_div(T, kTile);
+    tiles_cap += (size_t)c.max_pages * ceil_div(c.page_size, kTile);
+    D = c.D;
+  }
+  L.slot_cap = units_base + kMaxTargetCtas;
+  const size_t units_cap = units_base + L.slot_cap;
+  size_t off = header_bytes();
+  off += align_up(st.size() * sizeof(KvReq), 16);
+  off += align_up(units_cap * sizeof(KvUnit), 16);
+  off += align_up(units_base * sizeof(KvMergeItem), 16);
+  off += align_up(tiles_cap * sizeof(KvTile), 16);
+  L.table_bytes = align_up(off, 256);
+  L.off_part_o = L.table_bytes;
+  L.off_part_lse = align_up(L.off_part_o + L.slot_cap * kTile * (size_t)D * 4, 256);
+  L.total = align_up(L.off_part_lse + L.slot_cap * kTile * 4, 256);
+  return L;
+}
+
+int build_plan(const std::vector<const PageState*>& st, const PlanInputs& in, HostPlan* out,
+               std::string* why) {
+  HostPlan& P = *out;
+  P = HostPlan();
+  const int n_req = (int)st.size();
+  const Config& c0 = st[0]->cfg;
+  const int H = c0.H;
+  int q_row0 = 0;
+  std::vector<int> tile0(n_req);
+  for (int r = 0; r < n_req; ++r) {
+    const PageState* s = st[r];
+    std::vector<int> table;
+    int lpl = 0;
+    const int rc = s->page_table(&table, &lpl);
+    if (rc != KV_OK) {
+      *why = "plan: a stream has no frame yet";
+      return rc;
+    }
+    tile0[r] = (int)P.tiles.size();
+    build_tiles(table, lpl, s->cfg.page_size, &P.tiles);
+    KvReq rq;
+    rq.q_row0 = q_row0;
+    rq.T = s->cfg.page_size + s->cfg.NS;
+    rq.page_size = s->cfg.page_size;
+    rq.n_tiles = (int)P.tiles.size() - tile0[r];
+    q_row0 += rq.T;
+    P.reqs.push_back(rq);
+    P.tables.push_back(table);
+    P.last_page_len.push_back(lpl);
+    P.visible += s->visible_tokens();
+  }
+
+  // Work units: (request, head, q-tile), each split into chunks of at most L
+  // K/V tiles so that the launch fills the machine.
+  int n_base = 0, max_n = 0;
+  for (int r = 0; r < n_req; ++r) {
+    const int qt = ceil_div(P.reqs[r].T, kTile);
+    n_base += qt * H;
+    max_n = std::max(max_n, P.reqs[r].n_tiles);
+  }
+  const int target = std::max(1, in.num_sms * in.ctas_per_sm);
+  int L;
+  if (in.tiles_per_split > 0) {
+    L = in.tiles_per_split;
+  } else {
+    // Pick the chunk size whose schedule finishes first when CTAs are handed
+    // to `target` slots greedily, longest first (what the block scheduler
+    // does); a CTA costs its tiles plus a fixed prologue/epilogue.
+    std::vector<int> lens;
+    for (int r = 0; r < n_req; ++r)
+      for (int k = 0; k < ceil_div(P.reqs[r].T, kTile) * H; ++k) lens.push_back(P.reqs[r].n_tiles);
+    L = max_n;
+    double best = 1e300;
+    for (int c = 1; c <= 32; ++c) {
+      const int cand = std::max(1, ceil_div(max_n, c));
+      if (c > 1 && cand == ceil_div(max_n, c - 1)) continue;
+      std::vector<double> costs;
+      for (int n : lens) {
+        const int ch = std::max(1, ceil_div(n, cand));
+        for (int k = 0; k < ch; ++k)
+          costs.push_back((double)((long long)(k + 1) * n / ch - (long long)k * n / ch) + 2.0 + (ch > 1 ? 1.0 : 0.0));
+      }
+      if ((int)costs.size() > target + n_base) break;
+      std::sort(costs.begin(), costs.end(), std::greater<double>());
+      std::vector<double> slot(std::min<size_t>(target, costs.size()), 0.0);
+      for (double x : costs) {
+        auto it = std::min_element(slot.begin(), slot.end());
+        *it += x;
+      }
+      const double makespan = *std::max_element(slot.begin(), slot.end());
+      if (makespan < best * 0.995) {
+        best = makespan;
+        L = cand;
+      }
+      if (cand <= 2) break;
+    }
+  }
+  const WorkspaceLayout WL = workspace_layout(st);
+  int n_slots = 0;
+  for (int r = 0; r < n_req; ++r) {
+    const int nt = P.reqs[r].n_tiles;
+    const int qtiles = ceil_div(P.reqs[r].T, kTile);
+    const int chunks = std::max(1, ceil_div(nt, L));
+    for (int h = 0; h < H; ++h) {
+      for (int qt = 0; qt < qtiles; ++qt) {
+        int slot0 = -1;
+        if (chunks > 1) {
+          slot0 = n_slots;
+          n_slots += chunks;
+          KvMergeItem m{};
+          m.req = (int16_t)r; m.head = (int16_t)h; m.qtile = (int16_t)qt;
+          m.n = (int16_t)chunks; m.slot0 = slot0;
+          P.merges.push_back(m);
+          ++P.n_split_units;
+        }
+        for (int k = 0; k < chunks; ++k) {
+          KvUnit u{};
+          u.req = (int16_t)r; u.head = (int16_t)h; u.qtile = (int16_t)qt;
+          u.tile_begin = tile0[r] + (int)((long long)k * nt / chunks);
+          u.tile_end = tile0[r] + (int)((long long)(k + 1) * nt / chunks);
+          u.slot = chunks > 1 ? slot0 + k : -1;
+          P.max_tiles_per_cta = std::max(P.max_tiles_per_cta, u.tile_end - u.tile_begin);
+          P.units.push_back(u);
+        }
+      }
+    }
+  }
+  if ((size_t)n_slots > WL.slot_cap || P.units.size() > 0x7fffffff) {
+    *why = "plan: split schedule exceeds the workspace's partial slots";
+    return KV_ERR_CAPACITY;
+  }
+  // Launch order: the chunks of one (request, head) sit next to each other so
+  // that co-resident CTAs share K/V tiles in L2.
+  std::stable_sort(P.units.begin(), P.units.end(), [](const KvUnit& a, const KvUnit& b) {
+    if (a.req != b.req) return a.req < b.req;
+    if (a.head != b.head) return a.head < b.head;
+    if (a.tile_begin != b.tile_begin) return a.tile_begin < b.tile_begin;
+    return a.qtile < b.qtile;
+  });
+
+  // Serialise.
+  KvPlanHeader& Hd = P.header;
+  std::memset(&Hd, 0, sizeof(Hd));
+  Hd.n_reqs = n_req;
+  Hd.n_units = (int)P.units.size();
+  Hd.n_merge = (int)P.merges.size();
+  Hd.n_tiles = (int)P.tiles.size();
+  size_t off = header_bytes();
+  Hd.off_reqs = (int)off;   off += align_up(P.reqs.size() * sizeof(KvReq), 16);
+  Hd.off_units = (int)off;  off += align_up(P.units.size() * sizeof(KvUnit), 16);
+  Hd.off_merge = (int)off;  off += align_up(P.merges.size() * sizeof(KvMergeItem), 16);
+  Hd.off_tiles = (int)off;  off += align_up(P.tiles.size() * sizeof(KvTile), 16);
+  Hd.upload_bytes = (int)off;
+  Hd.off_part_o = (int64_t)WL.off_part_o;
+  Hd.off_part_lse = (int64_t)WL.off_part_lse;
+  if (off > WL.table_bytes) {
+    *why = "plan: tables exceed the workspace layout";
+    return KV_ERR_CAPACITY;
+  }
+  P.image.assign(off, 0);
+  std::memcpy(P.image.data(), &Hd, sizeof(Hd));
+  std::memcpy(P.image.data() + Hd.off_reqs, P.reqs.data(), P.reqs.size() * sizeof(KvReq));
+  std::memcpy(P.image.data() + Hd.off_units, P.units.data(), P.units.size() * sizeof(KvUnit));
+  if (!P.merges.empty())
+    std::memcpy(P.image.data() + Hd.off_merge, P.merges.data(), P.merges.size() * sizeof(KvMergeItem));
+  std::memcpy(P.image.data() + Hd.off_tiles, P.tiles.data(), P.tiles.size() * sizeof(KvTile));
+  return KV_OK;
+}
+
+}  // namespace pkv

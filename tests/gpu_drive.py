@@ -1,0 +1,90 @@
+"""Drives streams of frames through the CUDA library and the oracle in lockstep
+(used by the GPU parity tests and by `__graft_entry__.smoke`)."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import workload
+from oracle.stream import StreamOracle, bits16
+
+MAX_ABS = 2e-2    # attention tolerance on unit-variance inputs (bf16/fp16 in, fp32 accumulate)
+MEAN_ABS = 2e-3
+
+
+class Frames:
+    """Seeded frames of one stream/block, drawn once and kept on the CPU."""
+
+    def __init__(self, wl, seed, stream=0, block=0):
+        self.wl, self.seed, self.stream, self.block = wl, seed, stream, block
+        self.cache = {}
+
+    def get(self, f):
+        if f not in self.cache:
+            self.cache = {k: v for k, v in self.cache.items() if k >= f - 1}
+            self.cache[f] = workload.frame_qkv(self.wl, self.seed, f, self.block, self.stream)
+        return self.cache[f]
+
+    def bits(self, f):
+        return tuple(bits16(x) for x in self.get(f))
+
+
+def errors(out: torch.Tensor, want: np.ndarray):
+    got = out.float().cpu().double().numpy()
+    d = np.abs(got - want)
+    return float(d.max()), float(d.mean())
+
+
+def assert_close(out, want, what=""):
+    mx, mean = errors(out, want)
+    assert np.isfinite(mx), f"{what}: non-finite output"
+    assert mx <= MAX_ABS and mean <= MEAN_ABS, f"{what}: max {mx:.3e} mean {mean:.3e}"
+    return mx, mean
+
+
+def new_cache(pkv, wl, num_blocks=1, patch_pages=0):
+    max_pages = (patch_pages or wl.patch_pages) + wl.special_pages
+    c = pkv.PagedKVCache(max_pages, wl.page_size, wl.H, wl.D, wl.S, wl.W, num_blocks=num_blocks,
+                         num_special=wl.NS, dtype=wl.dtype, patch_pages=patch_pages)
+    c.allocate_pools("cuda")
+    return c
+
+
+def workspace(pkv, caches):
+    return torch.empty(pkv.workspace_bytes(caches), dtype=torch.uint8, device="cuda")
+
+
+def run_stream(pkv, wl, seed, n_frames, check, rows=None, defer=None, keep=None,
+               tiles_per_split=0, patch_pages=0, collect=None):
+    """Append frames 0..n_frames-1 of block 0; at frames in `check`, plan + run
+    and compare the chosen query rows with the oracle. defer[f] / keep[f]:
+    frame f is appended with eviction deferred and then committed (keep) or
+    rolled back. Returns {frame: (max_err, mean_err)}."""
+    fr = Frames(wl, seed)
+    cache = new_cache(pkv, wl, patch_pages=patch_pages)
+    ws = workspace(pkv, [cache])
+    so = StreamOracle(wl.S, wl.W, wl.NS, wl.P, wl.dtype, fr.bits)
+    res = {}
+    for f in range(n_frames):
+        q, k, v = (x.cuda() for x in fr.get(f))
+        d = bool(defer[f]) if defer is not None else False
+        cache.defer_eviction(d)
+        cache.append_frame(0, k, v)
+        cache.evict_frames()
+        so.begin_frame(f, d)
+        if f in check:
+            plan = pkv.Plan([cache], ws, tiles_per_split=tiles_per_split)
+            out = plan.run(0, q)
+            plan.check_device()
+            sel = slice(None) if rows is None else torch.as_tensor(rows)
+            res[f] = assert_close(out[sel], so.expected(rows), f"frame {f}")
+            if collect is not None:
+                collect[f] = out.clone()
+        if d:
+            if keep is None or keep[f]:
+                cache.commit_frame()
+            else:
+                cache.rollback_last_frame()
+            so.end_frame(keep is None or bool(keep[f]))
+        assert cache.get_stats()["special_tokens"] == len(so.sim.SP)
+    return res

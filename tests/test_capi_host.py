@@ -1,0 +1,315 @@
+"""Host-side tests of the C-ABI library (no GPU, no kernel launches).
+
+The library loads without a GPU; the page state machine, the visible page
+table, last_page_len, the free list, the statistics and the K/V tiling are
+compared bit for bit with the oracle's page-level model. Appends pass NULL
+k/v (state only) and plans are host-only (no workspace).
+"""
+import json
+import math
+import os
+import re
+
+import pytest
+from hypothesis import given, settings, strategies as st
+
+from oracle import PageModel, OracleError
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="session")
+def pkv():
+    from paged_kv_cache_frame_b200 import build
+    build.build()
+    import paged_kv_cache_frame_b200 as m
+    return m
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "kv.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w\s\*]*?\b(kv_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_library_exports_every_declared_function(pkv):
+    import ctypes
+    names = declared_functions()
+    assert len(names) >= 20
+    lib = ctypes.CDLL(pkv.capi.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(pkv.capi.SIGNATURES)
+
+
+def test_strerror_covers_codes(pkv):
+    for code in range(0, -11, -1):
+        assert pkv.kv_strerror(code) != "unknown status"
+    assert pkv.kv_strerror(-99) == "unknown status"
+
+
+def mk(pkv, S, W, ps, max_pages, NS=6, B=1, patch_pages=0, H=2, D=64):
+    return pkv.kv_init(max_pages, ps, H, D, S, W, B, NS, pkv.KV_BF16, patch_pages)
+
+
+def step(pkv, c, B=1):
+    for b in range(B):
+        pkv.kv_append_frame(c, b, None, None)
+        pkv.kv_evict_frames(c)
+
+
+def table(pkv, caches):
+    p = pkv.kv_plan(caches)
+    try:
+        return [pkv.kv_get_page_table(p, i) for i in range(len(caches))]
+    finally:
+        pkv.kv_plan_free(p)
+
+
+def test_stats_example_through_capi(pkv):
+    g = json.load(open(os.path.join(ROOT, "tests", "golden", "cache_stats_12_frames.json")))
+    c = g["config"]
+    h = mk(pkv, c["scale_frames"], c["sliding_window"], c["page_size"], g["patch_pages"] + 2,
+           NS=c["num_special"], patch_pages=g["patch_pages"])
+    for _ in range(c["frames"]):
+        step(pkv, h)
+    assert pkv.kv_get_stats(h) == g["expected"]
+    pkv.kv_destroy(h)
+
+
+def test_interval_keyframes_through_capi(pkv):
+    g = json.load(open(os.path.join(ROOT, "tests", "golden", "keyframe_interval_200.json")))
+    h = mk(pkv, 8, g["sliding_window"], 256, 73 + 4)
+    for t in range(g["frames"]):
+        if t % g["keyframe_interval"] == 0:
+            step(pkv, h)
+        else:
+            pkv.kv_defer_eviction(h, True)
+            step(pkv, h)
+            pkv.kv_rollback_last_frame(h)
+    s = pkv.kv_get_stats(h)
+    assert s["frame_count"] == g["expected_keyframes"]
+    assert s["special_tokens"] == g["special_tokens_per_frame"] * g["expected_keyframes"]
+
+
+@pytest.mark.parametrize("ps,n,pages,lpl", [(16, 12, 5, 8), (256, 320, 8, 128), (999, 1000, 7, 6)])
+def test_special_stream_sizes_through_capi(pkv, ps, n, pages, lpl):
+    h = mk(pkv, 8, 64, ps, 73 + pages)
+    for _ in range(n):
+        step(pkv, h)
+    (tbl, last), = table(pkv, [h])
+    assert len([p for p in tbl if p >= 73]) == pages and last == lpl
+    assert len(tbl) == min(n, 72) + pages
+
+
+def test_error_codes(pkv):
+    E = pkv.capi
+    h = mk(pkv, 1, 1, 16, 4, B=2)          # 3 patch pages, 1 special page of 16 tokens
+    with pytest.raises(pkv.KVError) as e:
+        pkv.kv_plan([h])
+    assert e.value.code == E.KV_ERR_EMPTY
+    with pytest.raises(pkv.KVError) as e:
+        pkv.kv_commit_frame(h)
+    assert e.value.code == E.KV_ERR_NO_PENDING
+    with pytest.raises(pkv.KVError) as e:
+        pkv.kv_rollback_last_frame(h)
+    assert e.value.code == E.KV_ERR_NO_PENDING
+    pkv.kv_append_frame(h, 0, None, None)
+    with pytest.raises(pkv.KVError) as e:
+        pkv.kv_append_frame(h, 0, None, None)          # block 0 twice in one step
+    assert e.value.code == E.KV_ERR_ORDER
+    with pytest.raises(pkv.KVError) as e:
+        pkv.kv_append_frame(h, 2, None, None)
+    assert e.value.code == E.KV_ERR_ARG
+    pkv.kv_append_frame(h, 1, None, None)
+    pkv.kv_evict_frames(h)
+    step(pkv, h, B=2)                                  # 12 special tokens used
+    with pytest.raises(pkv.KVError) as e:
+        pkv.kv_append_frame(h, 0, None, None)          # 18 > 16: special stream full
+    assert e.value.code == E.KV_ERR_CAPACITY
+    assert pkv.kv_get_stats(h)["special_tokens"] == 12  # unchanged by the failed append
+    # defer: turning it off while a frame is pending is out of order
+    h2 = mk(pkv, 1, 1, 16, 8, B=2)
+    pkv.kv_defer_eviction(h2, True)
+    pkv.kv_append_frame(h2, 0, None, None)
+    with pytest.raises(pkv.KVError) as e:
+        pkv.kv_defer_eviction(h2, False)
+    assert e.value.code == E.KV_ERR_ORDER
+    with pytest.raises(pkv.KVError) as e:
+        pkv.kv_commit_frame(h2)                        # block 1 not yet appended
+    assert e.value.code == E.KV_ERR_ORDER
+    pkv.kv_append_frame(h2, 1, None, None)
+    pkv.kv_commit_frame(h2)
+    # kv_init arguments
+    with pytest.raises(pkv.KVError) as e:
+        mk(pkv, 2, 2, 16, 5)                           # needs 5 patch + 1 special page
+    assert e.value.code == E.KV_ERR_CAPACITY
+    with pytest.raises(pkv.KVError) as e:
+        pkv.kv_init(10, 0, 2, 64, 1, 1, 1, 6, 0, 0)
+    assert e.value.code == E.KV_ERR_ARG
+    # a host-only plan cannot run
+    p = pkv.kv_plan([h2])
+    with pytest.raises(pkv.KVError) as e:
+        pkv.kv_run(p, 0, 16, 16)
+    assert e.value.code == E.KV_ERR_ARG
+    pkv.kv_plan_free(p)
+    for x in (h, h2):
+        pkv.kv_destroy(x)
+
+
+def test_frame_step_rule_multi_block(pkv):
+    h = mk(pkv, 2, 2, 16, 10, B=3)
+    pkv.kv_append_frame(h, 1, None, None)              # any block may open the step
+    assert pkv.kv_get_stats(h)["frame_count"] == 1
+    pkv.kv_append_frame(h, 0, None, None)
+    pkv.kv_append_frame(h, 2, None, None)
+    assert pkv.kv_get_stats(h)["frame_count"] == 1
+    pkv.kv_append_frame(h, 0, None, None)              # all appended -> new step
+    assert pkv.kv_get_stats(h)["frame_count"] == 2
+    pkv.kv_destroy(h)
+
+
+OPS = st.lists(st.sampled_from(["key", "key", "key", "defer_keep", "defer_drop", "evict",
+                                "bad_commit", "bad_rollback"]), min_size=1, max_size=50)
+
+
+@settings(max_examples=120, deadline=None)
+@given(ops=OPS, S=st.integers(0, 3), W=st.integers(0, 4), ps=st.sampled_from([1, 5, 16, 130]),
+       B=st.integers(1, 3))
+def test_state_machine_bit_exact_vs_oracle(pkv, ops, S, W, ps, B):
+    NS = 6
+    max_pages = S + W + 1 + (NS * 60) // ps + 2
+    m = PageModel(S, W, ps, max_pages, NS=NS)
+    h = mk(pkv, S, W, ps, max_pages, B=B)
+    E = pkv.capi
+    try:
+        f = 0
+        for op in ops:
+            if op == "evict":
+                m.evict(); pkv.kv_evict_frames(h)
+            elif op == "key":
+                m.set_defer(False); pkv.kv_defer_eviction(h, False)
+                m.append(f); m.evict()
+                step(pkv, h, B)
+                f += 1
+            elif op in ("defer_keep", "defer_drop"):
+                m.set_defer(True); pkv.kv_defer_eviction(h, True)
+                m.append(f); m.evict()
+                step(pkv, h, B)
+                assert table(pkv, [h])[0] == m.page_table()
+                if op == "defer_keep":
+                    m.commit(); pkv.kv_commit_frame(h)
+                else:
+                    m.rollback(); pkv.kv_rollback_last_frame(h)
+                f += 1
+            elif op == "bad_commit":
+                with pytest.raises(OracleError):
+                    m.commit()
+                with pytest.raises(pkv.KVError) as e:
+                    pkv.kv_commit_frame(h)
+                assert e.value.code == E.KV_ERR_NO_PENDING
+            elif op == "bad_rollback":
+                with pytest.raises(OracleError):
+                    m.rollback()
+                with pytest.raises(pkv.KVError) as e:
+                    pkv.kv_rollback_last_frame(h)
+                assert e.value.code == E.KV_ERR_NO_PENDING
+            assert pkv.kv_get_free_list(h) == m.free
+            assert pkv.kv_get_stats(h) == m.stats()
+            if m.committed or m.pending is not None:
+                assert table(pkv, [h])[0] == m.page_table()
+    finally:
+        pkv.kv_destroy(h)
+
+
+@settings(max_examples=60, deadline=None)
+@given(n=st.integers(0, 80), S=st.integers(0, 4), W=st.integers(0, 5))
+def test_rollback_restores_state_through_capi(pkv, n, S, W):
+    h = mk(pkv, S, W, 7, S + W + 1 + 80, B=2)
+    for _ in range(n):
+        step(pkv, h, 2)
+    before = (pkv.kv_get_free_list(h), pkv.kv_get_stats(h), table(pkv, [h]) if n else None)
+    pkv.kv_defer_eviction(h, True)
+    step(pkv, h, 2)
+    pkv.kv_rollback_last_frame(h)
+    after = (pkv.kv_get_free_list(h), pkv.kv_get_stats(h), table(pkv, [h]) if n else None)
+    assert before == after
+    pkv.kv_destroy(h)
+
+
+def tile_cover(tiles, ps):
+    """(page, token) pairs the tiles mark visible, with multiplicity."""
+    out = []
+    for row, lo, hi in tiles:
+        for col in range(lo, hi):
+            r = row + col
+            page, rem = divmod(r, 2 * ps)
+            assert rem < ps, "a visible column must be a K row of its page"
+            out.append((page, rem))
+    return out
+
+
+@pytest.mark.parametrize("ps,n", [(16, 12), (256, 320), (999, 30), (130, 40), (128, 9), (64, 100)])
+def test_kv_tiles_cover_visible_tokens_exactly_once(pkv, ps, n):
+    S, W = 8, 64
+    pages = math.ceil(6 * n / ps) + 1
+    h = mk(pkv, S, W, ps, 73 + pages)
+    m = PageModel(S, W, ps, 73 + pages)
+    for f in range(n):
+        step(pkv, h)
+        m.append(f); m.evict()
+    p = pkv.kv_plan([h])
+    tiles = pkv.kv_get_kv_tiles(p)
+    tbl, last = m.page_table()
+    want = []
+    for i, pg in enumerate(tbl):
+        cnt = last if i == len(tbl) - 1 else ps
+        want += [(pg, t) for t in range(cnt)]
+    got = tile_cover(tiles, ps)
+    assert sorted(got) == sorted(want)
+    for row, lo, hi in tiles:
+        assert 0 <= lo < hi <= 128
+        if ps >= 128:   # long pages: a box never leaves its page's K rows
+            assert (row % (2 * ps)) + 128 <= ps
+    s = pkv.kv_plan_get_stats(p)
+    assert s["visible_tokens"] == m.visible_token_count()
+    assert s["n_kv_tiles"] == len(tiles)
+    pkv.kv_plan_free(p)
+
+
+def test_split_schedule_covers_each_unit(pkv):
+    """Host plan for the 224x224 shape at frame 320: 159 tiles per head,
+    16 heads x 3 query tiles; a forced split of 10 tiles per CTA."""
+    h = pkv.kv_init(81, 256, 16, 64, 8, 64, 1, 6, pkv.KV_BF16, 0)
+    for _ in range(320):
+        step(pkv, h)
+    p = pkv.kv_plan([h], tiles_per_split=10)
+    s = pkv.kv_plan_get_stats(p)
+    assert s["n_kv_tiles"] == 159
+    assert s["visible_tokens"] == 72 * 256 + 6 * 320
+    assert s["n_split_units"] == 48
+    assert s["n_ctas"] == 48 * 16           # ceil(159 / 10) = 16 chunks each
+    assert s["tiles_per_cta"] <= 10
+    pkv.kv_plan_free(p)
+    p = pkv.kv_plan([h])                   # automatic: fills 148 SMs
+    s = pkv.kv_plan_get_stats(p)
+    assert 100 <= s["n_ctas"] <= 2 * 148 + 48
+    pkv.kv_plan_free(p)
+    pkv.kv_destroy(h)
+
+
+def test_workspace_bytes_and_batch_checks(pkv):
+    a = pkv.kv_init(81, 256, 8, 128, 8, 64, 2, 6, pkv.KV_FP16, 0)
+    b = pkv.kv_init(81, 256, 8, 128, 8, 64, 2, 6, pkv.KV_FP16, 0)
+    c = pkv.kv_init(81, 256, 8, 64, 8, 64, 2, 6, pkv.KV_FP16, 0)
+    assert pkv.kv_workspace_bytes([a, b]) > pkv.kv_workspace_bytes([a]) > 0
+    assert pkv.kv_workspace_bytes([a, c]) == 0        # mixed head_dim
+    for x in (a, b):
+        step(pkv, x, 2)
+    p = pkv.kv_plan([a, b])
+    assert pkv.kv_plan_get_stats(p)["n_streams"] == 2
+    pkv.kv_plan_free(p)
+    with pytest.raises(pkv.KVError):
+        pkv.kv_plan([a, c])
+    for x in (a, b, c):
+        pkv.kv_destroy(x)

@@ -1,0 +1,243 @@
+"""GPU parity: the CUDA path through the C-ABI against the CPU oracle.
+
+Bit-exact: pool contents after every append (scatter), page tables.
+Attention: max |err| <= 2e-2 and mean |err| <= 2e-3 against the float64
+oracle on unit-variance bf16/fp16 inputs.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import workload
+from oracle import PageModel, PoolImage
+from oracle.stream import StreamOracle, bits16
+
+from gpu_drive import Frames, assert_close, new_cache, run_stream, workspace
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def pkv():
+    from paged_kv_cache_frame_b200 import build
+    build.build()
+    import paged_kv_cache_frame_b200 as m
+    return m
+
+
+W0 = workload.WORKLOADS[0]
+
+
+def small(ps, H=2, D=64, S=2, W=3, dtype="bf16", frames=20):
+    return dataclasses.replace(W0, name=f"ps{ps}", H=H, D=D, P=ps, page_size=ps, S=S, W=W,
+                               frames=frames, dtype=dtype)
+
+
+# --------------------------------------------------------------- append scatter
+@pytest.mark.parametrize("wl", [W0, small(256), small(999, H=1), small(130), small(64, D=128, dtype="fp16")],
+                         ids=lambda w: w.name)
+def test_append_scatter_pool_bit_exact(pkv, wl):
+    fr = Frames(wl, seed=7)
+    cache = new_cache(pkv, wl)
+    m = PageModel(wl.S, wl.W, wl.page_size, wl.max_pages, NS=wl.NS)
+    img = PoolImage(m, wl.H, wl.D)
+    rng = np.random.default_rng(3)
+    for f in range(14):
+        _, k, v = fr.get(f)
+        defer = bool(rng.random() < 0.3)
+        cache.defer_eviction(defer)
+        m.set_defer(defer)
+        cache.append_frame(0, k.cuda(), v.cuda())
+        cache.evict_frames()
+        page, sp0 = m.append(f)
+        m.evict()
+        img.write(page, sp0, bits16(k), bits16(v))
+        pool = cache.pools[0].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+        np.testing.assert_array_equal(pool, img.bits, err_msg=f"frame {f}")
+        if defer:
+            if rng.random() < 0.5:
+                cache.commit_frame(); m.commit()
+            else:
+                cache.rollback_last_frame(); m.rollback()
+        assert cache.free_list() == m.free
+
+
+# --------------------------------------------------------------- attention
+def test_tiny_config_every_frame_every_row(pkv):
+    res = run_stream(pkv, W0, seed=11, n_frames=W0.frames, check=set(range(W0.frames)))
+    assert len(res) == W0.frames
+
+
+@pytest.mark.parametrize("tps", [1, 2, 3])
+def test_forced_split_kv_matches_oracle(pkv, tps):
+    run_stream(pkv, W0, seed=12, n_frames=12, check={0, 5, 11}, tiles_per_split=tps)
+    wl = small(256, frames=9)
+    run_stream(pkv, wl, seed=13, n_frames=9, check={8}, tiles_per_split=tps)
+
+
+def test_split_and_unsplit_agree(pkv):
+    wl = small(256, H=3, S=2, W=4, frames=8)
+    a, b = {}, {}
+    run_stream(pkv, wl, seed=14, n_frames=8, check={7}, collect=a)
+    run_stream(pkv, wl, seed=14, n_frames=8, check={7}, tiles_per_split=2, collect=b)
+    d = (a[7].float() - b[7].float()).abs()
+    assert d.max().item() <= 1e-2
+
+
+@pytest.mark.parametrize("ps", [16, 64, 100, 128, 129, 256, 999])
+def test_page_sizes_with_eviction(pkv, ps):
+    wl = small(ps, H=2, S=2, W=3, frames=12)
+    run_stream(pkv, wl, seed=20 + ps, n_frames=12, check={0, 1, 4, 5, 6, 11})
+
+
+def test_head_dim_128_fp16(pkv):
+    wl = small(256, H=2, D=128, dtype="fp16", frames=10)
+    run_stream(pkv, wl, seed=31, n_frames=10, check={0, 9})
+    run_stream(pkv, wl, seed=32, n_frames=10, check={9}, tiles_per_split=2)
+
+
+def test_deferred_frames_commit_and_rollback(pkv):
+    wl = small(256, H=2, S=2, W=3, frames=24)
+    keep = workload.keyframe_mask(dataclasses.replace(wl, keyframes="bernoulli"), seed=5)
+    defer = np.ones(wl.frames, dtype=bool)          # every frame deferred, decided after
+    run_stream(pkv, wl, seed=33, n_frames=wl.frames, check=set(range(wl.frames)), defer=defer,
+               keep=keep)
+    # interval mode: non-keyframes deferred then rolled back, keyframes appended directly
+    k4 = workload.interval_mask(wl.frames, 4)
+    run_stream(pkv, wl, seed=34, n_frames=wl.frames, check=set(range(0, wl.frames, 3)),
+               defer=~k4, keep=k4)
+
+
+def test_patch_pool_size_does_not_change_results(pkv):
+    """Relabelling the special pages (a larger patch pool moves them) gives
+    bit-identical outputs: the kernel reads pages only through the table."""
+    wl = small(256, H=2, S=2, W=3, frames=9)
+    a, b = {}, {}
+    run_stream(pkv, wl, seed=35, n_frames=9, check={8}, collect=a)
+    run_stream(pkv, wl, seed=35, n_frames=9, check={8}, collect=b, patch_pages=wl.patch_pages + 7)
+    assert torch.equal(a[8], b[8])
+
+
+def test_batched_streams_ragged_ages(pkv):
+    wl = small(256, H=2, D=128, dtype="fp16", S=2, W=3, frames=16)
+    ages = [3, 9, 1, 14]
+    caches, oracles, qs = [], [], []
+    for s, age in enumerate(ages):
+        fr = Frames(wl, seed=40, stream=s)
+        c = new_cache(pkv, wl)
+        so = StreamOracle(wl.S, wl.W, wl.NS, wl.P, wl.dtype, fr.bits)
+        for f in range(age):
+            q, k, v = fr.get(f)
+            c.append_frame(0, k.cuda(), v.cuda())
+            c.evict_frames()
+            so.begin_frame(f)
+        caches.append(c)
+        oracles.append(so)
+        qs.append(q)
+    ws = workspace(pkv, caches)
+    plan = pkv.Plan(caches, ws)
+    q = torch.cat(qs).cuda()
+    out = plan.run(0, q)
+    plan.check_device()
+    for s, so in enumerate(oracles):
+        assert_close(out[s * wl.T:(s + 1) * wl.T], so.expected(), f"stream {s}")
+
+
+def test_closed_forms_on_gpu(pkv):
+    """Constant V gives that constant; identical keys give the mean of V."""
+    wl = small(128, H=2, S=1, W=2, frames=4)
+    cache = new_cache(pkv, wl)
+    ws = workspace(pkv, [cache])
+    g = torch.Generator().manual_seed(0)
+    vs = []
+    for f in range(3):
+        q = torch.randn(wl.T, wl.H, wl.D, generator=g).bfloat16()
+        k = torch.full((wl.T, wl.H, wl.D), 0.5).bfloat16()
+        v = torch.full((wl.T, wl.H, wl.D), 0.75).bfloat16()
+        v[:, 1] = torch.randn(wl.T, wl.D, generator=g).bfloat16()
+        vs.append(v)
+        cache.append_frame(0, k.cuda(), v.cuda())
+        cache.evict_frames()
+    out = pkv.Plan([cache], ws).run(0, q.cuda()).float().cpu()
+    assert torch.all(out[:, 0] == 0.75)
+    # head 1: all keys equal -> uniform weights over the 3 * 134 visible tokens
+    allv = torch.cat([x[:, 1].float() for x in vs])
+    mean = allv.mean(0)
+    assert (out[:, 1] - mean).abs().max().item() < 4e-3
+
+
+def test_run_errors(pkv):
+    wl = small(64, H=2, frames=3)
+    cache = new_cache(pkv, wl, num_blocks=1)
+    ws = workspace(pkv, [cache])
+    fr = Frames(wl, seed=50)
+    q, k, v = (x.cuda() for x in fr.get(0))
+    cache.append_frame(0, k, v)
+    plan = pkv.Plan([cache], ws)
+    plan.run(0, q)
+    cache.evict_frames()
+    q, k, v = (x.cuda() for x in fr.get(1))
+    cache.append_frame(0, k, v)                 # state changed: the plan is stale
+    with pytest.raises(pkv.KVError) as e:
+        plan.run(0, q)
+    assert e.value.name == "STALE_PLAN"
+    small_ws = torch.empty(1024, dtype=torch.uint8, device="cuda")
+    with pytest.raises(pkv.KVError) as e:
+        pkv.Plan([cache], small_ws)
+    assert e.value.name == "CAPACITY"
+    plan = pkv.Plan([cache], ws)
+    plan.run(0, q)
+    plan.check_device()
+
+
+# --------------------------------------------------------------- full-size workloads
+def sample_rows(T, seed, n=24):
+    rng = np.random.default_rng(seed)
+    return sorted(set([0, 1, 5, T - 1, 128, 255, 256, T - 6]) | set(rng.integers(0, T, n).tolist()))
+
+
+def test_full_224_stream_block0_sampled(pkv):
+    wl = workload.WORKLOADS[1]
+    run_stream(pkv, wl, seed=1, n_frames=wl.frames, check={0, 71, 72, 159, 319},
+               rows=sample_rows(wl.T, 1))
+
+
+def test_full_224_keyframes_block0_sampled(pkv):
+    wl = workload.WORKLOADS[2]
+    keep = workload.keyframe_mask(wl, seed=2)
+    run_stream(pkv, wl, seed=2, n_frames=wl.frames, check={50, 200, 319}, rows=sample_rows(wl.T, 2),
+               defer=np.ones(wl.frames, dtype=bool), keep=keep)
+
+
+def test_full_518x378_stream_block0_sampled(pkv):
+    wl = workload.WORKLOADS[3]
+    run_stream(pkv, wl, seed=3, n_frames=wl.frames, check={0, 499, 999},
+               rows=sample_rows(wl.T, 3, n=12))
+
+
+def test_full_batched_ragged_sampled(pkv):
+    wl = workload.WORKLOADS[4]
+    ages = workload.stream_ages(wl, seed=4)
+    caches, oracles, qs = [], [], []
+    for s, age in enumerate(ages):
+        fr = Frames(wl, seed=4, stream=s)
+        c = new_cache(pkv, wl)
+        so = StreamOracle(wl.S, wl.W, wl.NS, wl.P, wl.dtype, fr.bits)
+        for f in range(int(age) + 1):
+            q, k, v = fr.get(f)
+            c.append_frame(0, k.cuda(), v.cuda())
+            c.evict_frames()
+            so.begin_frame(f)
+        caches.append(c)
+        oracles.append(so)
+        qs.append(q)
+    ws = workspace(pkv, caches)
+    plan = pkv.Plan(caches, ws)
+    out = plan.run(0, torch.cat(qs).cuda())
+    plan.check_device()
+    rows = sample_rows(wl.T, 4, n=8)
+    for s, so in enumerate(oracles):
+        got = out[s * wl.T:(s + 1) * wl.T][torch.as_tensor(rows)]
+        assert_close(got, so.expected(rows), f"stream {s} age {ages[s]}")

@@ -140,6 +140,7 @@ def test_stream_oracle_sees_the_page_models_tokens():
     for f in range(12):
         so.begin_frame(f)
     ks, vs = so.visible_kv()
+    ks, vs = ks.astype(np.float64), vs.astype(np.float64)
     kp, vp = _paged_run(wl, frames)
     key = lambda k, v: sorted(map(bytes, np.concatenate([k, v], axis=-1).reshape(k.shape[0], -1)))
     assert key(ks, vs) == key(kp, vp)
