@@ -9,7 +9,9 @@ from __future__ import annotations
 import ctypes
 import os
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib", "libpkv.so")
+# PKV_LIB selects another build of the same library (e.g. an instrumented one).
+LIB_PATH = os.environ.get("PKV_LIB") or os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib",
+                                                     "libpkv.so")
 
 KV_OK = 0
 KV_ERR_ARG = -1

@@ -59,5 +59,8 @@ cudaError_t upload_plan(void* dst, const void* src, size_t bytes, cudaStream_t s
 
 // Attention CTAs that fit on one SM for this head_dim (used by the planner).
 int attention_ctas_per_sm(int D);
+// Whether the attention kernel computes <= 16-row tail tiles inside the
+// preceding unit for this head_dim (used by the planner).
+bool attention_tail_ok(int D);
 
 }  // namespace pkv

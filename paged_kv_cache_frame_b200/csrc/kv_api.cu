@@ -275,6 +275,7 @@ int kv_plan(kv_plan_t** out, kv_cache_t* const* caches, int n_streams, int tiles
   in.num_sms = workspace ? device_sms() : 148;
   in.ctas_per_sm = pkv::attention_ctas_per_sm(g.D);
   in.tiles_per_split = tiles_per_split;
+  in.tail_ok = pkv::attention_tail_ok(g.D);
   kv_plan_t* p = new kv_plan_t();
   std::string why;
   rc = pkv::build_plan(st, in, &p->hp, &why);

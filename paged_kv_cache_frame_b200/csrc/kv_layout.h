@@ -10,7 +10,7 @@
 namespace pkv {
 
 constexpr int kTile = 128;           // query rows per CTA tile == K/V tokens per tile
-constexpr int kMaxTargetCtas = 1024; // bound on CTAs the split schedule may add
+constexpr int kMaxTargetCtas = 512;  // bound on CTAs the split schedule may add
 
 // One request (video stream) of the batch.
 struct KvReq {
@@ -29,17 +29,22 @@ struct KvTile {
   int16_t hi;
 };
 
-// One CTA of the attention launch.
+// One CTA of the attention launch: one or two consecutive 128-row query
+// tiles of one head, optionally followed by a short tail tile (<= 16 rows),
+// against a range of K/V tiles.
 struct KvUnit {
   int16_t req;
   int16_t head;
-  int16_t qtile;       // query rows [qtile*128, qtile*128 + 128) of the request
+  int16_t qtile;       // first query tile: rows [qtile*128, qtile*128 + 128)
+  int16_t nq;          // full query tiles in the unit (1 or 2)
+  int16_t tail_rows;   // rows of the tail tile qtile + nq (0 = none)
   int16_t pad;
   int32_t tile_begin;  // absolute index into the tile table
   int32_t tile_end;
-  int32_t slot;        // -1: write `out`; else split-KV partial slot
-  int32_t pad2;
+  int32_t slot[3];     // per query tile (tail last): -1 = write `out`, else partial slot
 };
+
+constexpr int kMaxTailRows = 16;   // tail rows computed with swapped operands (N = 16)
 
 // One (request, head, q-tile) whose K/V range was split over n CTAs.
 struct KvMergeItem {

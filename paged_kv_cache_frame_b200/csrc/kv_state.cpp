@@ -217,7 +217,7 @@ WorkspaceLayout workspace_layout(const std::vector<const PageState*>& st) {
     tiles_cap += (size_t)c.max_pages * ceil_div(c.page_size, kTile);
     D = c.D;
   }
-  L.slot_cap = units_base + kMaxTargetCtas;
+  L.slot_cap = 2 * (units_base + kMaxTargetCtas);
   const size_t units_cap = units_base + L.slot_cap;
   size_t off = header_bytes();
   off += align_up(st.size() * sizeof(KvReq), 16);
@@ -263,12 +263,28 @@ int build_plan(const std::vector<const PageState*>& st, const PlanInputs& in, Ho
     P.visible += s->visible_tokens();
   }
 
-  // Work units: (request, head, q-tile), each split into chunks of at most L
-  // K/V tiles so that the launch fills the machine.
+  // Work units: (request, head, pair of query tiles) -- a lone last tile
+  // forms a single unit -- each split into chunks of at most L K/V tiles so
+  // that the launch fills the machine. When the kernel supports it, a last
+  // query tile of at most 16 rows rides as a tail on the preceding unit,
+  // which computes it with swapped operands (S^T = K Q^T, N = 16). Per K/V
+  // tile a pair costs about 1.0, a single unit about 0.7, a tail 0.3 more.
+  struct Group { int req, qt, nq, tail, n; double w; };
+  std::vector<Group> groups;
   int n_base = 0, max_n = 0;
   for (int r = 0; r < n_req; ++r) {
-    const int qt = ceil_div(P.reqs[r].T, kTile);
-    n_base += qt * H;
+    const int T = P.reqs[r].T;
+    int qtiles = ceil_div(T, kTile);
+    const int last_rows = T - (qtiles - 1) * kTile;
+    const bool tail = in.tail_ok && qtiles >= 2 && last_rows <= kMaxTailRows;
+    if (tail) --qtiles;
+    for (int qt = 0; qt < qtiles; qt += 2) {
+      const int nq = std::min(2, qtiles - qt);
+      const bool last = qt + nq >= qtiles;
+      groups.push_back({r, qt, nq, (tail && last) ? last_rows : 0, P.reqs[r].n_tiles,
+                        (nq == 2 ? 1.0 : 0.7) + ((tail && last) ? 0.3 : 0.0)});
+    }
+    n_base += ceil_div(qtiles, 2) * H;
     max_n = std::max(max_n, P.reqs[r].n_tiles);
   }
   const int target = std::max(1, in.num_sms * in.ctas_per_sm);
@@ -278,20 +294,19 @@ int build_plan(const std::vector<const PageState*>& st, const PlanInputs& in, Ho
   } else {
     // Pick the chunk size whose schedule finishes first when CTAs are handed
     // to `target` slots greedily, longest first (what the block scheduler
-    // does); a CTA costs its tiles plus a fixed prologue/epilogue.
-    std::vector<int> lens;
-    for (int r = 0; r < n_req; ++r)
-      for (int k = 0; k < ceil_div(P.reqs[r].T, kTile) * H; ++k) lens.push_back(P.reqs[r].n_tiles);
+    // does); a CTA costs its weighted tiles plus a fixed prologue/epilogue.
     L = max_n;
     double best = 1e300;
     for (int c = 1; c <= 32; ++c) {
       const int cand = std::max(1, ceil_div(max_n, c));
       if (c > 1 && cand == ceil_div(max_n, c - 1)) continue;
       std::vector<double> costs;
-      for (int n : lens) {
-        const int ch = std::max(1, ceil_div(n, cand));
-        for (int k = 0; k < ch; ++k)
-          costs.push_back((double)((long long)(k + 1) * n / ch - (long long)k * n / ch) + 2.0 + (ch > 1 ? 1.0 : 0.0));
+      for (const Group& g : groups) {
+        const int ch = std::max(1, ceil_div(g.n, cand));
+        for (int k = 0; k < ch; ++k) {
+          const double tiles = (double)((long long)(k + 1) * g.n / ch - (long long)k * g.n / ch);
+          for (int h = 0; h < H; ++h) costs.push_back(tiles * g.w + 2.0 + (ch > 1 ? 1.0 : 0.0));
+        }
       }
       if ((int)costs.size() > target + n_base) break;
       std::sort(costs.begin(), costs.end(), std::greater<double>());
@@ -310,31 +325,32 @@ int build_plan(const std::vector<const PageState*>& st, const PlanInputs& in, Ho
   }
   const WorkspaceLayout WL = workspace_layout(st);
   int n_slots = 0;
-  for (int r = 0; r < n_req; ++r) {
-    const int nt = P.reqs[r].n_tiles;
-    const int qtiles = ceil_div(P.reqs[r].T, kTile);
+  for (const Group& g : groups) {
+    const int nt = g.n;
     const int chunks = std::max(1, ceil_div(nt, L));
+    const int ntiles_q = g.nq + (g.tail ? 1 : 0);
     for (int h = 0; h < H; ++h) {
-      for (int qt = 0; qt < qtiles; ++qt) {
-        int slot0 = -1;
-        if (chunks > 1) {
-          slot0 = n_slots;
+      int slot0[3] = {-1, -1, -1};
+      if (chunks > 1) {
+        for (int t = 0; t < ntiles_q; ++t) {
+          slot0[t] = n_slots;
           n_slots += chunks;
           KvMergeItem m{};
-          m.req = (int16_t)r; m.head = (int16_t)h; m.qtile = (int16_t)qt;
-          m.n = (int16_t)chunks; m.slot0 = slot0;
+          m.req = (int16_t)g.req; m.head = (int16_t)h; m.qtile = (int16_t)(g.qt + t);
+          m.n = (int16_t)chunks; m.slot0 = slot0[t];
           P.merges.push_back(m);
           ++P.n_split_units;
         }
-        for (int k = 0; k < chunks; ++k) {
-          KvUnit u{};
-          u.req = (int16_t)r; u.head = (int16_t)h; u.qtile = (int16_t)qt;
-          u.tile_begin = tile0[r] + (int)((long long)k * nt / chunks);
-          u.tile_end = tile0[r] + (int)((long long)(k + 1) * nt / chunks);
-          u.slot = chunks > 1 ? slot0 + k : -1;
-          P.max_tiles_per_cta = std::max(P.max_tiles_per_cta, u.tile_end - u.tile_begin);
-          P.units.push_back(u);
-        }
+      }
+      for (int k = 0; k < chunks; ++k) {
+        KvUnit u{};
+        u.req = (int16_t)g.req; u.head = (int16_t)h; u.qtile = (int16_t)g.qt; u.nq = (int16_t)g.nq;
+        u.tail_rows = (int16_t)g.tail;
+        u.tile_begin = tile0[g.req] + (int)((long long)k * nt / chunks);
+        u.tile_end = tile0[g.req] + (int)((long long)(k + 1) * nt / chunks);
+        for (int t = 0; t < 3; ++t) u.slot[t] = (chunks > 1 && t < ntiles_q) ? slot0[t] + k : -1;
+        P.max_tiles_per_cta = std::max(P.max_tiles_per_cta, u.tile_end - u.tile_begin);
+        P.units.push_back(u);
       }
     }
   }

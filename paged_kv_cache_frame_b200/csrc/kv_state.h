@@ -82,6 +82,7 @@ struct PlanInputs {
   int num_sms;           // SMs of the device
   int ctas_per_sm;       // attention CTAs resident per SM
   int tiles_per_split;   // > 0: forced chunk size (tests); 0: automatic
+  bool tail_ok;          // the attention kernel computes <= 16-row tail tiles in-unit
 };
 
 struct HostPlan {

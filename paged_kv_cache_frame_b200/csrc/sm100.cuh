@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "tmem_access.cuh"
+
 namespace pkv {
 
 // A wait that has not completed after this long gives up and reports an error
@@ -128,6 +130,18 @@ __device__ __forceinline__ void umma_f16_ss(uint32_t d_tmem, uint64_t adesc, uin
       : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem desc], kind::f16. A (M x K, K-major) sits in
+// TMEM with lane = row and two 16-bit elements per 32-bit column.
+__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive on `bar` once every tcgen05 op issued so far by this thread completes.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -139,8 +153,9 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
 // [4,6) D format (1 = f32), [7,10) A format, [10,13) B format (0 = f16,
 // 1 = bf16), [15] A major, [16] B major (0 = K, 1 = MN), [17,23) N >> 3,
 // [24,29) M >> 4.
-__host__ __device__ constexpr uint32_t umma_idesc_f16(int M, int N, bool fp16, bool b_mn_major) {
-  return (1u << 4) | ((fp16 ? 0u : 1u) << 7) | ((fp16 ? 0u : 1u) << 10) |
+__host__ __device__ constexpr uint32_t umma_idesc_f16(int M, int N, bool fp16, bool b_mn_major,
+                                                    bool a_mn_major = false) {
+  return (1u << 4) | ((fp16 ? 0u : 1u) << 7) | ((fp16 ? 0u : 1u) << 10) | ((a_mn_major ? 1u : 0u) << 15) |
          ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
@@ -160,31 +175,10 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   return d;
 }
 
-// TMEM load of 32 consecutive 32-bit columns of this warp's 32 lanes (one row
-// per thread), waiting for completion before the values are used.
-#define PKV_R8(i) "=r"(r[i]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), "=r"(r[i + 4]), \
-                  "=r"(r[i + 5]), "=r"(r[i + 6]), "=r"(r[i + 7])
-__device__ __forceinline__ void tmem_ld32_wait(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : PKV_R8(0), PKV_R8(8), PKV_R8(16), PKV_R8(24)
-      : "r"(taddr)
-      : "memory");
+// Named barrier over `count` threads (id 0 is __syncthreads).
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
-#undef PKV_R8
-
-#define PKV_W8(i) "r"(r[i]), "r"(r[i + 1]), "r"(r[i + 2]), "r"(r[i + 3]), "r"(r[i + 4]), "r"(r[i + 5]), \
-                  "r"(r[i + 6]), "r"(r[i + 7])
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
-      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-      PKV_W8(0), PKV_W8(8), PKV_W8(16), PKV_W8(24)
-      : "memory");
-}
-#undef PKV_W8
 
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
@@ -194,6 +188,77 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// ---- packed fp32 pairs (one instruction for two lanes of work)
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// Two 16-bit floats (round to nearest even) packed low = a, high = b.
+__device__ __forceinline__ uint32_t cvt_pack_bf16(float a, float b) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+  return r;
+}
+__device__ __forceinline__ uint32_t cvt_pack_f16(float a, float b) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+  return r;
+}
+
+// 2^x for a pair of arguments on the FMA pipe instead of the MUFU unit.
+// Cody-Waite style reduction x = n + f, n = round(x), f in [-1/2, 1/2]; 2^f by
+// a degree-3 minimax polynomial (relative error <= 7.5e-5, well below the
+// 2^-9 rounding of the 16-bit P it feeds); 2^n by adding n to the exponent
+// field. Coefficients: `python -m paged_kv_cache_frame_b200.csrc.exp2_poly`.
+// Arguments below -126 are clamped, so the exponent field never wraps (c0 < 1
+// has biased exponent 126); the result is then ~1e-38, not 0.
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+  constexpr float kRound = 12582912.0f;   // 1.5 * 2^23: adding it rounds to an integer
+  float a, b;
+  f2_unpack(x2, a, b);
+  a = fmaxf(a, -126.f);
+  b = fmaxf(b, -126.f);
+  const uint64_t x = f2_pack(a, b);
+  const uint64_t j = f2_add(x, f2_pack(kRound, kRound));           // n in the low mantissa bits
+  const uint64_t n = f2_add(j, f2_pack(-kRound, -kRound));          // n as a float
+  const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), x);             // f = x - n
+  uint64_t p = f2_fma(f, f2_pack(5.517166853e-02f, 5.517166853e-02f), f2_pack(2.426111251e-01f, 2.426111251e-01f));
+  p = f2_fma(p, f, f2_pack(6.932609677e-01f, 6.932609677e-01f));
+  p = f2_fma(p, f, f2_pack(9.999280572e-01f, 9.999280572e-01f));
+  float pa, pb, ja, jb;
+  f2_unpack(p, pa, pb);
+  f2_unpack(j, ja, jb);
+  const float ra = __int_as_float(__float_as_int(pa) + (__float_as_int(ja) << 23));
+  const float rb = __int_as_float(__float_as_int(pb) + (__float_as_int(jb) << 23));
+  return f2_pack(ra, rb);
 }
 
 }  // namespace pkv

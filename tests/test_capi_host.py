@@ -279,7 +279,8 @@ def test_kv_tiles_cover_visible_tokens_exactly_once(pkv, ps, n):
 
 def test_split_schedule_covers_each_unit(pkv):
     """Host plan for the 224x224 shape at frame 320: 159 tiles per head,
-    16 heads x 3 query tiles; a forced split of 10 tiles per CTA."""
+    16 heads x 3 query tiles (one pair-plus-tail unit per head); a forced
+    split of 10 tiles per CTA."""
     h = pkv.kv_init(81, 256, 16, 64, 8, 64, 1, 6, pkv.KV_BF16, 0)
     for _ in range(320):
         step(pkv, h)
@@ -287,13 +288,15 @@ def test_split_schedule_covers_each_unit(pkv):
     s = pkv.kv_plan_get_stats(p)
     assert s["n_kv_tiles"] == 159
     assert s["visible_tokens"] == 72 * 256 + 6 * 320
-    assert s["n_split_units"] == 48
-    assert s["n_ctas"] == 48 * 16           # ceil(159 / 10) = 16 chunks each
+    assert s["n_split_units"] == 48          # every (head, query tile) is split
+    # per head one unit: query tiles 0-1 plus the 6-row tail tile 2, in
+    # ceil(159/10) = 16 chunks
+    assert s["n_ctas"] == 16 * 16
     assert s["tiles_per_cta"] <= 10
     pkv.kv_plan_free(p)
     p = pkv.kv_plan([h])                   # automatic: fills 148 SMs
     s = pkv.kv_plan_get_stats(p)
-    assert 100 <= s["n_ctas"] <= 2 * 148 + 48
+    assert 100 <= s["n_ctas"] <= 2 * 148 + 16
     pkv.kv_plan_free(p)
     pkv.kv_destroy(h)
 
