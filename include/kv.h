@@ -242,6 +242,45 @@ int kv_plan_get_stats(const kv_plan_t* plan, kv_plan_stats* out);
  * word. KV_OK, KV_ERR_DEVICE_CHECK (bit set by a kernel) or KV_ERR_CUDA. */
 int kv_check_device(const kv_plan_t* plan, void* stream);
 
+/* Size of the library-owned device array that kv_run_static uses as scratch. */
+#define KV_STATIC_SCRATCH_BYTES (32u << 20)
+
+/* kv_run_static -- kv_plan + kv_run for one block in a single call that
+ * allocates no memory. The paper has no counterpart: this entry point is for
+ * callers that cannot call cudaMalloc, or do not want to allocate, for
+ * example a host engine that runs under a fixed memory budget, or code that
+ * runs while an allocator is locked. The caller still provides the caches
+ * (with their bound pools), q and out as for kv_plan and kv_run. The plan's
+ * tables and the split-KV partials go into one static device array of
+ * KV_STATIC_SCRATCH_BYTES that the library holds instead of a caller
+ * workspace.
+ *
+ * Arguments are as for kv_plan followed by kv_run. check != 0 also
+ * synchronises `stream` and reads the kernels' error word, returning
+ * KV_ERR_DEVICE_CHECK if a wait timed out. `stream` must belong to the
+ * current device.
+ *
+ * Memory and set-up:
+ *   - The array is reserved on every device where the library's code is
+ *     loaded, and it stays there until the process exits.
+ *   - On the first call on a device, with that device current, the library
+ *     looks up the array's device address. Make that first call before any
+ *     stream capture on the device.
+ *   - Each call rewrites the tables, and with them the zeroed error word, at
+ *     the start of the array. Partials are written before they are read.
+ *
+ * Concurrency: every call on a device shares the array. Two calls that
+ * overlap on the GPU (for example on two streams with no ordering between
+ * them) race and corrupt each other's output. Calls on one stream are
+ * ordered and safe.
+ *
+ * Errors: as kv_plan and kv_run, plus KV_ERR_CAPACITY when the call needs
+ * more than KV_STATIC_SCRATCH_BYTES of scratch. That check runs before any
+ * GPU work. A 224x224 frame (16 heads, 262 tokens, 320-frame stream) needs
+ * about 15 MB with automatic splitting. */
+int kv_run_static(kv_cache_t* const* caches, int n_streams, int block, int tiles_per_split,
+                  const void* q, void* out, int check, void* stream);
+
 /* kv_strerror -- static text for a status code. */
 const char* kv_strerror(int status);
 

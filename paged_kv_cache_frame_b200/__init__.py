@@ -22,7 +22,7 @@ from __future__ import annotations
 import ctypes
 
 from . import capi
-from .capi import KVError, KV_BF16, KV_FP16, KV_MAX_STREAMS
+from .capi import KVError, KV_BF16, KV_FP16, KV_MAX_STREAMS, KV_STATIC_SCRATCH_BYTES
 
 __all__ = [
     "PagedKVCache", "Plan", "KVError", "workspace_bytes", "KV_BF16", "KV_FP16", "KV_MAX_STREAMS",
@@ -30,7 +30,7 @@ __all__ = [
     "kv_evict_frames", "kv_defer_eviction", "kv_commit_frame", "kv_rollback_last_frame",
     "kv_get_stats", "kv_get_free_list", "kv_workspace_bytes", "kv_plan", "kv_run",
     "kv_plan_free", "kv_get_page_table", "kv_get_kv_tiles", "kv_plan_get_stats",
-    "kv_check_device", "kv_strerror", "kv_last_error",
+    "kv_check_device", "kv_strerror", "kv_last_error", "kv_run_static",
 ]
 
 
@@ -173,6 +173,15 @@ def kv_plan_get_stats(plan) -> dict:
 
 def kv_check_device(plan, stream=None) -> None:
     capi.check(capi.lib().kv_check_device(plan, _stream(stream)), "kv_check_device")
+
+
+def kv_run_static(caches, block, q, out, tiles_per_split=0, check=False, stream=None) -> None:
+    """kv_plan + kv_run for one block without any allocation: the plan tables
+    and split-KV partials go to the library's static device array
+    (KV_STATIC_SCRATCH_BYTES). For callers that cannot allocate device memory;
+    calls that overlap on the GPU share that array and race."""
+    capi.check(capi.lib().kv_run_static(_handles(caches), len(caches), block, tiles_per_split, _ptr(q),
+                                        _ptr(out), int(bool(check)), _stream(stream)), "kv_run_static")
 
 
 def kv_strerror(status) -> str:

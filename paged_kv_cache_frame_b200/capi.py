@@ -27,6 +27,7 @@ KV_ERR_STALE_PLAN = -10
 KV_BF16 = 0
 KV_FP16 = 1
 KV_MAX_STREAMS = 32
+KV_STATIC_SCRATCH_BYTES = 32 << 20
 
 ERR_NAMES = {
     KV_ERR_ARG: "ARG", KV_ERR_CAPACITY: "CAPACITY", KV_ERR_ORDER: "ORDER",
@@ -82,6 +83,7 @@ SIGNATURES = {
     "kv_get_kv_tiles": (_I, [_P, _I, _IP, _IP, _IP, _I, _IP]),
     "kv_plan_get_stats": (_I, [_P, ctypes.POINTER(kv_plan_stats)]),
     "kv_check_device": (_I, [_P, _P]),
+    "kv_run_static": (_I, [ctypes.POINTER(_P), _I, _I, _I, _P, _P, _I, _P]),
     "kv_strerror": (ctypes.c_char_p, [_I]),
     "kv_last_error": (ctypes.c_char_p, []),
 }

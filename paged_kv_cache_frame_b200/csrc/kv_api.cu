@@ -4,8 +4,10 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -404,3 +406,111 @@ int kv_check_device(const kv_plan_t* p, void* stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// kv_run_static: kv_plan + kv_run for one block with the scratch (plan tables
+// and split-KV partials) in a library-owned device array, for callers that
+// cannot allocate device memory. Nothing here calls an allocator.
+
+// Every device that loads this module holds this array until the process
+// exits. In host code the name is only a stand-in for the device symbol: its
+// device address comes from cudaGetSymbolAddress below.
+static __device__ __align__(256) uint8_t g_static_scratch[KV_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 256;
+std::mutex g_static_mu;
+void* g_static_addr[kMaxDevices] = {};   // device address of g_static_scratch, per device
+
+// Device address of the array on the current device, looked up once per
+// device with that device current.
+int static_scratch(void** ptr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "kv_run_static: cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(KV_ERR_UNSUPPORTED, "kv_run_static: device ordinal out of range");
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (!g_static_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "kv_run_static: cudaGetSymbolAddress");
+    g_static_addr[dev] = p;
+  }
+  *ptr = g_static_addr[dev];
+  return KV_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace
+
+extern "C" int kv_run_static(kv_cache_t* const* caches, int n_streams, int block, int tiles_per_split,
+                             const void* q, void* out, int check, void* stream) {
+  if (!q || !out) return fail(KV_ERR_ARG, "kv_run_static: NULL q/out");
+  if (tiles_per_split < 0) return fail(KV_ERR_ARG, "kv_run_static: tiles_per_split < 0");
+  std::vector<const pkv::PageState*> st;
+  int rc = check_batch(caches, n_streams, &st);
+  if (rc != KV_OK) return rc;
+  const pkv::Config& g = st[0]->cfg;
+  if (g.D != 64 && g.D != 128) return fail(KV_ERR_UNSUPPORTED, "kv_run_static: head_dim must be 64 or 128");
+  if (!aligned16(q) || !aligned16(out)) return fail(KV_ERR_ARG, "kv_run_static: q/out not 16-byte aligned");
+  if (block < 0 || block >= g.B) return fail(KV_ERR_ARG, "kv_run_static: block out of range");
+  for (int i = 0; i < n_streams; ++i) {
+    if (!caches[i]->st.is_appended(block)) return fail(KV_ERR_NOT_APPENDED, "kv_run_static: block not appended in this step");
+    if (!caches[i]->bound[block]) return fail(KV_ERR_ARG, "kv_run_static: no pool bound for this block");
+  }
+
+  kv_plan_t p;
+  pkv::PlanInputs in;
+  in.num_sms = device_sms();
+  in.ctas_per_sm = pkv::attention_ctas_per_sm(g.D);
+  in.tiles_per_split = tiles_per_split;
+  in.tail_ok = pkv::attention_tail_ok(g.D);
+  std::string why;
+  rc = pkv::build_plan(st, in, &p.hp, &why);
+  if (rc != KV_OK) return fail(rc, "kv_run_static: " + why);
+
+  // Packed layout in the array: tables, then the partials of the slots the
+  // schedule uses (not the worst case that kv_workspace_bytes provisions).
+  size_t n_slots = 0;
+  for (const pkv::KvMergeItem& m : p.hp.merges) n_slots = std::max(n_slots, (size_t)m.slot0 + (size_t)m.n);
+  const size_t off_o = align256(p.hp.image.size());
+  const size_t off_lse = align256(off_o + n_slots * pkv::kTile * (size_t)g.D * 4);
+  const size_t need = align256(off_lse + n_slots * pkv::kTile * 4);
+  if (need > KV_STATIC_SCRATCH_BYTES)
+    return fail(KV_ERR_CAPACITY, "kv_run_static: this call needs " + std::to_string(need) +
+                                     " bytes of scratch but the static array holds " +
+                                     std::to_string((size_t)KV_STATIC_SCRATCH_BYTES) +
+                                     "; use kv_plan/kv_run with a workspace or a larger tiles_per_split");
+  pkv::KvPlanHeader& hd = p.hp.header;
+  hd.off_part_o = (int64_t)off_o;
+  hd.off_part_lse = (int64_t)off_lse;
+  hd.error = 0;   // uploaded with the tables: the kernels' error word starts at zero on every call
+  std::memcpy(p.hp.image.data(), &hd, sizeof(hd));
+
+  void* scratch = nullptr;
+  rc = static_scratch(&scratch);
+  if (rc != KV_OK) return rc;
+  cudaError_t e = pkv::upload_plan(scratch, p.hp.image.data(), p.hp.image.size(), (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "kv_run_static: upload");
+  for (int i = 0; i < n_streams; ++i) {
+    p.caches.push_back(caches[i]);
+    p.epochs.push_back(caches[i]->st.epoch);
+    p.total_T += g.page_size + g.NS;
+  }
+  p.H = g.H;
+  p.D = g.D;
+  p.dtype = g.dtype;
+  p.ws = scratch;
+  p.ws_bytes = KV_STATIC_SCRATCH_BYTES;
+  rc = kv_run(&p, block, q, out, stream);
+  if (rc != KV_OK || !check) return rc;
+  e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "kv_run_static: synchronize");
+  uint32_t w = 0;
+  e = cudaMemcpy(&w, scratch, sizeof(w), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "kv_run_static: read error word");
+  if (w) return fail(KV_ERR_DEVICE_CHECK, "kernel error word " + std::to_string(w));
+  return KV_OK;
+}
