@@ -43,6 +43,37 @@ def peaks():
     return PEAKS_FALLBACK, "fallback"
 
 
+TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "paged_prefill_attn_224x224_dram.txt")
+KERNEL_SOURCES = ("paged_attn.cu", "sm100.cuh", "tmem_access.cuh", "kernels.h", "kv_layout.h")
+
+
+def kernel_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "paged_kv_cache_frame_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic():
+    """DRAM bytes per attention launch from the committed ncu summary, or None
+    when that summary was taken on other kernel sources than the ones built."""
+    if not os.path.exists(TRAFFIC_PROFILE):
+        return None
+    fields = {}
+    for line in open(TRAFFIC_PROFILE):
+        if ":" in line and not line.startswith("#"):
+            k, v = line.split(":", 1)
+            fields[k.strip()] = v.strip()
+    if fields.get("kernel_sources_sha256_16") != kernel_source_hash():
+        return None
+    try:
+        return float(fields["dram_bytes_per_launch_mean"])
+    except (KeyError, ValueError):
+        return None
+
+
 def call_flops(T, lkv, H, D):
     """Tensor FLOPs of one attention call: Q K^T and P V, 2 per MAC."""
     return 4.0 * T * lkv * H * D
@@ -314,7 +345,7 @@ def run_gpu(args):
                           "run_ms_per_pass": round(run_s * 1e3, 3)},
             "roofline": {"bound": "tensor", "achieved": round(tflops, 2),
                          "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                         "frac": round(tflops / pk["bf16_tflops"], 4), "traffic": None,
+                         "frac": round(tflops / pk["bf16_tflops"], 4), "traffic": measured_traffic(),
                          "peak_kind": f"{pk_kind} bf16 dense burst",
                          "kernel": "paged_prefill_attn + splitkv_merge (kv_run), event-timed per call"},
             "gpu_launches": launches,

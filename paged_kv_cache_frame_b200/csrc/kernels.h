@@ -18,6 +18,7 @@ struct AttnMaps {
 };
 
 struct AttnArgs {
+  const void* q;       // [sum T, H, D] (the tail rows are read directly)
   const KvReq* reqs;
   const KvUnit* units;
   const KvTile* tiles;

@@ -329,6 +329,7 @@ int kv_run(const kv_plan_t* p, int block, const void* q, void* out, void* stream
   uint8_t* ws = static_cast<uint8_t*>(p->ws);
   const pkv::KvPlanHeader& hd = p->hp.header;
   pkv::AttnArgs a;
+  a.q = q;
   a.reqs = reinterpret_cast<const pkv::KvReq*>(ws + hd.off_reqs);
   a.units = reinterpret_cast<const pkv::KvUnit*>(ws + hd.off_units);
   a.tiles = reinterpret_cast<const pkv::KvTile*>(ws + hd.off_tiles);

@@ -54,6 +54,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking: whether the phase with the given parity has completed.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase with the given parity to complete. Returns false if
 // `*abort` is raised by another thread or the wait exceeds kWaitLimitNs (then
 // it raises `*abort` itself).
@@ -259,6 +272,43 @@ __device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
   const float ra = __int_as_float(__float_as_int(pa) + (__float_as_int(ja) << 23));
   const float rb = __int_as_float(__float_as_int(pb) + (__float_as_int(jb) << 23));
   return f2_pack(ra, rb);
+}
+
+// ---- warp-level tensor-core MMA (the legacy mma.sync path), for small tiles
+// whose operands and accumulators stay in registers. Fragment layouts of
+// m16n8k16 (g = lane / 4, q = lane % 4): A rows g and g + 8, 16-bit columns
+// 2q, 2q + 1 (regs 0, 1) and 2q + 8, 2q + 9 (regs 2, 3); B column g, rows 2q,
+// 2q + 1 (reg 0) and 2q + 8, 2q + 9 (reg 1); C rows g (c0, c1) and g + 8
+// (c2, c3), columns 2q, 2q + 1.
+template <bool kFP16>
+__device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  if (kFP16)
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  else
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Four 8x8 16-bit matrices from shared memory; lanes 8m .. 8m + 7 give the
+// row addresses of matrix m. Lane l receives row l / 4, elements 2 (l % 4)
+// and 2 (l % 4) + 1 of each matrix (transposed: column l / 4, rows 2 (l % 4)
+// and 2 (l % 4) + 1).
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
 }
 
 }  // namespace pkv
