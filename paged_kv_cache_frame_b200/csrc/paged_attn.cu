@@ -11,7 +11,7 @@
 // Enables Long Sequence Inference in LingBot-Map", [P3] "FlashInfer Paged KV
 // Cache Performance Benefits in LingBot-Map".)
 //
-// Roles (head_dim 64: 448 threads; head_dim 128: 320):
+// Roles (head_dim 64: 384 threads; head_dim 128: 320):
 //   warps 0-3, 4-7  softmax warpgroups, one per 128-row query tile. Thread i
 //                   owns query row i == TMEM lane i. Per K/V tile it reads its
 //                   S row once, in two 64-column halves, keeps the running
@@ -19,21 +19,22 @@
 //                   rescales its O row when the running max grows by more
 //                   than 2^8 (lazy rescale: between rescales P may exceed 1,
 //                   which the final division by the same sum cancels).
-//   warp 8          TMA producer: the query tiles once, then K/V tiles of the
+//   warp 8 (9)      TMA producer: the query tiles once, then K/V tiles of the
 //                   page table into a STAGES-deep ring. A tile is 128 pool rows
 //                   of one head, one 3-D box load per 64 columns; the page table
 //                   gives each tile's row, so pages need not be contiguous.
-//   warp 9          TMEM allocator and MMA issuer (tcgen05 kind::f16, fp32
+//   warp 9 (11)     TMEM allocator and MMA issuer (tcgen05 kind::f16, fp32
 //                   accumulators in TMEM): S_t = Q_t K^T (M=128, N=128, K=D)
 //                   and O_t += P_t V (M=128, N=D, K=128, P read from TMEM).
-//   warps 10-13     (head_dim 64) the unit's tail: a last query tile of at most
-//                   16 rows (262 = 2 x 128 + 6 tokens per frame). An M = 128
+//   warps 8, 10     (head_dim 64; producer and MMA issuer then move to warps 9
+//                   and 11) the unit's tail: a last query tile of at most 16
+//                   rows (262 = 2 x 128 + 6 tokens per frame). An M = 128
 //                   tensor-core tile would be almost all padding, so each of
-//                   these warps computes the tail's scores and output for 32 of
+//                   these warps computes the tail's scores and output for 64 of
 //                   every K/V tile's 128 columns with warp-level mma.sync
 //                   m16n8k16, reading K and V straight from the shared-memory
 //                   ring, with its own running max/sum and O in registers. The
-//                   four partial results are merged at the end.
+//                   two partial results are merged at the end.
 // TMEM. head_dim 64: S_t at [128 t, +128), P_t at [256 + 64 t, +64), O_t at
 // [384 + 64 t, +64). P has its own columns, so the tensor core computes
 // S_t(j+1) as soon as the softmax has read S_t(j), while the exponentials of
@@ -63,8 +64,11 @@ __device__ unsigned long long g_pkv_trace[6][64][8];
 template <int D>
 struct AttnRoles {
   static constexpr bool kTail = D == 64;
-  static constexpr int kProducer = 8, kMma = 9, kTail0 = 10;
-  static constexpr int kWarps = kTail ? 14 : 10;
+  // head_dim 64: warps 8 and 10 are the tail (with the softmax warpgroups,
+  // three warps per SM sub-partition), 9 the producer, 11 the MMA issuer
+  static constexpr int kTailWarps = 2;   // each takes 64 of a K/V tile's 128 columns
+  static constexpr int kProducer = kTail ? 9 : 8, kMma = kTail ? 11 : 9;
+  static constexpr int kWarps = kTail ? 12 : 10;
   static constexpr int kThreads = 32 * kWarps;
 };
 
@@ -75,10 +79,11 @@ struct AttnSmem {
   static constexpr int kQ = 0;                       // two query tiles
   static constexpr int kK = 2 * kTileBytes;
   static constexpr int kV = kK + STAGES * kTileBytes;
-  // tail merge: per warp [16 rows][D] fp32 outputs, then [4][16] maxima and sums
+  // tail merge: per tail warp [16 rows][D] fp32 outputs, then maxima and sums
+  static constexpr int kTW = AttnRoles<D>::kTailWarps;
   static constexpr int kTailO = kV + STAGES * kTileBytes;
-  static constexpr int kTailML = kTailO + (kTail ? 4 * 16 * D * 4 : 0);
-  static constexpr int kTiles = kTailML + (kTail ? 2 * 4 * 16 * 4 : 0);
+  static constexpr int kTailML = kTailO + (kTail ? kTW * 16 * D * 4 : 0);
+  static constexpr int kTiles = kTailML + (kTail ? 2 * kTW * 16 * 4 : 0);
   static constexpr int kBars = kTiles + kMaxSmemTiles * 8;
   static constexpr int kBytes = kBars + 256;
   static constexpr int kAlloc = kBytes + 1024;      // slack to align the base to 1 KB
@@ -174,7 +179,7 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&bar_kv_full[s], 1);
       // released by the MMA issuer's commit and, with a tail, by each tail warp
-      mbar_init(&bar_kv_empty[s], 1 + (has_tail ? 4 : 0));
+      mbar_init(&bar_kv_empty[s], 1 + (has_tail ? R::kTailWarps : 0));
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bar_s_full[t], 1);
@@ -270,55 +275,64 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
       bool ok = mbar_wait(bar_q, 0, abort_flag) && wait_kv(0);
       if (ok)
         for (int t = 0; t < nq; ++t) issue_s(t, 0);
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        const bool more = j + 1 < n_tiles;
-        PKV_TRACE_AT(4, j, 0);
-        if (kSepP) {
-          // Four independent issues per tile: S_t(j+1) once softmax t has read
-          // S_t(j) and K(j+1) has landed, PV_t(j) once P_t(j) is written.
-          // Issue whichever is ready first (non-blocking polls, one bounded
-          // wait over all of them).
-          const uint32_t qmask = (1u << nq) - 1u;
-          const uint32_t want = (more ? qmask : 0u) | (qmask << 2);
-          uint32_t done = 0;
-          bool kv_next = !more || j + 1 <= kv_ready;
-          const uint64_t t0 = globaltimer_ns();
-          for (uint32_t spin = 1; done != want; ++spin) {
-            bool progress = false;
-            if (!kv_next && mbar_test_wait(&bar_kv_full[(j + 1) % STAGES], ((j + 1) / STAGES) & 1)) {
-              tc_fence_after();
-              kv_ready = j + 1;
-              kv_next = true;
-            }
+      if (kSepP) {
+        // Each query tile advances on its own: S_t(j) once softmax t has read
+        // S_t(j-1) and K(j) has landed, PV_t(j) once P_t(j) is written. The
+        // scores come first (the softmax waits on them); a K/V stage is
+        // released once every MMA that reads it has been issued. Non-blocking
+        // polls under one bounded wait.
+        int ns[2] = {1, 1};   // next S_t to issue
+        int np[2] = {0, 0};   // next PV_t to issue
+        if (nq < 2) ns[1] = np[1] = n_tiles;
+        int ne = 0;           // next K/V stage release
+        uint64_t t0 = globaltimer_ns();
+        for (uint32_t spin = 1; ok && ne < n_tiles; ++spin) {
+          bool progress = false;
 #pragma unroll
-            for (int t = 0; t < 2; ++t) {
-              if (t >= nq) break;
-              if (more && kv_next && !(done & (1u << t)) && mbar_test_wait(&bar_s_free[t], j & 1)) {
-                PKV_TRACE_AT(4, j, 1 + t);
-                tc_fence_after();
-                issue_s(t, j + 1);
-                done |= 1u << t;
-                progress = true;
+          for (int t = 0; t < 2; ++t) {
+            const int j = ns[t];
+            if (j < n_tiles && mbar_test_wait(&bar_s_free[t], (j - 1) & 1)) {
+              if (j > kv_ready) {
+                if (!mbar_test_wait(&bar_kv_full[j % STAGES], (j / STAGES) & 1)) continue;
+                kv_ready = j;
               }
-              if (!(done & (4u << t)) && mbar_test_wait(&bar_p_full[t], j & 1)) {
-                PKV_TRACE_AT(4, j, 4 + t);
-                tc_fence_after();
-                issue_pv(t, j);
-                done |= 4u << t;
-                progress = true;
-              }
-            }
-            if (!progress && (spin & 63u) == 0) {
-              if (*abort_flag) { ok = false; break; }
-              if (globaltimer_ns() - t0 > kWaitLimitNs) {
-                *abort_flag = 1;
-                ok = false;
-                break;
-              }
+              PKV_TRACE_AT(4, j - 1, 1 + t);
+              tc_fence_after();
+              issue_s(t, j);
+              ns[t] = j + 1;
+              progress = true;
             }
           }
-          if (!ok) break;
-        } else {
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            const int j = np[t];
+            if (j < n_tiles && mbar_test_wait(&bar_p_full[t], j & 1)) {
+              PKV_TRACE_AT(4, j, 4 + t);
+              tc_fence_after();
+              issue_pv(t, j);
+              np[t] = j + 1;
+              progress = true;
+            }
+          }
+          while (ne < min(np[0], np[1])) {   // PV_t(ne) issued for every t (and so S_t(ne))
+            umma_commit(&bar_kv_empty[ne % STAGES]);
+            PKV_TRACE_AT(4, ne, 7);
+            ++ne;
+            progress = true;
+          }
+          if (progress) {
+            t0 = globaltimer_ns();
+          } else if ((spin & 63u) == 0) {
+            if (*abort_flag || globaltimer_ns() - t0 > kWaitLimitNs) {
+              *abort_flag = 1;
+              ok = false;
+            }
+          }
+        }
+      } else {
+        for (int j = 0; ok && j < n_tiles; ++j) {
+          const bool more = j + 1 < n_tiles;
+          PKV_TRACE_AT(4, j, 0);
           // P_t(j) sits in the S_t columns: S_t(j+1) follows PV_t(j)
           for (int t = 0; t < nq; ++t) {
             if (!mbar_wait(&bar_p_full[t], j & 1, abort_flag)) { ok = false; break; }
@@ -331,9 +345,9 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
             }
           }
           if (!ok) break;
+          umma_commit(&bar_kv_empty[j % STAGES]);
+          PKV_TRACE_AT(4, j, 7);
         }
-        umma_commit(&bar_kv_empty[j % STAGES]);
-        PKV_TRACE_AT(4, j, 7);
       }
       umma_commit(bar_o_final);
       // every MMA of this CTA must be complete before TMEM is released
@@ -366,7 +380,7 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
         const bool masked = tl.lo > 0 || tl.hi < kTile;
         float alpha = 1.f;
         bool need = false;
-        uint32_t pk[64];   // this row of P_t(j), 16-bit pairs
+        uint32_t pa[32], pb[32];   // this row of P_t(j): columns 0-63, 64-127 as 16-bit pairs
         uint64_t acc[4] = {0, 0, 0, 0};
         auto load_half = [&](int h, uint32_t (&r)[64]) {
           tmem_ld_x64_wait(tS + 64 * h, r);
@@ -387,10 +401,10 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
           }
           return fmax3(mx0, mx1, fmaxf(mx2, mx3)) * sl2;
         };
-        // P = 2^(s * sl2 - m_run) in 16-bit pairs into pk[o, o + 32), summed
+        // P = 2^(s * sl2 - m_run) in 16-bit pairs into pk, summed
         // in fp32 into acc. A half can be fully masked (a short last tile of a
         // page), so the first half may leave m_run at -inf.
-        auto exp_half = [&](const uint32_t (&sv)[64], int o) {
+        auto exp_half = [&](const uint32_t (&sv)[64], uint32_t (&pk)[32]) {
           // m_run is -inf only while every column so far was masked: P is 0
           const float mu = m_run == -INFINITY ? 0.f : m_run;
           const uint64_t negm2 = f2_pack(-mu, -mu);
@@ -408,7 +422,7 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
             acc[(c >> 1) & 3] = f2_add(acc[(c >> 1) & 3], e);
             float e0, e1;
             f2_unpack(e, e0, e1);
-            pk[o + (c >> 1)] = pack16<kFP16>(e0, e1);
+            pk[c >> 1] = pack16<kFP16>(e0, e1);
           }
         };
         if (active) {
@@ -421,49 +435,60 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
             m_run = m0;
             need = true;
           }
-          exp_half(r, 0);
-          load_half(1, r);
-          const float m1 = half_max(r);
-          if (m1 > m_run + kRescaleLog2) {
-            // Rare: the second half raised the max past the threshold after
-            // the first half's P was formed. Scale that half (and its sum)
-            // down to the new max; the extra rounding stays at the 16-bit
-            // level of P.
-            const float a2 = ex2_approx(m_run - m1);
-            alpha *= a2;
-            l_run *= a2;
-            m_run = m1;
-            need = true;
-            const uint64_t a22 = f2_pack(a2, a2);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) acc[i] = f2_mul(acc[i], a22);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              float p0, p1;
-              unpack16<kFP16>(pk[i], p0, p1);
-              pk[i] = pack16<kFP16>(p0 * a2, p1 * a2);
-            }
-          }
-          if (kSepP) {   // S_t(j) fully read: the next tile's scores may overwrite it
-            tc_fence_before();
-            mbar_arrive(&bar_s_free[t]);
-          }
-          exp_half(r, 32);
-          float s0, s1;
-          f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), s0, s1);
-          l_run += s0 + s1;
-        } else if (kSepP) {
-          mbar_arrive(&bar_s_free[t]);
+          exp_half(r, pa);
         }
         if (row == 0) PKV_TRACE_AT(t, j, 1);
-        // P_t's columns and O_t are free once PV_t(j-1) is complete
+        // P_t's columns and O_t are free once PV_t(j-1) is complete; the
+        // first half of P goes out now, so its store overlaps the second half
         if (kSepP && j > 0) {
           if (!__all_sync(0xffffffffu, mbar_wait(&bar_pv_done[t], (j - 1) & 1, abort_flag))) { ok = false; break; }
           tc_fence_after();
         }
         if (active) {
-          tmem_st_x32(tP, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-          tmem_st_x32(tP + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+          if (kSepP) tmem_st_x32(tP, pa);
+          uint32_t r[64];
+          load_half(1, r);
+          const float m1 = half_max(r);
+          const bool rare = m1 > m_run + kRescaleLog2;
+          if (__any_sync(0xffffffffu, rare)) {
+            // Rare: the second half raised the max past the threshold after
+            // the first half's P was formed. Scale that half (and its sum)
+            // down to the new max; the extra rounding stays at the 16-bit
+            // level of P. The TMEM accesses are warp-collective, so the
+            // whole warp takes this branch; other rows scale by 1 (exact).
+            float a2 = 1.f;
+            if (rare) {
+              a2 = ex2_approx(m_run - m1);
+              alpha *= a2;
+              l_run *= a2;
+              m_run = m1;
+              need = true;
+            }
+            const uint64_t a22 = f2_pack(a2, a2);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[i] = f2_mul(acc[i], a22);
+            if (kSepP) {
+              tmem_wait_st();
+              tmem_ld_x32_wait(tP, pa);
+            }
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              float p0, p1;
+              unpack16<kFP16>(pa[i], p0, p1);
+              pa[i] = pack16<kFP16>(p0 * a2, p1 * a2);
+            }
+            if (kSepP) tmem_st_x32(tP, pa);
+          }
+          if (kSepP) {   // S_t(j) fully read: the next tile's scores may overwrite it
+            tc_fence_before();
+            mbar_arrive(&bar_s_free[t]);
+          }
+          exp_half(r, pb);
+          float s0, s1;
+          f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), s0, s1);
+          l_run += s0 + s1;
+          if (!kSepP) tmem_st_x32(tP, pa);   // over S_t, now read
+          tmem_st_x32(tP + 32, pb);
           // rescale O_t if the running max moved
           if (j > 0 && __any_sync(0xffffffffu, need)) {
             const uint64_t a2 = f2_pack(alpha, alpha);
@@ -482,6 +507,8 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
             }
           }
           tmem_wait_st();
+        } else if (kSepP) {
+          mbar_arrive(&bar_s_free[t]);
         }
         tc_fence_before();
         if (row == 0) PKV_TRACE_AT(t, j, 2);
@@ -522,12 +549,15 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
         if (store && slot >= 0) a.part_lse[(size_t)slot * kTile + row] = m_run + log2f(l_run);
       }
     }
-  } else if (kTail && has_tail) {
+  } else if (kTail && has_tail && (warp == 8 || warp == 10)) {
     // ------------------------------------------------------------ tail
-    // Warp w takes columns [32 w, 32 w + 32) of every K/V tile: S = Q_tail K^T
-    // as 4 n-tiles x 4 k-steps of m16n8k16, then O += P V as 8 n-tiles x 2
-    // k-steps. Query rows past the tail are zero and never stored.
-    const int w = warp - R::kTail0;
+    // Tail warp w takes columns [64 w, 64 w + 64) of every K/V tile:
+    // S = Q_tail K^T as 8 n-tiles x 4 k-steps of m16n8k16, then O += P V as
+    // 8 n-tiles x 4 k-steps. Query rows past the tail are zero and never
+    // stored.
+    constexpr int kCW = kTile / R::kTailWarps;   // columns per tail warp
+    constexpr int kNI = kCW / 8;                 // S n-tiles
+    const int w = (warp - 8) >> 1;
     const int g = lane >> 2, q4 = lane & 3;
     const float sl2 = a.scale_log2;
     const int row0 = rq.q_row0 + (u.qtile + nq) * kTile;   // first tail row in q/out
@@ -561,13 +591,13 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
       const KvTile tl = tile_at(j);
       const uint32_t ks = k_base + s * L::kTileBytes;
       const uint32_t vs = v_base + s * L::kTileBytes;
-      // S (16 x 32): n-tile i covers K/V rows 32 w + 8 i .. + 7; each ldmatrix
-      // brings the B fragments of two k-steps (16-byte chunks 4 k2 .. + 3)
-      float sc[4][4];
+      // S (16 x kCW): n-tile i covers K/V rows kCW w + 8 i .. + 7; each
+      // ldmatrix brings the B fragments of two k-steps (16-byte chunks 4 k2 .. + 3)
+      float sc[kNI][4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < kNI; ++i) {
         sc[i][0] = sc[i][1] = sc[i][2] = sc[i][3] = 0.f;
-        const int kr = 32 * w + 8 * i + (lane & 7);
+        const int kr = kCW * w + 8 * i + (lane & 7);
 #pragma unroll
         for (int k2 = 0; k2 < D / 32; ++k2) {
           const int ch = 4 * k2 + (lane >> 3);
@@ -577,13 +607,13 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
           mma_16816<kFP16>(sc[i], qa[2 * k2 + 1], b[2], b[3]);
         }
       }
-      // mask columns outside [lo, hi), then the row maxima over this warp's 32 columns
+      // mask columns outside [lo, hi), then the row maxima over this warp's columns
       float mx_a = -INFINITY, mx_b = -INFINITY;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < kNI; ++i) {
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          const int col = 32 * w + 8 * i + 2 * q4 + e;
+          const int col = kCW * w + 8 * i + 2 * q4 + e;
           if (col < tl.lo || col >= tl.hi) sc[i][e] = sc[i][2 + e] = -INFINITY;
         }
         mx_a = fmax3(mx_a, sc[i][0], sc[i][1]);
@@ -609,46 +639,47 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
         for (int n = 0; n < D / 8; ++n) { o[n][2] *= al; o[n][3] *= al; }
         m_b = mx_b;
       }
-      // P as A fragments (k-step kk = columns 16 kk .. + 15 of the warp's 32);
+      // P as A fragments (k-step kk = columns 16 kk .. + 15 of the warp's);
       // while every column so far was masked the max is -inf and P is 0
       const float ma = m_a == -INFINITY ? 0.f : m_a;
       const float mb = m_b == -INFINITY ? 0.f : m_b;
-      uint32_t pa[2][4];
+      uint32_t pf[kNI / 2][4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < kNI; ++i) {
         const float p0 = ex2_approx(fmaf(sc[i][0], sl2, -ma));
         const float p1 = ex2_approx(fmaf(sc[i][1], sl2, -ma));
         const float p2 = ex2_approx(fmaf(sc[i][2], sl2, -mb));
         const float p3 = ex2_approx(fmaf(sc[i][3], sl2, -mb));
         l_a += p0 + p1;
         l_b += p2 + p3;
-        pa[i >> 1][(i & 1) * 2 + 0] = pack16<kFP16>(p0, p1);
-        pa[i >> 1][(i & 1) * 2 + 1] = pack16<kFP16>(p2, p3);
+        pf[i >> 1][(i & 1) * 2 + 0] = pack16<kFP16>(p0, p1);
+        pf[i >> 1][(i & 1) * 2 + 1] = pack16<kFP16>(p2, p3);
       }
-      // O += P V: B fragments by transposed loads of V rows 32 w + 16 kk .. + 15
+      // O += P V: B fragments by transposed loads of V rows kCW w + 16 kk .. + 15
 #pragma unroll
-      for (int kk = 0; kk < 2; ++kk) {
-        const int vr = 32 * w + 16 * kk + (lane & 7) + 8 * ((lane >> 3) & 1);
+      for (int kk = 0; kk < kNI / 2; ++kk) {
+        const int vr = kCW * w + 16 * kk + (lane & 7) + 8 * ((lane >> 3) & 1);
 #pragma unroll
         for (int n2 = 0; n2 < D / 16; ++n2) {
           const int ch = 2 * n2 + (lane >> 4);   // 16-byte chunk = output columns 8 ch .. + 7
           uint32_t b[4];
           ldsm_x4_t(vs + (ch >> 3) * 16384 + vr * 128 + (((ch & 7) ^ (vr & 7)) << 4), b);
-          mma_16816<kFP16>(o[2 * n2], pa[kk], b[0], b[1]);
-          mma_16816<kFP16>(o[2 * n2 + 1], pa[kk], b[2], b[3]);
+          mma_16816<kFP16>(o[2 * n2], pf[kk], b[0], b[1]);
+          mma_16816<kFP16>(o[2 * n2 + 1], pf[kk], b[2], b[3]);
         }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar_kv_empty[s]);
       PKV_TRACE_AT(2, j, 1);
     }
-    // this warp's sums over its 32 columns
+    // this warp's sums over its columns
     l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
     l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
     l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
     l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
-    float* xo = reinterpret_cast<float*>(smem + L::kTailO);    // [4][16][D]
-    float* xm = reinterpret_cast<float*>(smem + L::kTailML);   // [4][16] maxima, then [4][16] sums
+    constexpr int kTW = R::kTailWarps;
+    float* xo = reinterpret_cast<float*>(smem + L::kTailO);    // [kTW][16][D]
+    float* xm = reinterpret_cast<float*>(smem + L::kTailML);   // [kTW][16] maxima, then [kTW][16] sums
 #pragma unroll
     for (int n = 0; n < D / 8; ++n) {
       *reinterpret_cast<float2*>(xo + (w * 16 + g) * D + 8 * n + 2 * q4) = make_float2(o[n][0], o[n][1]);
@@ -657,41 +688,42 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
     if (q4 == 0) {
       xm[w * 16 + g] = m_a;
       xm[w * 16 + g + 8] = m_b;
-      xm[64 + w * 16 + g] = l_a;
-      xm[64 + w * 16 + g + 8] = l_b;
+      xm[kTW * 16 + w * 16 + g] = l_a;
+      xm[kTW * 16 + w * 16 + g + 8] = l_b;
     }
-    named_bar_sync(1, 128);
+    named_bar_sync(1, 32 * kTW);
     ok = __all_sync(0xffffffffu, ok);
-    // merge: thread i of the four warps finishes row i / 8, columns 8 (i % 8) .. + 7
-    const int i = threadIdx.x - 32 * R::kTail0;
-    const int r = i >> 3, c0 = (i & 7) * (D / 8);
+    // merge: thread i of the tail warps finishes row i / 4, columns 16 (i % 4) .. + 15
+    constexpr int kCols = D / 4;
+    const int i = w * 32 + lane;
+    const int r = i >> 2, c0 = (i & 3) * kCols;
     if (ok && r < tail_rows) {
-      float mw[4], M = -INFINITY;
+      float mw[kTW], M = -INFINITY;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < kTW; ++q) {
         mw[q] = xm[q * 16 + r];
         M = fmaxf(M, mw[q]);
       }
-      float wq[4], Lsum = 0.f;
+      float wq[kTW], Lsum = 0.f;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < kTW; ++q) {
         wq[q] = mw[q] == -INFINITY ? 0.f : ex2_approx(mw[q] - M);
-        Lsum += wq[q] * xm[64 + q * 16 + r];
+        Lsum += wq[q] * xm[kTW * 16 + q * 16 + r];
       }
       const float inv = 1.f / Lsum;
-      float res[D / 8];
+      float res[kCols];
 #pragma unroll
-      for (int c = 0; c < D / 8; ++c) {
+      for (int c = 0; c < kCols; ++c) {
         float v = 0.f;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) v = fmaf(wq[q], xo[(q * 16 + r) * D + c0 + c], v);
+        for (int q = 0; q < kTW; ++q) v = fmaf(wq[q], xo[(q * 16 + r) * D + c0 + c], v);
         res[c] = v * inv;
       }
       const int slot = u.slot[nq];
       if (slot < 0) {
         uint16_t* po = reinterpret_cast<uint16_t*>(a.out) + ((size_t)(row0 + r) * a.H + u.head) * D + c0;
 #pragma unroll
-        for (int c = 0; c < D / 8; c += 8) {
+        for (int c = 0; c < kCols; c += 8) {
           uint4 v;
           v.x = pack16<kFP16>(res[c + 0], res[c + 1]);
           v.y = pack16<kFP16>(res[c + 2], res[c + 3]);
@@ -702,7 +734,7 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
       } else {
         float* po = a.part_o + ((size_t)slot * kTile + r) * D + c0;
 #pragma unroll
-        for (int c = 0; c < D / 8; c += 4)
+        for (int c = 0; c < kCols; c += 4)
           *reinterpret_cast<float4*>(po + c) = make_float4(res[c], res[c + 1], res[c + 2], res[c + 3]);
         if (c0 == 0) a.part_lse[(size_t)slot * kTile + r] = M + log2f(Lsum);
       }
