@@ -11,10 +11,13 @@
 // 16-byte vector; consecutive threads move consecutive vectors of a token row,
 // so loads and stores are fully coalesced.
 #include "kernels.h"
+#include "launch.cuh"
 
 namespace pkv {
 
 __global__ void __launch_bounds__(256) append_scatter_kernel(const AppendArgs a) {
+  pdl_wait();      // k/v may come from the previous kernel; the pool from the one before
+  pdl_trigger();   // the attention kernel may set up meanwhile (it waits for this one)
   const long long per_kv = (long long)a.T * a.row_vecs;
   const long long total = 2 * per_kv;
   const uint4* k = reinterpret_cast<const uint4*>(a.k);
@@ -45,8 +48,7 @@ cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream) {
   if (total == 0) return cudaSuccess;
   long long blocks = (total + 255) / 256;
   if (blocks > 148 * 8) blocks = 148 * 8;
-  append_scatter_kernel<<<(int)blocks, 256, 0, stream>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(append_scatter_kernel, dim3((unsigned)blocks), dim3(256), 0, stream, a);
 }
 
 }  // namespace pkv

@@ -45,6 +45,7 @@
 #include <math.h>
 
 #include "kernels.h"
+#include "launch.cuh"
 #include "sm100.cuh"
 
 namespace pkv {
@@ -55,10 +56,15 @@ constexpr int kMaxSmemTiles = 512;   // tile descriptors cached in shared memory
 // Instrumented builds only: per-tile clock64() stamps of each role of CTA 0,
 // read back with kv_debug_trace(). Layout [role 0..5][tile < 64][event < 8].
 __device__ unsigned long long g_pkv_trace[6][64][8];
+// per CTA: globaltimer at entry, after the prologue, at exit; and its SM
+__device__ unsigned long long g_pkv_cta[1024][4];
 #define PKV_TRACE_AT(role, j, ev) \
   do { if (blockIdx.x == 0 && (j) < 64) g_pkv_trace[role][j][ev] = clock64(); } while (0)
+#define PKV_CTA_AT(ev) \
+  do { if (threadIdx.x == 0 && blockIdx.x < 1024) g_pkv_cta[blockIdx.x][ev] = globaltimer_ns(); } while (0)
 #else
 #define PKV_TRACE_AT(role, j, ev) do { } while (0)
+#define PKV_CTA_AT(ev) do { } while (0)
 #endif
 
 template <int D>
@@ -155,6 +161,7 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   KvTile* tile_cache = reinterpret_cast<KvTile*>(smem + L::kTiles);
 
+  PKV_CTA_AT(0);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const KvUnit u = a.units[blockIdx.x];
@@ -200,6 +207,10 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // The setup above overlaps the previous kernel (the frame's K/V append);
+  // the pool and q are read only after it has completed.
+  pdl_wait();
+  PKV_CTA_AT(1);
 
   if (warp == R::kProducer) {
     // ------------------------------------------------------------ producer
@@ -350,6 +361,7 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
         }
       }
       umma_commit(bar_o_final);
+      pdl_trigger();   // the merge kernel may be scheduled (it waits for this grid)
       // every MMA of this CTA must be complete before TMEM is released
       umma_commit(bar_drain);
       mbar_drain_wait(bar_drain, 0);
@@ -749,6 +761,14 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
     tmem_dealloc(tmem, kTmemCols);
   }
   if (threadIdx.x == 0 && *abort_flag) atomicOr(a.err, 1u);
+#ifdef PKV_TRACE
+  if (threadIdx.x == 0 && blockIdx.x < 1024) {
+    uint32_t smid;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    g_pkv_cta[blockIdx.x][3] = smid;
+  }
+#endif
+  PKV_CTA_AT(2);
 }
 
 // Exponentials on the FMA pipe: pair positions {5, 6, 7} of every 8 (37.5 %).
@@ -764,8 +784,7 @@ static cudaError_t launch_attn_t(const AttnMaps& maps, const AttnArgs& a, int n_
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  kern<<<n_units, AttnRoles<D>::kThreads, L::kAlloc, stream>>>(maps, a);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(n_units), dim3(AttnRoles<D>::kThreads), L::kAlloc, stream, maps, a);
 }
 
 cudaError_t launch_attention(const AttnMaps& maps, const AttnArgs& a, int D, bool fp16, int n_units,
@@ -786,6 +805,10 @@ bool attention_tail_ok(int D) { return D == 64; }
 extern "C" int kv_debug_trace(void* host, size_t bytes) {
   if (bytes < sizeof(g_pkv_trace)) return -1;
   return cudaMemcpyFromSymbol(host, g_pkv_trace, sizeof(g_pkv_trace)) == cudaSuccess ? 0 : -7;
+}
+extern "C" int kv_debug_cta(void* host, size_t bytes) {
+  if (bytes < sizeof(g_pkv_cta)) return -1;
+  return cudaMemcpyFromSymbol(host, g_pkv_cta, sizeof(g_pkv_cta)) == cudaSuccess ? 0 : -7;
 }
 #endif
 

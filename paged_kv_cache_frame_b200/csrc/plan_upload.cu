@@ -3,6 +3,7 @@
 // launch), so the upload is asynchronous on the caller's stream, needs no
 // pinned buffer and never waits for earlier work.
 #include "kernels.h"
+#include "launch.cuh"
 
 namespace pkv {
 
@@ -15,6 +16,7 @@ struct UploadChunk {
 
 template <int kWords>
 __global__ void __launch_bounds__(256) plan_upload_kernel(const __grid_constant__ UploadChunk<kWords> c) {
+  pdl_wait();   // earlier kernels may still read the tables this overwrites
   for (int i = threadIdx.x; i < c.n_words; i += blockDim.x) c.dst[i] = c.words[i];
 }
 
@@ -24,8 +26,7 @@ static cudaError_t launch_chunk(uint32_t* dst, const uint32_t* src, int n, cudaS
   c.dst = dst;
   c.n_words = n;
   for (int i = 0; i < n; ++i) c.words[i] = src[i];
-  plan_upload_kernel<kWords><<<1, 256, 0, stream>>>(c);
-  return cudaGetLastError();
+  return launch_pdl(plan_upload_kernel<kWords>, dim3(1), dim3(256), 0, stream, c);
 }
 
 cudaError_t upload_plan(void* dst, const void* src, size_t bytes, cudaStream_t stream) {

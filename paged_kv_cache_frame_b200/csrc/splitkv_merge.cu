@@ -10,6 +10,7 @@
 #include <math.h>
 
 #include "kernels.h"
+#include "launch.cuh"
 #include "sm100.cuh"
 
 namespace pkv {
@@ -29,6 +30,8 @@ template <int D, bool kFP16>
 __global__ void __launch_bounds__(256) splitkv_merge_kernel(const MergeArgs m) {
   constexpr int V = D / 32;   // columns per lane: 2 (D = 64) or 4 (D = 128)
   using Vec = typename VecF<V>::T;
+  pdl_wait();      // the partials come from the attention kernel
+  pdl_trigger();
   const int gwarp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int item = gwarp / kTile;
@@ -94,16 +97,13 @@ cudaError_t launch_merge(const MergeArgs& m, int D, bool fp16, cudaStream_t stre
   if (m.n_items <= 0) return cudaSuccess;
   const long long warps = (long long)m.n_items * kTile;
   const int blocks = (int)((warps * 32 + 255) / 256);
-  if (D == 64) {
-    if (fp16) splitkv_merge_kernel<64, true><<<blocks, 256, 0, stream>>>(m);
-    else splitkv_merge_kernel<64, false><<<blocks, 256, 0, stream>>>(m);
-  } else if (D == 128) {
-    if (fp16) splitkv_merge_kernel<128, true><<<blocks, 256, 0, stream>>>(m);
-    else splitkv_merge_kernel<128, false><<<blocks, 256, 0, stream>>>(m);
-  } else {
-    return cudaErrorInvalidValue;
-  }
-  return cudaGetLastError();
+  if (D == 64)
+    return fp16 ? launch_pdl(splitkv_merge_kernel<64, true>, dim3(blocks), dim3(256), 0, stream, m)
+                : launch_pdl(splitkv_merge_kernel<64, false>, dim3(blocks), dim3(256), 0, stream, m);
+  if (D == 128)
+    return fp16 ? launch_pdl(splitkv_merge_kernel<128, true>, dim3(blocks), dim3(256), 0, stream, m)
+                : launch_pdl(splitkv_merge_kernel<128, false>, dim3(blocks), dim3(256), 0, stream, m);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace pkv
