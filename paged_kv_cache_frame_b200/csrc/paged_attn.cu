@@ -31,8 +31,9 @@
 //                   rows (262 = 2 x 128 + 6 tokens per frame). An M = 128
 //                   tensor-core tile would be almost all padding, so each of
 //                   these warps computes the tail's scores and output for 64 of
-//                   every K/V tile's 128 columns with warp-level mma.sync
-//                   m16n8k16, reading K and V straight from the shared-memory
+//                   every K/V tile's 128 rows with warp-level mma.sync
+//                   m16n8k16, transposed so that the tail rows fill the N = 8
+//                   side, reading K and V straight from the shared-memory
 //                   ring, with its own running max/sum and O in registers. The
 //                   two partial results are merged at the end.
 // TMEM. head_dim 64: S_t at [128 t, +128), P_t at [256 + 64 t, +64), O_t at
@@ -43,6 +44,8 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <math.h>
+
+#include <type_traits>
 
 #include "kernels.h"
 #include "launch.cuh"
@@ -57,11 +60,13 @@ constexpr int kMaxSmemTiles = 512;   // tile descriptors cached in shared memory
 // read back with kv_debug_trace(). Layout [role 0..5][tile < 64][event < 8].
 __device__ unsigned long long g_pkv_trace[6][64][8];
 // per CTA: globaltimer at entry, after the prologue, at exit; and its SM
-__device__ unsigned long long g_pkv_cta[1024][4];
+__device__ unsigned long long g_pkv_cta[1024][6];
 #define PKV_TRACE_AT(role, j, ev) \
   do { if (blockIdx.x == 0 && (j) < 64) g_pkv_trace[role][j][ev] = clock64(); } while (0)
 #define PKV_CTA_AT(ev) \
-  do { if (threadIdx.x == 0 && blockIdx.x < 1024) g_pkv_cta[blockIdx.x][ev] = globaltimer_ns(); } while (0)
+  do { if (threadIdx.x == 0 && blockIdx.x < 1024) { \
+         g_pkv_cta[blockIdx.x][ev] = globaltimer_ns(); \
+         if ((ev) != 1) g_pkv_cta[blockIdx.x][4 + (ev) / 2] = clock64(); } } while (0)
 #else
 #define PKV_TRACE_AT(role, j, ev) do { } while (0)
 #define PKV_CTA_AT(ev) do { } while (0)
@@ -333,8 +338,11 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
           }
           if (progress) {
             t0 = globaltimer_ns();
-          } else if ((spin & 63u) == 0) {
-            if (*abort_flag || globaltimer_ns() - t0 > kWaitLimitNs) {
+          } else {
+            // back off: this warp shares its SM sub-partition with two
+            // softmax warps, whose issue slots a tight poll would take
+            __nanosleep(32);
+            if ((spin & 15u) == 0 && (*abort_flag || globaltimer_ns() - t0 > kWaitLimitNs)) {
               *abort_flag = 1;
               ok = false;
             }
@@ -563,194 +571,223 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
     }
   } else if (kTail && has_tail && (warp == 8 || warp == 10)) {
     // ------------------------------------------------------------ tail
-    // Tail warp w takes columns [64 w, 64 w + 64) of every K/V tile:
-    // S = Q_tail K^T as 8 n-tiles x 4 k-steps of m16n8k16, then O += P V as
-    // 8 n-tiles x 4 k-steps. Query rows past the tail are zero and never
-    // stored.
-    constexpr int kCW = kTile / R::kTailWarps;   // columns per tail warp
-    constexpr int kNI = kCW / 8;                 // S n-tiles
-    const int w = (warp - 8) >> 1;
-    const int g = lane >> 2, q4 = lane & 3;
-    const float sl2 = a.scale_log2;
-    const int row0 = rq.q_row0 + (u.qtile + nq) * kTile;   // first tail row in q/out
-    uint32_t qa[D / 16][4];                                // A fragments of Q_tail
-    {
-      const uint32_t* qg = reinterpret_cast<const uint32_t*>(a.q);
-      const bool va = g < tail_rows, vb = g + 8 < tail_rows;
-      const size_t ra = ((size_t)(row0 + g) * a.H + u.head) * (D / 2);
-      const size_t rb = ((size_t)(row0 + g + 8) * a.H + u.head) * (D / 2);
+    // Tail warp w takes K/V rows [64 w, 64 w + 64) of every tile and works
+    // transposed, so the few tail rows sit in the narrow dimension:
+    // S^T = K Q_tail^T as 4 m-tiles (16 K/V rows) x 4 k-steps x NQ n-tiles
+    // (8 query rows each) of m16n8k16, softmax per query column, then
+    // O^T += V^T P^T (4 m-tiles of 16 output columns x 4 k-steps x NQ). P^T
+    // goes from the accumulator layout to the operand layout with movmatrix.
+    // Query rows past the tail are zero and never stored.
+    auto tail_body = [&](auto nq_tag) {
+      constexpr int NQ = decltype(nq_tag)::value;   // 8-row query groups (1 or 2)
+      constexpr int kCW = kTile / R::kTailWarps;     // K/V rows per tail warp (64)
+      constexpr int kMT = kCW / 16;                  // S^T m-tiles
+      constexpr int kDT = D / 16;                    // O^T m-tiles
+      const int w = (warp - 8) >> 1;
+      const int g = lane >> 2, q4 = lane & 3;
+      const float sl2 = a.scale_log2;
+      const int row0 = rq.q_row0 + (u.qtile + nq) * kTile;   // first tail row in q/out
+      // B fragments of Q_tail^T: query row 8 n + g, columns 16 k + 2 q4 (+8)
+      uint32_t qb[NQ][D / 16][2];
+      {
+        const uint32_t* qg = reinterpret_cast<const uint32_t*>(a.q);
 #pragma unroll
-      for (int k = 0; k < D / 16; ++k) {
-        const int c = 8 * k + q4;   // 32-bit word holding columns 16 k + 2 q4, +1
-        qa[k][0] = va ? qg[ra + c] : 0u;
-        qa[k][1] = vb ? qg[rb + c] : 0u;
-        qa[k][2] = va ? qg[ra + c + 4] : 0u;
-        qa[k][3] = vb ? qg[rb + c + 4] : 0u;
-      }
-    }
-    float o[D / 8][4];   // O_tail fragments: rows g, g + 8; columns 8 n + 2 q4, +1
+        for (int n = 0; n < NQ; ++n) {
+          const bool v = 8 * n + g < tail_rows;
+          const size_t rr = ((size_t)(row0 + 8 * n + g) * a.H + u.head) * (D / 2);
 #pragma unroll
-    for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-    float m_a = -INFINITY, m_b = -INFINITY;   // running maxima of rows g, g + 8 (log2 domain)
-    float l_a = 0.f, l_b = 0.f;               // this lane's share of the running sums
-    const uint32_t k_base = smem_u32(smem + L::kK);
-    const uint32_t v_base = smem_u32(smem + L::kV);
-    bool ok = true;
-    for (int j = 0; j < n_tiles; ++j) {
-      const int s = j % STAGES;
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar_kv_full[s], (j / STAGES) & 1, abort_flag))) { ok = false; break; }
-      PKV_TRACE_AT(2, j, 0);
-      const KvTile tl = tile_at(j);
-      const uint32_t ks = k_base + s * L::kTileBytes;
-      const uint32_t vs = v_base + s * L::kTileBytes;
-      // S (16 x kCW): n-tile i covers K/V rows kCW w + 8 i .. + 7; each
-      // ldmatrix brings the B fragments of two k-steps (16-byte chunks 4 k2 .. + 3)
-      float sc[kNI][4];
-#pragma unroll
-      for (int i = 0; i < kNI; ++i) {
-        sc[i][0] = sc[i][1] = sc[i][2] = sc[i][3] = 0.f;
-        const int kr = kCW * w + 8 * i + (lane & 7);
-#pragma unroll
-        for (int k2 = 0; k2 < D / 32; ++k2) {
-          const int ch = 4 * k2 + (lane >> 3);
-          uint32_t b[4];
-          ldsm_x4(ks + (ch >> 3) * 16384 + kr * 128 + (((ch & 7) ^ (kr & 7)) << 4), b);
-          mma_16816<kFP16>(sc[i], qa[2 * k2], b[0], b[1]);
-          mma_16816<kFP16>(sc[i], qa[2 * k2 + 1], b[2], b[3]);
+          for (int k = 0; k < D / 16; ++k) {
+            qb[n][k][0] = v ? qg[rr + 8 * k + q4] : 0u;
+            qb[n][k][1] = v ? qg[rr + 8 * k + 4 + q4] : 0u;
+          }
         }
       }
-      // mask columns outside [lo, hi), then the row maxima over this warp's columns
-      float mx_a = -INFINITY, mx_b = -INFINITY;
+      float o[kDT][NQ][4];   // O^T: output columns 16 dm + g (+8), query rows 8 n + 2 q4 (+1)
 #pragma unroll
-      for (int i = 0; i < kNI; ++i) {
+      for (int dm = 0; dm < kDT; ++dm)
+#pragma unroll
+        for (int n = 0; n < NQ; ++n) o[dm][n][0] = o[dm][n][1] = o[dm][n][2] = o[dm][n][3] = 0.f;
+      float m_q[NQ][2], l_q[NQ][2];   // per query row 8 n + 2 q4 + e: running max (log2), this lane's sum
+#pragma unroll
+      for (int n = 0; n < NQ; ++n) m_q[n][0] = m_q[n][1] = -INFINITY, l_q[n][0] = l_q[n][1] = 0.f;
+      const uint32_t k_base = smem_u32(smem + L::kK);
+      const uint32_t v_base = smem_u32(smem + L::kV);
+      bool ok = true;
+      for (int j = 0; j < n_tiles; ++j) {
+        const int s = j % STAGES;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar_kv_full[s], (j / STAGES) & 1, abort_flag))) { ok = false; break; }
+        PKV_TRACE_AT(2, j, 0);
+        const KvTile tl = tile_at(j);
+        const uint32_t ks = k_base + s * L::kTileBytes;
+        const uint32_t vs = v_base + s * L::kTileBytes;
+        // S^T: m-tile i = K/V rows kCW w + 16 i .. + 15 (accumulator rows g, g + 8)
+        float sc[kMT][NQ][4];
+#pragma unroll
+        for (int i = 0; i < kMT; ++i) {
+#pragma unroll
+          for (int n = 0; n < NQ; ++n) sc[i][n][0] = sc[i][n][1] = sc[i][n][2] = sc[i][n][3] = 0.f;
+          const int kr = kCW * w + 16 * i + (lane & 7) + 8 * ((lane >> 3) & 1);
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const int ch = 2 * k + (lane >> 4);
+            uint32_t af[4];
+            ldsm_x4(ks + (ch >> 3) * 16384 + kr * 128 + (((ch & 7) ^ (kr & 7)) << 4), af);
+#pragma unroll
+            for (int n = 0; n < NQ; ++n) mma_16816<kFP16>(sc[i][n], af, qb[n][k][0], qb[n][k][1]);
+          }
+          // mask K/V rows outside [lo, hi)
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int kvr = kCW * w + 16 * i + g + 8 * h;
+            if (kvr < tl.lo || kvr >= tl.hi)
+#pragma unroll
+              for (int n = 0; n < NQ; ++n) sc[i][n][2 * h] = sc[i][n][2 * h + 1] = -INFINITY;
+          }
+        }
+        // per query column: max over this warp's K/V rows (lane values, then
+        // the eight lanes with the same q4)
+#pragma unroll
+        for (int n = 0; n < NQ; ++n) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            float mx = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < kMT; ++i) mx = fmax3(mx, sc[i][n][e], sc[i][n][2 + e]);
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+            mx *= sl2;
+            if (mx > m_q[n][e] + kRescaleLog2) {   // never true while every row was masked (-inf)
+              const float al = ex2_approx(m_q[n][e] - mx);
+              l_q[n][e] *= al;
+#pragma unroll
+              for (int dm = 0; dm < kDT; ++dm) { o[dm][n][e] *= al; o[dm][n][2 + e] *= al; }
+              m_q[n][e] = mx;
+            }
+          }
+        }
+        // P^T as B fragments: k-step i = K/V rows 16 i .. + 15 of this warp's
+        // (while every row so far was masked the max is -inf and P is 0)
+        uint32_t pb[kMT][NQ][2];
+#pragma unroll
+        for (int n = 0; n < NQ; ++n) {
+          const float m0 = m_q[n][0] == -INFINITY ? 0.f : m_q[n][0];
+          const float m1 = m_q[n][1] == -INFINITY ? 0.f : m_q[n][1];
+#pragma unroll
+          for (int i = 0; i < kMT; ++i) {
+            const float p0 = ex2_approx(fmaf(sc[i][n][0], sl2, -m0));
+            const float p1 = ex2_approx(fmaf(sc[i][n][1], sl2, -m1));
+            const float p2 = ex2_approx(fmaf(sc[i][n][2], sl2, -m0));
+            const float p3 = ex2_approx(fmaf(sc[i][n][3], sl2, -m1));
+            l_q[n][0] += p0 + p2;
+            l_q[n][1] += p1 + p3;
+            pb[i][n][0] = movmatrix_t(pack16<kFP16>(p0, p1));
+            pb[i][n][1] = movmatrix_t(pack16<kFP16>(p2, p3));
+          }
+        }
+        // O^T += V^T P^T: A fragments by transposed loads of V
+#pragma unroll
+        for (int dm = 0; dm < kDT; ++dm) {
+#pragma unroll
+          for (int i = 0; i < kMT; ++i) {
+            const int vr = kCW * w + 16 * i + (lane & 7) + 8 * (lane >> 4);
+            const int ch = 2 * dm + ((lane >> 3) & 1);
+            uint32_t af[4];
+            ldsm_x4_t(vs + (ch >> 3) * 16384 + vr * 128 + (((ch & 7) ^ (vr & 7)) << 4), af);
+#pragma unroll
+            for (int n = 0; n < NQ; ++n) mma_16816<kFP16>(o[dm][n], af, pb[i][n][0], pb[i][n][1]);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar_kv_empty[s]);
+        PKV_TRACE_AT(2, j, 1);
+      }
+      // this warp's sums per query row
+#pragma unroll
+      for (int n = 0; n < NQ; ++n)
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          const int col = kCW * w + 8 * i + 2 * q4 + e;
-          if (col < tl.lo || col >= tl.hi) sc[i][e] = sc[i][2 + e] = -INFINITY;
+          float v = l_q[n][e];
+          v += __shfl_xor_sync(0xffffffffu, v, 4);
+          v += __shfl_xor_sync(0xffffffffu, v, 8);
+          v += __shfl_xor_sync(0xffffffffu, v, 16);
+          l_q[n][e] = v;
         }
-        mx_a = fmax3(mx_a, sc[i][0], sc[i][1]);
-        mx_b = fmax3(mx_b, sc[i][2], sc[i][3]);
+      constexpr int kTW = R::kTailWarps;
+      float* xo = reinterpret_cast<float*>(smem + L::kTailO);    // [kTW][16 query rows][D]
+      float* xm = reinterpret_cast<float*>(smem + L::kTailML);   // [kTW][16] maxima, then [kTW][16] sums
+#pragma unroll
+      for (int dm = 0; dm < kDT; ++dm)
+#pragma unroll
+        for (int n = 0; n < NQ; ++n)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int qr = 8 * n + 2 * q4 + e;
+            xo[(w * 16 + qr) * D + 16 * dm + g] = o[dm][n][e];
+            xo[(w * 16 + qr) * D + 16 * dm + g + 8] = o[dm][n][2 + e];
+          }
+      if (g == 0) {
+#pragma unroll
+        for (int n = 0; n < NQ; ++n)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            xm[w * 16 + 8 * n + 2 * q4 + e] = m_q[n][e];
+            xm[kTW * 16 + w * 16 + 8 * n + 2 * q4 + e] = l_q[n][e];
+          }
       }
-      mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 1));
-      mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 2));
-      mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 1));
-      mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 2));
-      mx_a *= sl2;
-      mx_b *= sl2;
-      if (mx_a > m_a + kRescaleLog2) {   // never true while every column was masked (-inf)
-        const float al = ex2_approx(m_a - mx_a);
-        l_a *= al;
+      named_bar_sync(1, 32 * kTW);
+      ok = __all_sync(0xffffffffu, ok);
+      // merge: thread i of the tail warps finishes row i / 4, columns 16 (i % 4) .. + 15
+      constexpr int kCols = D / 4;
+      const int i = w * 32 + lane;
+      const int r = i >> 2, c0 = (i & 3) * kCols;
+      if (ok && r < tail_rows) {
+        float mw[kTW], M = -INFINITY;
 #pragma unroll
-        for (int n = 0; n < D / 8; ++n) { o[n][0] *= al; o[n][1] *= al; }
-        m_a = mx_a;
-      }
-      if (mx_b > m_b + kRescaleLog2) {
-        const float al = ex2_approx(m_b - mx_b);
-        l_b *= al;
+        for (int q = 0; q < kTW; ++q) {
+          mw[q] = xm[q * 16 + r];
+          M = fmaxf(M, mw[q]);
+        }
+        float wq[kTW], Lsum = 0.f;
 #pragma unroll
-        for (int n = 0; n < D / 8; ++n) { o[n][2] *= al; o[n][3] *= al; }
-        m_b = mx_b;
-      }
-      // P as A fragments (k-step kk = columns 16 kk .. + 15 of the warp's);
-      // while every column so far was masked the max is -inf and P is 0
-      const float ma = m_a == -INFINITY ? 0.f : m_a;
-      const float mb = m_b == -INFINITY ? 0.f : m_b;
-      uint32_t pf[kNI / 2][4];
+        for (int q = 0; q < kTW; ++q) {
+          wq[q] = mw[q] == -INFINITY ? 0.f : ex2_approx(mw[q] - M);
+          Lsum += wq[q] * xm[kTW * 16 + q * 16 + r];
+        }
+        const float inv = 1.f / Lsum;
+        float res[kCols];
 #pragma unroll
-      for (int i = 0; i < kNI; ++i) {
-        const float p0 = ex2_approx(fmaf(sc[i][0], sl2, -ma));
-        const float p1 = ex2_approx(fmaf(sc[i][1], sl2, -ma));
-        const float p2 = ex2_approx(fmaf(sc[i][2], sl2, -mb));
-        const float p3 = ex2_approx(fmaf(sc[i][3], sl2, -mb));
-        l_a += p0 + p1;
-        l_b += p2 + p3;
-        pf[i >> 1][(i & 1) * 2 + 0] = pack16<kFP16>(p0, p1);
-        pf[i >> 1][(i & 1) * 2 + 1] = pack16<kFP16>(p2, p3);
-      }
-      // O += P V: B fragments by transposed loads of V rows kCW w + 16 kk .. + 15
+        for (int c = 0; c < kCols; ++c) {
+          float v = 0.f;
 #pragma unroll
-      for (int kk = 0; kk < kNI / 2; ++kk) {
-        const int vr = kCW * w + 16 * kk + (lane & 7) + 8 * ((lane >> 3) & 1);
+          for (int q = 0; q < kTW; ++q) v = fmaf(wq[q], xo[(q * 16 + r) * D + c0 + c], v);
+          res[c] = v * inv;
+        }
+        const int slot = u.slot[nq];
+        if (slot < 0) {
+          uint16_t* po = reinterpret_cast<uint16_t*>(a.out) + ((size_t)(row0 + r) * a.H + u.head) * D + c0;
 #pragma unroll
-        for (int n2 = 0; n2 < D / 16; ++n2) {
-          const int ch = 2 * n2 + (lane >> 4);   // 16-byte chunk = output columns 8 ch .. + 7
-          uint32_t b[4];
-          ldsm_x4_t(vs + (ch >> 3) * 16384 + vr * 128 + (((ch & 7) ^ (vr & 7)) << 4), b);
-          mma_16816<kFP16>(o[2 * n2], pf[kk], b[0], b[1]);
-          mma_16816<kFP16>(o[2 * n2 + 1], pf[kk], b[2], b[3]);
+          for (int c = 0; c < kCols; c += 8) {
+            uint4 v;
+            v.x = pack16<kFP16>(res[c + 0], res[c + 1]);
+            v.y = pack16<kFP16>(res[c + 2], res[c + 3]);
+            v.z = pack16<kFP16>(res[c + 4], res[c + 5]);
+            v.w = pack16<kFP16>(res[c + 6], res[c + 7]);
+            *reinterpret_cast<uint4*>(po + c) = v;
+          }
+        } else {
+          float* po = a.part_o + ((size_t)slot * kTile + r) * D + c0;
+#pragma unroll
+          for (int c = 0; c < kCols; c += 4)
+            *reinterpret_cast<float4*>(po + c) = make_float4(res[c], res[c + 1], res[c + 2], res[c + 3]);
+          if (c0 == 0) a.part_lse[(size_t)slot * kTile + r] = M + log2f(Lsum);
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar_kv_empty[s]);
-      PKV_TRACE_AT(2, j, 1);
-    }
-    // this warp's sums over its columns
-    l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
-    l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
-    l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
-    l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
-    constexpr int kTW = R::kTailWarps;
-    float* xo = reinterpret_cast<float*>(smem + L::kTailO);    // [kTW][16][D]
-    float* xm = reinterpret_cast<float*>(smem + L::kTailML);   // [kTW][16] maxima, then [kTW][16] sums
-#pragma unroll
-    for (int n = 0; n < D / 8; ++n) {
-      *reinterpret_cast<float2*>(xo + (w * 16 + g) * D + 8 * n + 2 * q4) = make_float2(o[n][0], o[n][1]);
-      *reinterpret_cast<float2*>(xo + (w * 16 + g + 8) * D + 8 * n + 2 * q4) = make_float2(o[n][2], o[n][3]);
-    }
-    if (q4 == 0) {
-      xm[w * 16 + g] = m_a;
-      xm[w * 16 + g + 8] = m_b;
-      xm[kTW * 16 + w * 16 + g] = l_a;
-      xm[kTW * 16 + w * 16 + g + 8] = l_b;
-    }
-    named_bar_sync(1, 32 * kTW);
-    ok = __all_sync(0xffffffffu, ok);
-    // merge: thread i of the tail warps finishes row i / 4, columns 16 (i % 4) .. + 15
-    constexpr int kCols = D / 4;
-    const int i = w * 32 + lane;
-    const int r = i >> 2, c0 = (i & 3) * kCols;
-    if (ok && r < tail_rows) {
-      float mw[kTW], M = -INFINITY;
-#pragma unroll
-      for (int q = 0; q < kTW; ++q) {
-        mw[q] = xm[q * 16 + r];
-        M = fmaxf(M, mw[q]);
-      }
-      float wq[kTW], Lsum = 0.f;
-#pragma unroll
-      for (int q = 0; q < kTW; ++q) {
-        wq[q] = mw[q] == -INFINITY ? 0.f : ex2_approx(mw[q] - M);
-        Lsum += wq[q] * xm[kTW * 16 + q * 16 + r];
-      }
-      const float inv = 1.f / Lsum;
-      float res[kCols];
-#pragma unroll
-      for (int c = 0; c < kCols; ++c) {
-        float v = 0.f;
-#pragma unroll
-        for (int q = 0; q < kTW; ++q) v = fmaf(wq[q], xo[(q * 16 + r) * D + c0 + c], v);
-        res[c] = v * inv;
-      }
-      const int slot = u.slot[nq];
-      if (slot < 0) {
-        uint16_t* po = reinterpret_cast<uint16_t*>(a.out) + ((size_t)(row0 + r) * a.H + u.head) * D + c0;
-#pragma unroll
-        for (int c = 0; c < kCols; c += 8) {
-          uint4 v;
-          v.x = pack16<kFP16>(res[c + 0], res[c + 1]);
-          v.y = pack16<kFP16>(res[c + 2], res[c + 3]);
-          v.z = pack16<kFP16>(res[c + 4], res[c + 5]);
-          v.w = pack16<kFP16>(res[c + 6], res[c + 7]);
-          *reinterpret_cast<uint4*>(po + c) = v;
-        }
-      } else {
-        float* po = a.part_o + ((size_t)slot * kTile + r) * D + c0;
-#pragma unroll
-        for (int c = 0; c < kCols; c += 4)
-          *reinterpret_cast<float4*>(po + c) = make_float4(res[c], res[c + 1], res[c + 2], res[c + 3]);
-        if (c0 == 0) a.part_lse[(size_t)slot * kTile + r] = M + log2f(Lsum);
-      }
-    }
+    };
+    if (tail_rows <= 8)
+      tail_body(std::integral_constant<int, 1>{});
+    else
+      tail_body(std::integral_constant<int, 2>{});
   }
 
   tc_fence_before();
@@ -771,8 +808,8 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
   PKV_CTA_AT(2);
 }
 
-// Exponentials on the FMA pipe: pair positions {5, 6, 7} of every 8 (37.5 %).
-constexpr uint32_t kEmu = 0xE0u;
+// Exponentials on the FMA pipe: pair positions {6, 7} of every 8 (25 %).
+constexpr uint32_t kEmu = 0xC0u;
 
 template <int D, bool kFP16, int STAGES>
 static cudaError_t launch_attn_t(const AttnMaps& maps, const AttnArgs& a, int n_units, cudaStream_t stream) {

@@ -311,4 +311,12 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
                : "memory");
 }
 
+// Transpose of an 8x8 16-bit matrix held one row pair per lane (lane l:
+// row l / 4, columns 2 (l % 4), +1) across the warp.
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t a) {
+  uint32_t d;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+  return d;
+}
+
 }  // namespace pkv
