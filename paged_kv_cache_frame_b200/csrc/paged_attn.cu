@@ -448,6 +448,7 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
         if (active) {
           uint32_t r[64];
           load_half(0, r);
+          if (row == 0) PKV_TRACE_AT(t, j, 3);
           const float m0 = half_max(r);
           if (m0 > m_run + kRescaleLog2) {
             alpha = ex2_approx(m_run - m0);   // 0 on the first tile (m_run = -inf)
@@ -464,10 +465,12 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
           if (!__all_sync(0xffffffffu, mbar_wait(&bar_pv_done[t], (j - 1) & 1, abort_flag))) { ok = false; break; }
           tc_fence_after();
         }
+        if (row == 0) PKV_TRACE_AT(t, j, 4);
         if (active) {
           if (kSepP) tmem_st_x32(tP, pa);
           uint32_t r[64];
           load_half(1, r);
+          if (row == 0) PKV_TRACE_AT(t, j, 5);
           const float m1 = half_max(r);
           const bool rare = m1 > m_run + kRescaleLog2;
           if (__any_sync(0xffffffffu, rare)) {
@@ -526,12 +529,14 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
               tmem_st_x16(tO + c, o);
             }
           }
+          if (row == 0) PKV_TRACE_AT(t, j, 6);
           tmem_wait_st();
         } else if (kSepP) {
           mbar_arrive(&bar_s_free[t]);
         }
         tc_fence_before();
         if (row == 0) PKV_TRACE_AT(t, j, 2);
+        if ((row & 31) == 0) PKV_TRACE_AT(3, j, 4 * t + (row >> 5));   // each warp's arrival
         mbar_arrive(&bar_p_full[t]);
       }
       ok = __all_sync(0xffffffffu, ok);
