@@ -358,9 +358,13 @@ int build_plan(const std::vector<const PageState*>& st, const PlanInputs& in, Ho
     *why = "plan: split schedule exceeds the workspace's partial slots";
     return KV_ERR_CAPACITY;
   }
-  // Launch order: the chunks of one (request, head) sit next to each other so
-  // that co-resident CTAs share K/V tiles in L2.
+  // Launch order: the block scheduler starts CTAs in index order over a few
+  // microseconds, so the longest chunks go first (no two CTAs read the same
+  // K/V tile, so the order costs no L2 reuse); ties keep (request, head,
+  // first tile) order.
   std::stable_sort(P.units.begin(), P.units.end(), [](const KvUnit& a, const KvUnit& b) {
+    const int la = a.tile_end - a.tile_begin, lb = b.tile_end - b.tile_begin;
+    if (la != lb) return la > lb;
     if (a.req != b.req) return a.req < b.req;
     if (a.head != b.head) return a.head < b.head;
     if (a.tile_begin != b.tile_begin) return a.tile_begin < b.tile_begin;
