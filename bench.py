@@ -170,6 +170,9 @@ class StreamRunner:
         self.launches = 0
         self._elt = elt
 
+    frames_per_pass = property(lambda self: self.wl.frames)
+    steps_per_pass = property(lambda self: self.wl.frames)
+
     def _chk(self, rc, what):
         if rc != 0:
             raise self.capi.KVError(rc, what, self.L.kv_last_error().decode())
@@ -231,6 +234,101 @@ class StreamRunner:
         return launches
 
 
+class BatchRunner:
+    """Several streams of different ages planned together (one kv_plan over
+    all caches per frame step, their query rows concatenated), as in the
+    batched workload. A pass is `steps` frame steps of every stream; the
+    streams keep growing from pass to pass."""
+
+    def __init__(self, wl, seed, steps, passes, ring=4):
+        import torch
+        import paged_kv_cache_frame_b200 as pkv
+        from paged_kv_cache_frame_b200 import capi
+        self.torch, self.pkv, self.capi = torch, pkv, capi
+        self.L = capi.lib()
+        self.wl, self.ring_n, self.steps = wl, ring, steps
+        self.stream = torch.cuda.current_stream()
+        self.sp = self.stream.cuda_stream
+        self.ages = workload.stream_ages(wl, seed)
+        span = int(self.ages.max()) + steps * passes
+        sp_pages = max(1, math.ceil(wl.NS * span / wl.page_size))
+        self.caches = [pkv.PagedKVCache(wl.patch_pages + sp_pages, wl.page_size, wl.H, wl.D, wl.S, wl.W,
+                                        num_blocks=wl.blocks, num_special=wl.NS, dtype=wl.dtype)
+                       for _ in range(wl.streams)]
+        for c in self.caches:
+            c.allocate_pools("cuda")
+        self.h = [c.handle for c in self.caches]
+        self.cache_arr = (ctypes.c_void_p * wl.streams)(*self.h)
+        self.ws = torch.empty(pkv.workspace_bytes(self.caches), dtype=torch.uint8, device="cuda")
+        self.ring = workload.qkv_ring_cuda(wl, seed, ring)            # [R, B, 3, streams*T, H, D]
+        self.out = torch.empty((wl.blocks, wl.streams * wl.T, wl.H, wl.D), dtype=wl.torch_dtype(), device="cuda")
+        row = wl.T * wl.H * wl.D * self.ring.element_size()
+        self.ptr = [[[self.ring[r, b, i].data_ptr() for i in range(3)] for b in range(wl.blocks)]
+                    for r in range(ring)]
+        self.row = row
+        self.optr = [self.out[b].data_ptr() for b in range(wl.blocks)]
+        self.ws_ptr, self.ws_bytes = self.ws.data_ptr(), self.ws.numel()
+        self.stats = []
+        # warm every stream to its age: page state only (metadata appends)
+        # (a frame step closes once every block has been appended)
+        for h, age in zip(self.h, self.ages):
+            for _ in range(int(age)):
+                for b in range(wl.blocks):
+                    self._chk(self.L.kv_append_frame(h, b, None, None, None), "warm append")
+                self._chk(self.L.kv_evict_frames(h), "warm evict")
+
+    frames_per_pass = property(lambda self: self.steps * self.wl.streams)
+    steps_per_pass = property(lambda self: self.steps)
+
+    def _chk(self, rc, what):
+        if rc != 0:
+            raise self.capi.KVError(rc, what, self.L.kv_last_error().decode())
+
+    def one_pass(self, events=None, host=None):
+        torch, L, wl, sp = self.torch, self.L, self.wl, self.sp
+        plan = ctypes.c_void_p()
+        self.stats = []
+        launches = 0
+        for f in range(self.steps):
+            r = f % self.ring_n
+            if host is not None:
+                hring, hout, dstage = host
+                dstage.copy_(hring[r], non_blocking=True)
+                ptr = [[dstage[b, i].data_ptr() for i in range(3)] for b in range(wl.blocks)]
+            else:
+                ptr = self.ptr[r]
+            for b in range(wl.blocks):
+                q, k, v = ptr[b]
+                for si, h in enumerate(self.h):
+                    self._chk(L.kv_append_frame(h, b, k + si * self.row, v + si * self.row, sp), "append")
+                    launches += 1
+                if b == 0:
+                    for h in self.h:
+                        self._chk(L.kv_evict_frames(h), "evict")
+                    if plan.value:
+                        L.kv_plan_free(plan)
+                    self._chk(L.kv_plan(ctypes.byref(plan), self.cache_arr, wl.streams, 0, self.ws_ptr,
+                                        self.ws_bytes, sp), "plan")
+                    st = self.capi.kv_plan_stats()
+                    L.kv_plan_get_stats(plan, ctypes.byref(st))
+                    launches += 1
+                    self.stats.append((st.visible_tokens, st.n_split_units))
+                if events is not None:
+                    e0 = torch.cuda.Event(enable_timing=True)
+                    e1 = torch.cuda.Event(enable_timing=True)
+                    e0.record(self.stream)
+                self._chk(L.kv_run(plan, b, q, self.optr[b], sp), "run")
+                launches += 1 + (1 if self.stats[-1][1] else 0)
+                if events is not None:
+                    e1.record(self.stream)
+                    events.append((e0, e1))
+            if host is not None:
+                hout[r].copy_(self.out, non_blocking=True)
+        if plan.value:
+            L.kv_plan_free(plan)
+        return launches
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -249,7 +347,11 @@ def run_gpu(args):
         import dataclasses
         wl = dataclasses.replace(wl, name=wl.name + "-profiling-case", frames=args.frames or wl.frames,
                                  blocks=args.blocks or wl.blocks)
-    runner = StreamRunner(wl, seed=args.seed + 1000 * rank)
+    if wl.streams > 1:
+        runner = BatchRunner(wl, seed=args.seed + 1000 * rank, steps=wl.steps,
+                             passes=args.warmup + 2 * args.steps + 3)
+    else:
+        runner = StreamRunner(wl, seed=args.seed + 1000 * rank)
     torch.cuda.synchronize()
 
     def barrier():
@@ -286,7 +388,7 @@ def run_gpu(args):
     if world > 1:
         dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
     ms_max = float(ms_t.item())
-    frames_total = args.steps * wl.frames * world
+    frames_total = args.steps * runner.frames_per_pass * world
     value = frames_total / (ms_max / 1e3)
 
     # per-call attention time (run = attention + merge) against the roofline
@@ -328,33 +430,56 @@ def run_gpu(args):
         if world > 1:
             dist.all_reduce(ems, op=dist.ReduceOp.MAX)
         e2e = {"value": frames_total / (float(ems.item()) / 1e3), "unit": "frames/s",
-               "h2d_bytes_per_step": int(dstage.numel() * dstage.element_size() * wl.frames),
-               "d2h_bytes_per_step": int(runner.out.numel() * runner.out.element_size() * wl.frames)}
+               "h2d_bytes_per_step": int(dstage.numel() * dstage.element_size() * runner.steps_per_pass),
+               "d2h_bytes_per_step": int(runner.out.numel() * runner.out.element_size() * runner.steps_per_pass)}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(wl, args.seed, budget_s=args.cpu_budget)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and wl.streams == 1:
+        cpu = cpu_baseline(wl, args.seed, budget_s=args.cpu_budget,
+                           frames_sample=tuple(sorted({0, min(71, wl.frames - 1), wl.frames // 2, wl.frames - 1})))
+
+    # steady state: frame steps whose window is full (more than S + W frames)
+    steady = [i for i in range(len(lkvs)) if i >= wl.S + wl.W] if wl.streams == 1 else list(range(len(lkvs)))
+    if steady:
+        st_ms = sum(run_ms[i * wl.blocks + b] for i in steady for b in range(wl.blocks))
+        st_fl = sum(call_flops(wl.T, lkvs[i], wl.H, wl.D) for i in steady) * wl.blocks
+        steady_tflops = st_fl / (st_ms / 1e3) / 1e12
+    else:
+        steady_tflops = None
 
     if rank == 0:
+        if args.workload == 1:
+            metric = "frames/s (24-block stack) at 224x224, 320 frames"
+        elif wl.streams > 1:
+            metric = f"frames/s ({wl.streams} streams x {wl.blocks}-block stack), {wl.name}"
+        else:
+            metric = f"frames/s ({wl.blocks}-block stack), {wl.name}"
+        config = {"workload": wl.name, "frames": wl.frames, "blocks": wl.blocks, "H": wl.H,
+                  "D": wl.D, "tokens_per_frame": wl.T, "page_size": wl.page_size,
+                  "scale_frames": wl.S, "window": wl.W, "keyframes": wl.keyframes,
+                  "parallelism": f"replicas x{world}",
+                  "l2": "inputs larger than L2 (one pool per block, all read every frame step)"}
+        if wl.streams > 1:
+            config.update({"streams": wl.streams, "stream_ages": [int(x) for x in runner.ages],
+                           "frame_steps_per_pass": runner.steps, "frames": None})
         line = {
-            "metric": "frames/s (24-block stack) at 224x224, 320 frames",
+            "metric": metric,
             "profiling_case_not_a_bench_value": profiling_case or None,
             "value": round(value, 2), "unit": "frames/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
-            "data": "synthetic (seeded N(0,1) Q/K/V, ring of 16 frame sets in HBM)",
-            "config": {"workload": wl.name, "frames": wl.frames, "blocks": wl.blocks, "H": wl.H,
-                       "D": wl.D, "tokens_per_frame": wl.T, "page_size": wl.page_size,
-                       "scale_frames": wl.S, "window": wl.W, "keyframes": wl.keyframes,
-                       "parallelism": f"replicas x{world}",
-                       "l2": "inputs larger than L2 (24 block pools, 1.9 GB, read every frame)"},
+            "data": f"synthetic (seeded N(0,1) Q/K/V, ring of {runner.ring_n} frame sets in HBM)",
+            "config": config,
             "attention": {"tflops": round(tflops, 2), "kv_gbs": round(gbs, 1),
                           "roofline_frac": round(roof_frac, 4),
+                          "frac_of_burst_peak": round(tflops / pk["bf16_tflops"], 4),
+                          "steady_state_tflops": round(steady_tflops, 2) if steady_tflops else None,
                           "roofline_ms_per_pass": round(t_roof * 1e3, 3),
                           "run_ms_per_pass": round(run_s * 1e3, 3)},
             "roofline": {"bound": "tensor", "achieved": round(tflops, 2),
                          "peak": peak_tf, "unit": "TFLOP/s",
-                         "frac": round(tflops / peak_tf, 4), "traffic": measured_traffic(),
+                         "frac": round(tflops / peak_tf, 4),
+                         "traffic": measured_traffic() if args.workload == 1 else None,
                          "peak_kind": f"{pk_kind} bf16 dense sustained (kernel timed inside a long step)",
                          "kernel": "paged_prefill_attn + splitkv_merge (kv_run), event-timed per call in one extra pass"},
             "gpu_launches": launches,

@@ -214,8 +214,11 @@ class PagedKVCache:
     def __del__(self):
         h = getattr(self, "handle", None)
         if h:
-            kv_destroy(h)
             self.handle = None
+            try:
+                kv_destroy(h)
+            except Exception:   # interpreter shutdown: the library may already be gone
+                pass
 
     def pool_bytes(self) -> int:
         return kv_pool_bytes(self.handle)
@@ -274,8 +277,11 @@ class Plan:
     def __del__(self):
         h = getattr(self, "handle", None)
         if h:
-            kv_plan_free(h)
             self.handle = None
+            try:
+                kv_plan_free(h)
+            except Exception:   # interpreter shutdown: the library may already be gone
+                pass
 
     def run(self, block, q, out=None, stream=None):
         if out is None:
