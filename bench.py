@@ -84,6 +84,27 @@ def call_kv_bytes(lkv, H, D, elt=2):
     return 2.0 * lkv * H * D * elt
 
 
+# ------------------------------------------------------------------ ranks
+def replica_seed(seed, rank):
+    """Each rank runs an independent replica stream with its own inputs."""
+    return seed + 1000 * rank
+
+
+def max_over_ranks(x, world, device="cpu"):
+    """The max of a per-rank number over all ranks (every rank gets it)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank, world, ms_max):
+    """Units processed by all ranks per second of the slowest rank."""
+    return units_per_rank * world / (ms_max / 1e3)
+
+
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
     def __init__(self, index):
@@ -348,10 +369,10 @@ def run_gpu(args):
         wl = dataclasses.replace(wl, name=wl.name + "-profiling-case", frames=args.frames or wl.frames,
                                  blocks=args.blocks or wl.blocks)
     if wl.streams > 1:
-        runner = BatchRunner(wl, seed=args.seed + 1000 * rank, steps=wl.steps,
+        runner = BatchRunner(wl, seed=replica_seed(args.seed, rank), steps=wl.steps,
                              passes=args.warmup + 2 * args.steps + 3)
     else:
-        runner = StreamRunner(wl, seed=args.seed + 1000 * rank)
+        runner = StreamRunner(wl, seed=replica_seed(args.seed, rank))
     torch.cuda.synchronize()
 
     def barrier():
@@ -383,13 +404,9 @@ def run_gpu(args):
     # passes, so they are recorded only here.)
     runner.one_pass(events=events)
     torch.cuda.synchronize()
-    ms = t0.elapsed_time(t1)
-    ms_t = torch.tensor([ms], device="cuda")
-    if world > 1:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
+    ms_max = max_over_ranks(t0.elapsed_time(t1), world, "cuda")
     frames_total = args.steps * runner.frames_per_pass * world
-    value = frames_total / (ms_max / 1e3)
+    value = whole_job_rate(args.steps * runner.frames_per_pass, world, ms_max)
 
     # per-call attention time (run = attention + merge) against the roofline
     run_ms = [a.elapsed_time(b) for a, b in events]
@@ -426,10 +443,8 @@ def run_gpu(args):
         b.record()
         torch.cuda.synchronize()
         barrier()
-        ems = torch.tensor([a.elapsed_time(b)], device="cuda")
-        if world > 1:
-            dist.all_reduce(ems, op=dist.ReduceOp.MAX)
-        e2e = {"value": frames_total / (float(ems.item()) / 1e3), "unit": "frames/s",
+        ems = max_over_ranks(a.elapsed_time(b), world, "cuda")
+        e2e = {"value": whole_job_rate(args.steps * runner.frames_per_pass, world, ems), "unit": "frames/s",
                "h2d_bytes_per_step": int(dstage.numel() * dstage.element_size() * runner.steps_per_pass),
                "d2h_bytes_per_step": int(runner.out.numel() * runner.out.element_size() * runner.steps_per_pass)}
 
