@@ -508,7 +508,7 @@ def run_gpu(args):
 
 
 # ------------------------------------------------------------------ oracle arm
-def cpu_baseline(wl, seed, budget_s=20.0, frames_sample=(0, 71, 159, 319), rows=48):
+def cpu_baseline(wl, seed, budget_s=20.0, frames_sample=(0, 71, 159, 319), rows=None):
     """Times the CPU oracle (float64 dense attention) on a bounded sample of
     the workload and extrapolates frames/s by FLOPs."""
     sys.path.insert(0, os.path.join(ROOT, "tests"))
@@ -523,6 +523,7 @@ def cpu_baseline(wl, seed, budget_s=20.0, frames_sample=(0, 71, 159, 319), rows=
 
     so = StreamOracle(wl.S, wl.W, wl.NS, wl.P, wl.dtype, fetch)
     rng = np.random.default_rng(seed)
+    rows = wl.T if rows is None else rows   # all query rows by default (about 10-15 s on one core)
     sel = sorted(rng.choice(wl.T, size=min(rows, wl.T), replace=False).tolist())
     t_att, fl = 0.0, 0.0
     done = []

@@ -42,6 +42,33 @@ def assert_close(out, want, what=""):
     return mx, mean
 
 
+def dense_fp32(cache, plan, block, q, stream_idx=0):
+    """Every row and head of the frame's attention in fp32 on the GPU: the
+    visible pages of `plan`'s table gathered densely from the block's pool
+    (a check on the kernel at full size, next to the oracle's sampled rows)."""
+    pool = cache.pools[block]                       # [max_pages, 2, page_size, H, D]
+    table, lpl = plan.page_table(stream_idx)
+    idx = torch.as_tensor(table, device=pool.device, dtype=torch.long)
+    kv = pool.index_select(0, idx).float()          # [n_pages, 2, page_size, H, D]
+    n = len(table)
+    k = kv[:, 0].reshape(n * cache.page_size, cache.H, cache.D)[: (n - 1) * cache.page_size + lpl]
+    v = kv[:, 1].reshape(n * cache.page_size, cache.H, cache.D)[: (n - 1) * cache.page_size + lpl]
+    out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    scale = cache.D ** -0.5
+    for h in range(cache.H):   # one head at a time keeps the score matrix small
+        s_ = (q[:, h].float() @ k[:, h].T) * scale
+        out[:, h] = torch.softmax(s_, dim=-1) @ v[:, h]
+    return out
+
+
+def assert_close_dense(out, want, what=""):
+    d = (out.float() - want).abs()
+    mx, mean = float(d.max()), float(d.mean())
+    assert np.isfinite(mx), f"{what}: non-finite output"
+    assert mx <= MAX_ABS and mean <= MEAN_ABS, f"{what}: max {mx:.3e} mean {mean:.3e}"
+    return mx, mean
+
+
 def new_cache(pkv, wl, num_blocks=1, patch_pages=0):
     max_pages = (patch_pages or wl.patch_pages) + wl.special_pages
     c = pkv.PagedKVCache(max_pages, wl.page_size, wl.H, wl.D, wl.S, wl.W, num_blocks=num_blocks,
@@ -55,11 +82,12 @@ def workspace(pkv, caches):
 
 
 def run_stream(pkv, wl, seed, n_frames, check, rows=None, defer=None, keep=None,
-               tiles_per_split=0, patch_pages=0, collect=None):
+               tiles_per_split=0, patch_pages=0, collect=None, dense=()):
     """Append frames 0..n_frames-1 of block 0; at frames in `check`, plan + run
     and compare the chosen query rows with the oracle. defer[f] / keep[f]:
     frame f is appended with eviction deferred and then committed (keep) or
-    rolled back. Returns {frame: (max_err, mean_err)}."""
+    rolled back. At frames in `dense`, every row is also checked against the
+    fp32 dense gather of the visible pages. Returns {frame: (max_err, mean_err)}."""
     fr = Frames(wl, seed)
     cache = new_cache(pkv, wl, patch_pages=patch_pages)
     ws = workspace(pkv, [cache])
@@ -78,6 +106,8 @@ def run_stream(pkv, wl, seed, n_frames, check, rows=None, defer=None, keep=None,
             plan.check_device()
             sel = slice(None) if rows is None else torch.as_tensor(rows)
             res[f] = assert_close(out[sel], so.expected(rows), f"frame {f}")
+            if f in dense:
+                assert_close_dense(out, dense_fp32(cache, plan, 0, q), f"frame {f} (all rows, fp32 dense)")
             if collect is not None:
                 collect[f] = out.clone()
         if d:
