@@ -13,7 +13,10 @@ Rules, each from the pages:
     never evicted ([P1] "Special Stream (Append-Only)"; [P2] "Special Stream
     (Append-Only)": six tokens per frame). With cross-frame special retention
     on (the default, [P2] "Configuration Parameters"), the special tokens of
-    evicted frames stay visible.
+    evicted frames stay visible; with it off, only the special tokens of
+    frames whose patches are still visible are ([P2] "Configuration
+    Parameters": kv_cache_cross_frame_special retains the special tokens of
+    evicted frames).
   * Scale frames are the first S committed frames and stay resident for good
     ([P2] "Patch Stream (Recyclable)": first kv_cache_scale_frames frames
     remain permanently resident).
@@ -29,8 +32,9 @@ from __future__ import annotations
 
 
 class FrameListSim:
-    def __init__(self, S: int, W: int, NS: int = 6):
+    def __init__(self, S: int, W: int, NS: int = 6, cross_frame_special: bool = True):
         self.S, self.W, self.NS = S, W, NS
+        self.cross_frame_special = cross_frame_special
         self.C: list[int] = []
         self.resident: list[int] = []
         self.pending: int | None = None
@@ -82,10 +86,17 @@ class FrameListSim:
         """Frames whose patch tokens are visible, oldest first."""
         return self.resident + ([self.pending] if self.pending is not None else [])
 
+    def visible_specials(self) -> list[tuple[int, int]]:
+        """Visible special tokens as (frame, slot), in stream order."""
+        if self.cross_frame_special:
+            return list(self.SP)
+        live = set(self.patch_frames())
+        return [(f, j) for (f, j) in self.SP if f in live]
+
     def visible_tokens(self, P: int) -> set:
         """Visible tokens as ('p', frame, patch_index) / ('s', frame, slot)."""
         out = {("p", f, t) for f in self.patch_frames() for t in range(P)}
-        out.update(("s", f, j) for (f, j) in self.SP)
+        out.update(("s", f, j) for (f, j) in self.visible_specials())
         return out
 
     def snapshot(self):

@@ -22,6 +22,13 @@ Table Attention"): scale pages in frame order, window pages oldest to newest,
 then the pending page if any, then special pages Np .. Np+k-1. Only the last
 page may be partial; last_page_len is the fill of the last special page.
 
+Without cross-frame special retention ([P2] "Configuration Parameters"), the
+special tokens of evicted frames drop out: the visible special tokens are the
+runs of the frames whose patches are visible. Evictions always take the
+oldest window frame, so those runs form at most two ranges of the stream
+(the scale frames' and the window's), and the table lists only special pages
+that hold a visible token.
+
 get_cache_stats keys ([P3] "Monitoring Cache Statistics"): frame_count,
 scale_pages, live_pages, free_pages, special_tokens.
 """
@@ -38,8 +45,9 @@ class OracleError(Exception):
 
 class PageModel:
     def __init__(self, S: int, W: int, page_size: int, max_pages: int,
-                 NS: int = 6, patch_pages: int | None = None):
+                 NS: int = 6, patch_pages: int | None = None, cross_frame_special: bool = True):
         self.S, self.W, self.ps, self.NS = S, W, page_size, NS
+        self.cross_frame_special = cross_frame_special
         self.Np = patch_pages if patch_pages else S + W + 1
         if self.Np < 1 or max_pages < self.Np + (1 if NS > 0 else 0):
             raise OracleError("CAPACITY", "pool too small")
@@ -128,18 +136,26 @@ class PageModel:
             out = out + [self.pending]
         return out
 
+    def visible_special_index(self) -> list[int]:
+        """Stream indices j of the visible special tokens, ascending."""
+        if self.cross_frame_special:
+            return list(range(self.sp_len))
+        live = {f for f, _ in self.patch_pages_visible()}
+        return [j for j in range(self.sp_len) if self.sp_owner[j][0] in live]
+
     def page_table(self) -> tuple[list[int], int]:
         """(kv_indices, last_page_len) of the visible page table."""
         if self.committed == 0 and self.pending is None:
             raise OracleError("EMPTY")
         patch = [p for _, p in self.patch_pages_visible()]
         k = -(-self.sp_len // self.ps)
-        special = [self.Np + i for i in range(k)]
+        pages = sorted({j // self.ps for j in self.visible_special_index()})
+        special = [self.Np + i for i in pages]
         last = self.sp_len - self.ps * (k - 1) if k else self.ps
         return patch + special, last
 
     def visible_token_count(self) -> int:
-        return len(self.patch_pages_visible()) * self.ps + self.sp_len
+        return len(self.patch_pages_visible()) * self.ps + len(self.visible_special_index())
 
     def stats(self) -> dict:
         pend = 1 if self.pending is not None else 0
@@ -160,13 +176,14 @@ class PageModel:
         slot is mapped to the frame that wrote it."""
         table, last = self.page_table()
         owner = {p: f for f, p in self.patch_pages_visible()}
+        vis = set(self.visible_special_index())
         out = set()
         for n, p in enumerate(table):
             cnt = last if n == len(table) - 1 else self.ps
             for t in range(cnt):
                 if p < self.Np:
                     out.add(("p", owner[p], t))
-                else:
+                elif (p - self.Np) * self.ps + t in vis:
                     out.add(("s",) + self.sp_owner[(p - self.Np) * self.ps + t])
         return out
 

@@ -5,7 +5,8 @@ Test infrastructure only (see the package docstring).
 Drives the frame-list simulator (`frames.FrameListSim`) through a stream and
 gathers the visible K/V straight from each frame's own tensors, with no pages
 involved, so that it checks the paged path from the outside: patch tokens of
-every visible frame, then all cached special tokens. Attention does not
+every visible frame, then the visible special tokens (all of them with
+cross-frame special retention, else those of the visible frames). Attention does not
 depend on the order of the visible tokens.
 
 Per frame step ([P1] "Runtime Flow for Frame Processing"; [P2] "Flow-Based
@@ -30,8 +31,8 @@ def bits16(t) -> np.ndarray:
 class StreamOracle:
     """fetch(frame) -> (q, k, v) as [T, H, D] uint16 bit patterns."""
 
-    def __init__(self, S: int, W: int, NS: int, P: int, dtype: str, fetch):
-        self.sim = FrameListSim(S, W, NS)
+    def __init__(self, S: int, W: int, NS: int, P: int, dtype: str, fetch, cross_frame_special: bool = True):
+        self.sim = FrameListSim(S, W, NS, cross_frame_special)
         self.NS, self.P, self.dtype, self.fetch = NS, P, dtype, fetch
         self.patch_kv: dict[int, tuple[np.ndarray, np.ndarray]] = {}
         self.special_kv: dict[int, tuple[np.ndarray, np.ndarray]] = {}
@@ -75,7 +76,7 @@ class StreamOracle:
             k, v = self.patch_kv[f]
             ks.append(k)
             vs.append(v)
-        for f, j in self.sim.SP:
+        for f, j in self.sim.visible_specials():
             k, v = self.special_kv[f]
             ks.append(k[j:j + 1])
             vs.append(v[j:j + 1])

@@ -152,11 +152,11 @@ OPS = st.lists(st.sampled_from(["key", "key", "key", "defer_keep", "defer_drop",
 
 
 @settings(max_examples=150, deadline=None)
-@given(ops=OPS, S=st.integers(0, 3), W=st.integers(0, 4), ps=st.sampled_from([1, 5, 16]))
-def test_page_model_matches_frame_list(ops, S, W, ps):
+@given(ops=OPS, S=st.integers(0, 3), W=st.integers(0, 4), ps=st.sampled_from([1, 5, 16]), xs=st.booleans())
+def test_page_model_matches_frame_list(ops, S, W, ps, xs):
     NS = 6
-    m = PageModel(S, W, ps, max_pages=S + W + 1 + (NS * 64) // ps + 2, NS=NS)
-    sim = FrameListSim(S, W, NS)
+    m = PageModel(S, W, ps, max_pages=S + W + 1 + (NS * 64) // ps + 2, NS=NS, cross_frame_special=xs)
+    sim = FrameListSim(S, W, NS, cross_frame_special=xs)
     f = 0
     for op in ops:
         if op == "evict":
@@ -222,3 +222,41 @@ def test_deferred_frame_is_visible_on_top_of_full_window():
     assert [f for f, _ in m.patch_pages_visible()] == [0, 1, 7, 8, 9, 10]
     m.commit()                                 # commit runs the eviction
     assert [f for f, _ in m.patch_pages_visible()] == [0, 1, 8, 9, 10]
+
+
+def test_cross_frame_special_off_worked_example():
+    """Tiny config (page 16, S=2, W=4), 12 frames, specials of evicted frames
+    dropped: frames 0, 1 (scale) and 8..11 (window) stay, so the visible
+    special stream indices are [0, 12) and [48, 72): special pages 0, 3 and 4
+    (16 slots each), the last one holding 72 - 64 = 8 tokens. Worked by hand."""
+    m = PageModel(2, 4, 16, max_pages=7 + 5, NS=6, cross_frame_special=False)
+    sim = FrameListSim(2, 4, 6, cross_frame_special=False)
+    for f in range(12):
+        m.append(f); m.evict()
+        sim.append(f); sim.evict()
+    table, lpl = m.page_table()
+    Np = 7
+    # pages 0..6 go to frames 0..6; from frame 6 on each append evicts the
+    # oldest window frame (2, 3, ...) and the next frame reuses its page, so
+    # frames 8..11 sit on pages 3, 4, 5, 6
+    assert table[:6] == [0, 1, 3, 4, 5, 6]
+    assert table[6:] == [Np + 0, Np + 3, Np + 4] and lpl == 8
+    assert m.visible_special_index() == list(range(12)) + list(range(48, 72))
+    assert m.visible_token_count() == 6 * 16 + 6 * 6
+    assert m.visible_tokens() == sim.visible_tokens(16)
+
+
+@pytest.mark.parametrize("S,W", [(0, 3), (2, 4), (8, 64)])
+def test_cross_frame_special_off_closed_form(S, W):
+    """Every visible frame keeps exactly its NS special tokens and no other
+    frame's: visible tokens = (frames visible) x (P + NS)."""
+    P, NS = 16, 6
+    on, off = FrameListSim(S, W, NS), FrameListSim(S, W, NS, cross_frame_special=False)
+    for n in range(1, 3 * (S + W) + 5):
+        for sim in (on, off):
+            sim.append(n - 1); sim.evict()
+        frames = min(n, S) + min(max(n - S, 0), W)
+        assert len(off.visible_tokens(P)) == frames * (P + NS)
+        assert len(on.visible_tokens(P)) == frames * P + NS * n
+        if n <= S + W:   # nothing evicted yet: the two settings agree
+            assert off.visible_tokens(P) == on.visible_tokens(P)
