@@ -174,7 +174,8 @@ class StreamRunner:
         self.stream = torch.cuda.current_stream()
         self.sp = self.stream.cuda_stream
         self.cache = pkv.PagedKVCache(wl.max_pages, wl.page_size, wl.H, wl.D, wl.S, wl.W,
-                                      num_blocks=wl.blocks, num_special=wl.NS, dtype=wl.dtype)
+                                      num_blocks=wl.blocks, num_special=wl.NS, dtype=wl.dtype,
+                                      cross_frame_special=wl.cross_special)
         self.cache.allocate_pools("cuda")
         self.h = self.cache.handle
         self.ws = torch.empty(pkv.workspace_bytes([self.cache]), dtype=torch.uint8, device="cuda")
@@ -472,6 +473,7 @@ def run_gpu(args):
         config = {"workload": wl.name, "frames": wl.frames, "blocks": wl.blocks, "H": wl.H,
                   "D": wl.D, "tokens_per_frame": wl.T, "page_size": wl.page_size,
                   "scale_frames": wl.S, "window": wl.W, "keyframes": wl.keyframes,
+                  "cross_frame_special": wl.cross_special,
                   "parallelism": f"replicas x{world}",
                   "l2": "inputs larger than L2 (one pool per block, all read every frame step)"}
         if wl.streams > 1:
@@ -521,7 +523,7 @@ def cpu_baseline(wl, seed, budget_s=20.0, frames_sample=(0, 71, 159, 319), rows=
             fr_cache[f] = tuple(bits16(x) for x in workload.frame_qkv(wl, seed, f, 0))
         return fr_cache[f]
 
-    so = StreamOracle(wl.S, wl.W, wl.NS, wl.P, wl.dtype, fetch)
+    so = StreamOracle(wl.S, wl.W, wl.NS, wl.P, wl.dtype, fetch, cross_frame_special=wl.cross_special)
     rng = np.random.default_rng(seed)
     rows = wl.T if rows is None else rows   # all query rows by default (about 10-15 s on one core)
     sel = sorted(rng.choice(wl.T, size=min(rows, wl.T), replace=False).tolist())
@@ -533,7 +535,7 @@ def cpu_baseline(wl, seed, budget_s=20.0, frames_sample=(0, 71, 159, 319), rows=
             t = time.perf_counter()
             so.expected(sel)
             dt = time.perf_counter() - t
-            lkv = len(so.sim.patch_frames()) * wl.P + len(so.sim.SP)
+            lkv = len(so.sim.patch_frames()) * wl.P + len(so.sim.visible_specials())
             t_att += dt
             fl += call_flops(len(sel), lkv, wl.H, wl.D)
             done.append(f)
@@ -541,7 +543,8 @@ def cpu_baseline(wl, seed, budget_s=20.0, frames_sample=(0, 71, 159, 319), rows=
                 break
     gflops = fl / t_att / 1e9
     # whole-workload FLOPs: every frame, every block
-    sim_l = [min(n, wl.S + wl.W) * wl.P + wl.NS * n for n in range(1, wl.frames + 1)]
+    sim_l = [min(n, wl.S + wl.W) * wl.P + wl.NS * (n if wl.cross_special else min(n, wl.S + wl.W))
+             for n in range(1, wl.frames + 1)]
     total = sum(call_flops(wl.T, l, wl.H, wl.D) for l in sim_l) * wl.blocks
     fps = wl.frames / (total / (gflops * 1e9))
     threads = 1   # numpy einsum without BLAS runs on one thread
@@ -585,7 +588,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=3)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", type=int, default=1, choices=[1, 2, 3, 4])
+    ap.add_argument("--workload", type=int, default=1, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--seed", type=int, default=1)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")

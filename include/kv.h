@@ -242,6 +242,18 @@ int kv_plan_get_stats(const kv_plan_t* plan, kv_plan_stats* out);
  * word. KV_OK, KV_ERR_DEVICE_CHECK (bit set by a kernel) or KV_ERR_CUDA. */
 int kv_check_device(const kv_plan_t* plan, void* stream);
 
+/* kv_set_cross_frame_special -- kv_cache_cross_frame_special ([P2]
+ * "Configuration Parameters"): on (1, the default) keeps the special tokens of
+ * evicted frames visible; off (0) leaves visible only the special tokens of
+ * frames whose patch tokens are (scale, window and pending frames). Evictions
+ * take the oldest window frame, so the hidden tokens form one range of the
+ * special stream and the K/V tiles skip it; kv_get_page_table then lists only
+ * special pages that hold a visible token. Takes effect for the next kv_plan
+ * (plans made before it become stale). include_scale_frames=False of the same
+ * section is scale_frames = 0 in kv_init.
+ * Errors: KV_ERR_ARG (NULL cache). */
+int kv_set_cross_frame_special(kv_cache_t* cache, int on);
+
 /* Size of the library-owned device array that kv_run_static uses as scratch. */
 #define KV_STATIC_SCRATCH_BYTES (32u << 20)
 

@@ -30,7 +30,7 @@ __all__ = [
     "kv_evict_frames", "kv_defer_eviction", "kv_commit_frame", "kv_rollback_last_frame",
     "kv_get_stats", "kv_get_free_list", "kv_workspace_bytes", "kv_plan", "kv_run",
     "kv_plan_free", "kv_get_page_table", "kv_get_kv_tiles", "kv_plan_get_stats",
-    "kv_check_device", "kv_strerror", "kv_last_error", "kv_run_static",
+    "kv_check_device", "kv_strerror", "kv_last_error", "kv_run_static", "kv_set_cross_frame_special",
 ]
 
 
@@ -99,6 +99,10 @@ def kv_commit_frame(c) -> None:
 
 def kv_rollback_last_frame(c) -> None:
     capi.check(capi.lib().kv_rollback_last_frame(c), "kv_rollback_last_frame")
+
+
+def kv_set_cross_frame_special(c, on) -> None:
+    capi.check(capi.lib().kv_set_cross_frame_special(c, int(bool(on))), "kv_set_cross_frame_special")
 
 
 def kv_get_stats(c) -> dict:
@@ -201,7 +205,7 @@ class PagedKVCache:
     """One video stream's paged cache (all transformer blocks)."""
 
     def __init__(self, max_pages, page_size, num_heads, head_dim, scale_frames=8, window=64,
-                 num_blocks=1, num_special=6, dtype="bf16", patch_pages=0):
+                 num_blocks=1, num_special=6, dtype="bf16", patch_pages=0, cross_frame_special=True):
         self.dtype = dtype
         code = KV_FP16 if dtype in ("fp16", "float16") or str(dtype) == "torch.float16" else KV_BF16
         self.handle = kv_init(max_pages, page_size, num_heads, head_dim, scale_frames, window,
@@ -210,6 +214,8 @@ class PagedKVCache:
         self.H, self.D, self.num_blocks, self.NS = num_heads, head_dim, num_blocks, num_special
         self.T = page_size + num_special
         self.pools = [None] * num_blocks
+        if not cross_frame_special:
+            kv_set_cross_frame_special(self.handle, False)
 
     def __del__(self):
         h = getattr(self, "handle", None)

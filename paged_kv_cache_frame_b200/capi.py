@@ -84,6 +84,7 @@ SIGNATURES = {
     "kv_plan_get_stats": (_I, [_P, ctypes.POINTER(kv_plan_stats)]),
     "kv_check_device": (_I, [_P, _P]),
     "kv_run_static": (_I, [ctypes.POINTER(_P), _I, _I, _I, _P, _P, _I, _P]),
+    "kv_set_cross_frame_special": (_I, [_P, _I]),
     "kv_strerror": (ctypes.c_char_p, [_I]),
     "kv_last_error": (ctypes.c_char_p, []),
 }

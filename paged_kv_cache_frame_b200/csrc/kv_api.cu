@@ -231,6 +231,16 @@ int kv_get_stats(const kv_cache_t* c, kv_stats* out) {
   return KV_OK;
 }
 
+int kv_set_cross_frame_special(kv_cache_t* c, int on) {
+  if (!c) return fail(KV_ERR_ARG, "kv_set_cross_frame_special: NULL cache");
+  const bool v = on != 0;
+  if (c->st.cross_special != v) {
+    c->st.cross_special = v;
+    ++c->st.epoch;
+  }
+  return KV_OK;
+}
+
 int kv_get_free_list(const kv_cache_t* c, int* ids, int cap, int* n) {
   if (!c || !n || cap < 0 || (cap > 0 && !ids)) return fail(KV_ERR_ARG, "kv_get_free_list: bad argument");
   const auto& f = c->st.free_;

@@ -83,7 +83,7 @@ int PageState::append(int block, int* page, int* sp0, std::string* why) {
     step_sp0 = sp_len;
     sp_len += cfg.NS;
     step_page = pg;
-    const FramePage fp{next_frame++, pg};
+    const FramePage fp{next_frame++, pg, step_sp0};
     if (defer) {
       has_pending = true;
       pending_ = fp;
@@ -161,43 +161,76 @@ int PageState::rollback(std::string* why) {
   return KV_OK;
 }
 
-int PageState::page_table(std::vector<int>* idx, int* last_page_len) const {
+void PageState::special_gap(int* g0, int* g1) const {
+  *g0 = *g1 = 0;
+  if (cross_special) return;
+  const int a = cfg.NS * (int)scale_.size();
+  const int b = !window_.empty() ? window_.front().sp0 : has_pending ? pending_.sp0 : sp_len;
+  if (b > a) {
+    *g0 = a;
+    *g1 = b;
+  }
+}
+
+int PageState::visible_runs(std::vector<PageRun>* runs) const {
   if (committed == 0 && !has_pending) return KV_ERR_EMPTY;
+  runs->clear();
+  const int ps = cfg.page_size;
+  for (const auto& fp : scale_) runs->push_back({fp.page, 0, ps});
+  for (const auto& fp : window_) runs->push_back({fp.page, 0, ps});
+  if (has_pending) runs->push_back({pending_.page, 0, ps});
+  int g0, g1;
+  special_gap(&g0, &g1);
+  const int k = ceil_div(sp_len, ps);
+  for (int i = 0; i < k; ++i) {
+    const int a = i * ps, b = std::min(sp_len, a + ps);   // this page's tokens [a, b) of the stream
+    // visible parts: [a, b) minus the hidden range [g0, g1)
+    const bool gap = g1 > g0;
+    const int pieces[2][2] = {{a, gap ? std::min(b, g0) : b}, {gap ? std::max(a, g1) : b, b}};
+    for (const auto& pc : pieces)
+      if (pc[1] > pc[0]) runs->push_back({cfg.Np + i, pc[0] - a, pc[1] - a});
+  }
+  return KV_OK;
+}
+
+int PageState::page_table(std::vector<int>* idx, int* last_page_len) const {
+  std::vector<PageRun> runs;
+  const int rc = visible_runs(&runs);
+  if (rc != KV_OK) return rc;
   idx->clear();
-  for (const auto& fp : scale_) idx->push_back(fp.page);
-  for (const auto& fp : window_) idx->push_back(fp.page);
-  if (has_pending) idx->push_back(pending_.page);
+  for (const PageRun& r : runs)
+    if (idx->empty() || idx->back() != r.page) idx->push_back(r.page);
   const int ps = cfg.page_size;
   const int k = ceil_div(sp_len, ps);
-  for (int i = 0; i < k; ++i) idx->push_back(cfg.Np + i);
   *last_page_len = k ? sp_len - ps * (k - 1) : ps;
   return KV_OK;
 }
 
 long long PageState::visible_tokens() const {
   const long long patch = (long long)scale_.size() + (long long)window_.size() + (has_pending ? 1 : 0);
-  return patch * cfg.page_size + sp_len;
+  int g0, g1;
+  special_gap(&g0, &g1);
+  return patch * cfg.page_size + sp_len - (g1 - g0);
 }
 
-void build_tiles(const std::vector<int>& table, int last_page_len, int page_size,
-                 std::vector<KvTile>* tiles) {
-  const int n = (int)table.size();
-  for (int i = 0; i < n; ++i) {
-    const int count = (i == n - 1) ? last_page_len : page_size;
-    const int base = table[i] * 2 * page_size;
-    for (int t0 = 0; t0 < count; t0 += kTile) {
-      const int nn = std::min(kTile, count - t0);
+void build_tiles(const std::vector<PageRun>& runs, int page_size, std::vector<KvTile>* tiles) {
+  for (const PageRun& r : runs) {
+    const int base = r.page * 2 * page_size;
+    for (int s = r.lo; s < r.hi; s += kTile) {
+      const int e = std::min(s + kTile, r.hi);
       KvTile t;
-      if (nn == kTile) {
-        t.row = base + t0; t.lo = 0; t.hi = kTile;
-      } else if (count >= kTile) {
-        // ragged end of a long page: anchor the box at the page's last valid
-        // row so no row outside the page is read; the first rows repeat the
-        // previous tile and are masked
-        t.row = base + count - kTile; t.lo = (int16_t)(kTile - nn); t.hi = kTile;
+      if (e - s == kTile) {
+        t.row = base + s; t.lo = 0; t.hi = kTile;
+      } else if (page_size >= kTile) {
+        // the box stays inside the page: anchored at the run's last row when
+        // it can be, else at the page's first row; rows outside [s, e) are
+        // masked (for the ragged end of a long page they repeat the
+        // previous tile)
+        const int row0 = e >= kTile ? e - kTile : 0;
+        t.row = base + row0; t.lo = (int16_t)(s - row0); t.hi = (int16_t)(e - row0);
       } else {
-        // a page shorter than one tile: the box runs past it, rows >= count masked
-        t.row = base; t.lo = 0; t.hi = (int16_t)nn;
+        // a page shorter than one tile: the box runs past it, rows >= e masked
+        t.row = base; t.lo = (int16_t)s; t.hi = (int16_t)e;
       }
       tiles->push_back(t);
     }
@@ -214,7 +247,7 @@ WorkspaceLayout workspace_layout(const std::vector<const PageState*>& st) {
     const Config& c = s->cfg;
     const int T = c.page_size + c.NS;
     units_base += (size_t)c.H * ceil_div(T, kTile);
-    tiles_cap += (size_t)c.max_pages * ceil_div(c.page_size, kTile);
+    tiles_cap += (size_t)c.max_pages * ceil_div(c.page_size, kTile) + 2;   // + the gap's split page
     D = c.D;
   }
   L.slot_cap = 2 * (units_base + kMaxTargetCtas);
@@ -249,8 +282,10 @@ int build_plan(const std::vector<const PageState*>& st, const PlanInputs& in, Ho
       *why = "plan: a stream has no frame yet";
       return rc;
     }
+    std::vector<PageRun> runs;
+    s->visible_runs(&runs);
     tile0[r] = (int)P.tiles.size();
-    build_tiles(table, lpl, s->cfg.page_size, &P.tiles);
+    build_tiles(runs, s->cfg.page_size, &P.tiles);
     KvReq rq;
     rq.q_row0 = q_row0;
     rq.T = s->cfg.page_size + s->cfg.NS;

@@ -14,7 +14,12 @@
 //     [Np, max_pages): token j sits on page Np + j / page_size, slot
 //     j % page_size;
 //   - a frame appended while eviction is deferred stays pending until it is
-//     committed or rolled back.
+//     committed or rolled back;
+//   - without cross-frame special retention ([P2] "Configuration
+//     Parameters"), the special tokens of evicted frames are not visible.
+//     Evictions take the oldest window frame, so the hidden tokens form one
+//     range of the special stream, between the scale frames' and the
+//     window's.
 // (The pages are titled "How the Paged KV Cache Attention Mechanism Enables
 // Long Sequence Inference in LingBot-Map" [P1] and "KV Cache Mechanism in
 // LingBot-Map for Streaming Inference: A Deep Dive" [P2].)
@@ -31,6 +36,13 @@ namespace pkv {
 struct FramePage {
   int frame;
   int page;
+  int sp0;   // the frame's first token in the special stream
+};
+
+// A visible range [lo, hi) of rows of one pool page.
+struct PageRun {
+  int page;
+  int lo, hi;
 };
 
 struct Config {
@@ -49,6 +61,7 @@ class PageState {
   int committed = 0;
   int next_frame = 0;
   bool defer = false;
+  bool cross_special = true;   // special tokens of evicted frames stay visible
   // frame step
   bool step_open = false;
   std::vector<uint8_t> appended;
@@ -68,6 +81,11 @@ class PageState {
   int commit(std::string* why);
   int rollback(std::string* why);
   int page_table(std::vector<int>* idx, int* last_page_len) const;
+  // Hidden range [g0, g1) of the special stream (empty unless cross-frame
+  // special retention is off and frames have been evicted).
+  void special_gap(int* g0, int* g1) const;
+  // The visible rows, page by page, in page-table order.
+  int visible_runs(std::vector<PageRun>* runs) const;
   int special_capacity() const { return (cfg.max_pages - cfg.Np) * cfg.page_size; }
   bool is_appended(int block) const {
     return step_open && block >= 0 && block < cfg.B && appended[block];
@@ -108,9 +126,8 @@ struct WorkspaceLayout {
 
 WorkspaceLayout workspace_layout(const std::vector<const PageState*>& st);
 
-// Builds the K/V tile list of one visible page table.
-void build_tiles(const std::vector<int>& table, int last_page_len, int page_size,
-                 std::vector<KvTile>* tiles);
+// Builds the K/V tile list of one stream's visible rows.
+void build_tiles(const std::vector<PageRun>& runs, int page_size, std::vector<KvTile>* tiles);
 
 int build_plan(const std::vector<const PageState*>& st, const PlanInputs& in, HostPlan* out,
                std::string* why);

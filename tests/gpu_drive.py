@@ -69,10 +69,11 @@ def assert_close_dense(out, want, what=""):
     return mx, mean
 
 
-def new_cache(pkv, wl, num_blocks=1, patch_pages=0):
+def new_cache(pkv, wl, num_blocks=1, patch_pages=0, cross_special=True):
     max_pages = (patch_pages or wl.patch_pages) + wl.special_pages
     c = pkv.PagedKVCache(max_pages, wl.page_size, wl.H, wl.D, wl.S, wl.W, num_blocks=num_blocks,
-                         num_special=wl.NS, dtype=wl.dtype, patch_pages=patch_pages)
+                         num_special=wl.NS, dtype=wl.dtype, patch_pages=patch_pages,
+                         cross_frame_special=cross_special)
     c.allocate_pools("cuda")
     return c
 
@@ -82,16 +83,16 @@ def workspace(pkv, caches):
 
 
 def run_stream(pkv, wl, seed, n_frames, check, rows=None, defer=None, keep=None,
-               tiles_per_split=0, patch_pages=0, collect=None, dense=()):
+               tiles_per_split=0, patch_pages=0, collect=None, dense=(), cross_special=True):
     """Append frames 0..n_frames-1 of block 0; at frames in `check`, plan + run
     and compare the chosen query rows with the oracle. defer[f] / keep[f]:
     frame f is appended with eviction deferred and then committed (keep) or
     rolled back. At frames in `dense`, every row is also checked against the
     fp32 dense gather of the visible pages. Returns {frame: (max_err, mean_err)}."""
     fr = Frames(wl, seed)
-    cache = new_cache(pkv, wl, patch_pages=patch_pages)
+    cache = new_cache(pkv, wl, patch_pages=patch_pages, cross_special=cross_special)
     ws = workspace(pkv, [cache])
-    so = StreamOracle(wl.S, wl.W, wl.NS, wl.P, wl.dtype, fr.bits)
+    so = StreamOracle(wl.S, wl.W, wl.NS, wl.P, wl.dtype, fr.bits, cross_frame_special=cross_special)
     res = {}
     for f in range(n_frames):
         q, k, v = (x.cuda() for x in fr.get(f))

@@ -175,12 +175,13 @@ OPS = st.lists(st.sampled_from(["key", "key", "key", "defer_keep", "defer_drop",
 
 @settings(max_examples=120, deadline=None)
 @given(ops=OPS, S=st.integers(0, 3), W=st.integers(0, 4), ps=st.sampled_from([1, 5, 16, 130]),
-       B=st.integers(1, 3))
-def test_state_machine_bit_exact_vs_oracle(pkv, ops, S, W, ps, B):
+       B=st.integers(1, 3), xs=st.booleans())
+def test_state_machine_bit_exact_vs_oracle(pkv, ops, S, W, ps, B, xs):
     NS = 6
     max_pages = S + W + 1 + (NS * 60) // ps + 2
-    m = PageModel(S, W, ps, max_pages, NS=NS)
+    m = PageModel(S, W, ps, max_pages, NS=NS, cross_frame_special=xs)
     h = mk(pkv, S, W, ps, max_pages, B=B)
+    pkv.kv_set_cross_frame_special(h, xs)
     E = pkv.capi
     try:
         f = 0
@@ -249,22 +250,23 @@ def tile_cover(tiles, ps):
     return out
 
 
-@pytest.mark.parametrize("ps,n", [(16, 12), (256, 320), (999, 30), (130, 40), (128, 9), (64, 100)])
-def test_kv_tiles_cover_visible_tokens_exactly_once(pkv, ps, n):
+@pytest.mark.parametrize("xs", [True, False])
+@pytest.mark.parametrize("ps,n", [(16, 12), (256, 320), (999, 30), (130, 40), (128, 9), (64, 100),
+                                  (16, 200), (300, 150)])
+def test_kv_tiles_cover_visible_tokens_exactly_once(pkv, ps, n, xs):
     S, W = 8, 64
     pages = math.ceil(6 * n / ps) + 1
     h = mk(pkv, S, W, ps, 73 + pages)
-    m = PageModel(S, W, ps, 73 + pages)
+    pkv.kv_set_cross_frame_special(h, xs)
+    m = PageModel(S, W, ps, 73 + pages, cross_frame_special=xs)
     for f in range(n):
         step(pkv, h)
         m.append(f); m.evict()
     p = pkv.kv_plan([h])
     tiles = pkv.kv_get_kv_tiles(p)
-    tbl, last = m.page_table()
-    want = []
-    for i, pg in enumerate(tbl):
-        cnt = last if i == len(tbl) - 1 else ps
-        want += [(pg, t) for t in range(cnt)]
+    assert pkv.kv_get_page_table(p) == m.page_table()
+    want = [(pg, t) for _, pg in m.patch_pages_visible() for t in range(ps)]
+    want += [(m.Np + j // ps, j % ps) for j in m.visible_special_index()]
     got = tile_cover(tiles, ps)
     assert sorted(got) == sorted(want)
     for row, lo, hi in tiles:

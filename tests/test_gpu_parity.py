@@ -198,6 +198,30 @@ def sample_rows(T, seed, n=24):
     return sorted(set([0, 1, 5, T - 1, 128, 255, 256, T - 6]) | set(rng.integers(0, T, n).tolist()))
 
 
+def test_cross_frame_special_off_tiny_every_frame(pkv):
+    """kv_cache_cross_frame_special = False: evicted frames' special tokens
+    leave the visible set (a hidden range that starts and ends inside pages)."""
+    wl = dataclasses.replace(W0, frames=30)
+    res = run_stream(pkv, wl, seed=41, n_frames=wl.frames, check=set(range(wl.frames)), cross_special=False)
+    assert len(res) == wl.frames
+
+
+def test_cross_frame_special_off_224_with_keyframes(pkv):
+    wl = dataclasses.replace(workload.WORKLOADS[2], frames=110)
+    keep = workload.keyframe_mask(wl, seed=42)
+    run_stream(pkv, wl, seed=42, n_frames=wl.frames, check={8, 72, 80, 109}, rows=sample_rows(wl.T, 42),
+               defer=np.ones(wl.frames, dtype=bool), keep=keep, cross_special=False, dense={109})
+
+
+def test_include_scale_frames_off_is_zero_scale_frames(pkv):
+    """kv_cache_include_scale_frames = False is scale_frames = 0: a pure
+    sliding window of W frames."""
+    run_stream(pkv, dataclasses.replace(W0, S=0, frames=20), seed=43, n_frames=20, check=set(range(20)))
+    wl = dataclasses.replace(workload.WORKLOADS[1], S=0, frames=90)
+    run_stream(pkv, wl, seed=44, n_frames=wl.frames, check={63, 64, 89}, rows=sample_rows(wl.T, 44),
+               dense={89})
+
+
 def test_full_224_stream_block0_sampled(pkv):
     wl = workload.WORKLOADS[1]
     run_stream(pkv, wl, seed=1, n_frames=wl.frames, check={0, 71, 72, 159, 319},

@@ -51,6 +51,7 @@ class Workload:
     age_lo: int = 0         # batched: seeded stream ages in [age_lo, age_hi]
     age_hi: int = 0
     steps: int = 0          # batched: timed steps after warming to the ages
+    cross_special: bool = True   # special tokens of evicted frames stay visible
 
     @property
     def T(self) -> int:
@@ -85,6 +86,8 @@ WORKLOADS = {
     3: Workload("518x378-1000f", H=16, D=64, P=999, page_size=999, S=8, W=64, blocks=24, frames=1000),
     4: Workload("batched-8x-ragged", H=8, D=128, P=256, page_size=256, S=8, W=64, blocks=24,
                 frames=0, dtype="fp16", streams=8, age_lo=10, age_hi=600, steps=32),
+    5: Workload("224x224-320f-no-cross-frame-special", H=16, D=64, P=256, page_size=256, S=8, W=64,
+                blocks=24, frames=320, cross_special=False),
 }
 
 
