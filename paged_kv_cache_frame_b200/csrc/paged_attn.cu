@@ -11,36 +11,42 @@
 // Enables Long Sequence Inference in LingBot-Map", [P3] "FlashInfer Paged KV
 // Cache Performance Benefits in LingBot-Map".)
 //
-// Roles (head_dim 64: 384 threads; head_dim 128: 320):
-//   warps 0-3, 4-7  softmax warpgroups, one per 128-row query tile. Thread i
-//                   owns query row i == TMEM lane i. Per K/V tile it reads its
-//                   S row once, in two 64-column halves, keeps the running
-//                   max/sum in the log2 domain, writes P (16-bit) to TMEM and
-//                   rescales its O row when the running max grows by more
-//                   than 2^8 (lazy rescale: between rescales P may exceed 1,
-//                   which the final division by the same sum cancels).
-//   warp 8 (9)      TMA producer: the query tiles once, then K/V tiles of the
-//                   page table into a STAGES-deep ring. A tile is 128 pool rows
-//                   of one head, one 3-D box load per 64 columns; the page table
-//                   gives each tile's row, so pages need not be contiguous.
-//   warp 9 (11)     TMEM allocator and MMA issuer (tcgen05 kind::f16, fp32
-//                   accumulators in TMEM): S_t = Q_t K^T (M=128, N=128, K=D)
-//                   and O_t += P_t V (M=128, N=D, K=128, P read from TMEM).
-//   warps 8, 10     (head_dim 64; producer and MMA issuer then move to warps 9
-//                   and 11) the unit's tail: a last query tile of at most 16
-//                   rows (262 = 2 x 128 + 6 tokens per frame). An M = 128
-//                   tensor-core tile would be almost all padding, so each of
-//                   these warps computes the tail's scores and output for 64 of
-//                   every K/V tile's 128 rows with warp-level mma.sync
-//                   m16n8k16, transposed so that the tail rows fill the N = 8
-//                   side, reading K and V straight from the shared-memory
-//                   ring, with its own running max/sum and O in registers. The
-//                   two partial results are merged at the end.
+// Roles. head_dim 64: 12 warps (384 threads); head_dim 128: 10 warps (320).
+//   warps 0-3, 4-7   softmax warpgroups, one per 128-row query tile. Thread i
+//                    owns query row i == TMEM lane i. Per K/V tile it reads its
+//                    S row in two 64-column halves, keeps the running max/sum
+//                    in the log2 domain, writes P (16-bit) to TMEM -- the first
+//                    half as soon as the previous PV has read P, so its store
+//                    overlaps the second half -- and rescales its O row when
+//                    the running max grows by more than 2^8 (lazy rescale:
+//                    between rescales P may exceed 1, which the final division
+//                    by the same sum cancels).
+//   producer         warp 9 (head_dim 64) / 8 (head_dim 128): TMA loads, the
+//                    query tiles once, then K/V tiles of the page table into a
+//                    STAGES-deep ring. A tile is 128 pool rows of one head, one
+//                    3-D box load per 64 columns; the tile table gives each
+//                    tile's row, so pages need not be contiguous.
+//   MMA issuer       warp 11 / 9, also the TMEM allocator (tcgen05 kind::f16,
+//                    fp32 accumulators in TMEM): S_t = Q_t K^T (M=128, N=128,
+//                    K=D) and O_t += P_t V (M=128, N=D, K=128, P read from
+//                    TMEM). Each query tile advances on its own, scores first.
+//   tail             warps 8 and 10 (head_dim 64): the unit's last query tile
+//                    of at most 16 rows (262 = 2 x 128 + 6 tokens per frame).
+//                    An M = 128 tensor-core tile would be almost all padding,
+//                    so each of these warps computes the tail's scores and
+//                    output for 64 of every K/V tile's 128 rows with warp-level
+//                    mma.sync m16n8k16, transposed so that the tail rows fill
+//                    the N = 8 side, reading K and V straight from the
+//                    shared-memory ring, with its own running max/sum and O in
+//                    registers. The two partial results are merged at the end.
 // TMEM. head_dim 64: S_t at [128 t, +128), P_t at [256 + 64 t, +64), O_t at
 // [384 + 64 t, +64). P has its own columns, so the tensor core computes
 // S_t(j+1) as soon as the softmax has read S_t(j), while the exponentials of
 // tile j run. head_dim 128: O_t takes [256 + 128 t, +128), so P_t is written
 // over the S_t columns it came from and S_t(j+1) follows PV_t(j).
+// The launch overlaps the previous kernel on the stream (programmatic
+// dependent launch): everything before pdl_wait() is setup that touches no
+// data an earlier kernel may still be writing.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <math.h>
