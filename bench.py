@@ -464,18 +464,8 @@ def run_gpu(args):
         steady_tflops = None
 
     if rank == 0:
-        if args.workload == 1:
-            metric = "frames/s (24-block stack) at 224x224, 320 frames"
-        elif wl.streams > 1:
-            metric = f"frames/s ({wl.streams} streams x {wl.blocks}-block stack), {wl.name}"
-        else:
-            metric = f"frames/s ({wl.blocks}-block stack), {wl.name}"
-        config = {"workload": wl.name, "frames": wl.frames, "blocks": wl.blocks, "H": wl.H,
-                  "D": wl.D, "tokens_per_frame": wl.T, "page_size": wl.page_size,
-                  "scale_frames": wl.S, "window": wl.W, "keyframes": wl.keyframes,
-                  "cross_frame_special": wl.cross_special,
-                  "parallelism": f"replicas x{world}",
-                  "l2": "inputs larger than L2 (one pool per block, all read every frame step)"}
+        metric = metric_name(args.workload, wl)
+        config = workload_config(wl, world)
         if wl.streams > 1:
             config.update({"streams": wl.streams, "stream_ages": [int(x) for x in runner.ages],
                            "frame_steps_per_pass": runner.steps, "frames": None})
@@ -510,6 +500,35 @@ def run_gpu(args):
 
 
 # ------------------------------------------------------------------ oracle arm
+def oracle_threads():
+    """Threads the oracle's numpy arithmetic can use (its einsum contractions
+    run in the BLAS thread pool)."""
+    try:
+        import threadpoolctl
+        n = [d["num_threads"] for d in threadpoolctl.threadpool_info() if d.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def metric_name(workload_id, wl):
+    if workload_id == 1:
+        return "frames/s (24-block stack) at 224x224, 320 frames"
+    if wl.streams > 1:
+        return f"frames/s ({wl.streams} streams x {wl.blocks}-block stack), {wl.name}"
+    return f"frames/s ({wl.blocks}-block stack), {wl.name}"
+
+
+def workload_config(wl, world):
+    """The config object of a bench line (the same for both arms)."""
+    return {"workload": wl.name, "frames": wl.frames, "blocks": wl.blocks, "H": wl.H,
+            "D": wl.D, "tokens_per_frame": wl.T, "page_size": wl.page_size,
+            "scale_frames": wl.S, "window": wl.W, "keyframes": wl.keyframes,
+            "cross_frame_special": wl.cross_special,
+            "parallelism": f"replicas x{world}",
+            "l2": "inputs larger than L2 (one pool per block, all read every frame step)"}
+
+
 def cpu_baseline(wl, seed, budget_s=20.0, frames_sample=(0, 71, 159, 319), rows=None):
     """Times the CPU oracle (float64 dense attention) on a bounded sample of
     the workload and extrapolates frames/s by FLOPs."""
@@ -547,8 +566,7 @@ def cpu_baseline(wl, seed, budget_s=20.0, frames_sample=(0, 71, 159, 319), rows=
              for n in range(1, wl.frames + 1)]
     total = sum(call_flops(wl.T, l, wl.H, wl.D) for l in sim_l) * wl.blocks
     fps = wl.frames / (total / (gflops * 1e9))
-    threads = 1   # numpy einsum without BLAS runs on one thread
-    return {"value": fps, "unit": "frames/s", "cores": threads, "kind": "oracle",
+    return {"value": fps, "unit": "frames/s", "cores": oracle_threads(), "kind": "oracle",
             "gflops": round(gflops, 3),
             "sample": f"float64 oracle attention of block 0 at frames {[d + 1 for d in done]} for "
                       f"{len(sel)} of {wl.T} query rows ({t_att:.1f} s); frames/s extrapolated by "
@@ -566,17 +584,19 @@ def run_reference(args):
         cpu_baseline(wl, args.seed, budget_s=budget / 4, frames_sample=(0,), rows=8)
     t = time.perf_counter()
     vals = []
+    n = max(1, wl.frames)
+    sample = tuple(sorted({min(wl.S + wl.W - 1, n - 1), n - 1}))   # a ramp frame and the last frame
     for _ in range(args.steps):
-        vals.append(cpu_baseline(wl, args.seed, budget_s=budget, frames_sample=(71, 319), rows=16))
+        vals.append(cpu_baseline(wl, args.seed, budget_s=budget, frames_sample=sample, rows=16))
     el = time.perf_counter() - t
     v = statistics.median(x["value"] for x in vals)
     line = {
-        "impl": "reference", "metric": "frames/s (24-block stack) at 224x224, 320 frames",
+        "impl": "reference", "metric": metric_name(args.workload, wl),
         "value": v, "unit": "frames/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(el * 1e3 / max(1, args.steps), 1), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "frames": wl.frames, "blocks": wl.blocks},
-        "cpu_baseline": {"value": v, "unit": "frames/s", "cores": 1, "kind": "oracle",
+        "config": workload_config(wl, world),
+        "cpu_baseline": {"value": v, "unit": "frames/s", "cores": oracle_threads(), "kind": "oracle",
                          "sample": vals[-1]["sample"]},
         "e2e": {"value": v, "unit": "frames/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
