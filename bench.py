@@ -579,6 +579,10 @@ def run_reference(args):
     if rank != 0:
         return
     wl = workload.WORKLOADS[args.workload]
+    if wl.streams > 1:
+        # the oracle runs one stream; a stream as old as the oldest in the batch
+        import dataclasses
+        wl = dataclasses.replace(wl, streams=1, frames=wl.age_hi)
     budget = max(5.0, 150.0 / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
         cpu_baseline(wl, args.seed, budget_s=budget / 4, frames_sample=(0,), rows=8)
