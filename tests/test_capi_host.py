@@ -318,3 +318,56 @@ def test_workspace_bytes_and_batch_checks(pkv):
         pkv.kv_plan([a, c])
     for x in (a, b, c):
         pkv.kv_destroy(x)
+
+
+def test_run_static_argument_checks_before_any_device_work(pkv):
+    """kv_run_static rejects bad calls on the host, before touching a device
+    (so these run without a GPU)."""
+    E = pkv.capi
+    h = mk(pkv, 2, 4, 16, 12, B=2)
+    q = out = 1 << 20                         # 16-byte aligned addresses that are never dereferenced
+
+    def code(*args, **kw):
+        with pytest.raises(pkv.KVError) as e:
+            pkv.kv_run_static(*args, **kw)
+        return e.value.code
+
+    step(pkv, h, 1)                          # only block 0 appended in this step
+    assert code([h], 0, None, out) == E.KV_ERR_ARG                  # NULL q
+    assert code([h], 0, q, out, tiles_per_split=-1) == E.KV_ERR_ARG
+    assert code([h], 0, q + 4, out) == E.KV_ERR_ARG                 # misaligned q
+    assert code([h], 5, q, out) == E.KV_ERR_ARG                     # block out of range
+    assert code([h], 1, q, out) == E.KV_ERR_NOT_APPENDED            # block 1 not appended yet
+    assert code([h], 0, q, out) == E.KV_ERR_ARG                     # no pool bound for block 0
+    assert code([], 0, q, out) == E.KV_ERR_ARG                      # no caches
+    pkv.kv_destroy(h)
+
+
+def test_cross_frame_special_setting_changes_the_visible_rows(pkv):
+    """Switching cross-frame special retention changes what the next plan
+    attends to (here: 2 patch frames of 16 plus 24 special tokens, then plus
+    only frames 0 and 3's 12); switching to the current value changes nothing."""
+    h = mk(pkv, 1, 1, 16, 10)
+    for _ in range(4):
+        step(pkv, h)
+
+    def visible():
+        p = pkv.kv_plan([h])
+        try:
+            return pkv.kv_plan_get_stats(p)["visible_tokens"], tile_cover(pkv.kv_get_kv_tiles(p), 16)
+        finally:
+            pkv.kv_plan_free(p)
+
+    n_on, cover_on = visible()
+    pkv.kv_set_cross_frame_special(h, True)   # already on: no change
+    assert visible() == (n_on, cover_on)
+    pkv.kv_set_cross_frame_special(h, False)
+    n_off, cover_off = visible()
+    assert (n_on, n_off) == (2 * 16 + 24, 2 * 16 + 12)
+    m = PageModel(1, 1, 16, 10, cross_frame_special=False)
+    for f in range(4):
+        m.append(f); m.evict()
+    want = [(pg, t) for _, pg in m.patch_pages_visible() for t in range(16)]
+    want += [(m.Np + j // 16, j % 16) for j in m.visible_special_index()]
+    assert sorted(cover_off) == sorted(want)
+    pkv.kv_destroy(h)
