@@ -31,7 +31,6 @@ struct AttnArgs {
 };
 
 struct MergeArgs {
-  const KvReq* reqs;
   const KvMergeItem* items;
   const float* part_o;
   const float* part_lse;

@@ -353,7 +353,6 @@ int kv_run(const kv_plan_t* p, int block, const void* q, void* out, void* stream
   if (e != cudaSuccess) return cuda_fail(e, "kv_run: attention launch");
   if (hd.n_merge > 0) {
     pkv::MergeArgs m;
-    m.reqs = a.reqs;
     m.items = reinterpret_cast<const pkv::KvMergeItem*>(ws + hd.off_merge);
     m.part_o = a.part_o;
     m.part_lse = a.part_lse;

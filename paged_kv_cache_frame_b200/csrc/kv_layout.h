@@ -48,12 +48,12 @@ constexpr int kMaxTailRows = 16;   // tail rows computed with swapped operands (
 
 // One (request, head, q-tile) whose K/V range was split over n CTAs.
 struct KvMergeItem {
-  int16_t req;
   int16_t head;
-  int16_t qtile;
+  int16_t rows;        // valid query rows of the tile (at most 128)
   int16_t n;           // partial slots slot0 .. slot0 + n - 1
+  int16_t pad;
   int32_t slot0;
-  int32_t pad;
+  int32_t row0;        // row of q/out holding the tile's first query row
 };
 
 struct KvPlanHeader {

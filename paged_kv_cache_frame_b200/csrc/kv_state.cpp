@@ -370,9 +370,12 @@ int build_plan(const std::vector<const PageState*>& st, const PlanInputs& in, Ho
         for (int t = 0; t < ntiles_q; ++t) {
           slot0[t] = n_slots;
           n_slots += chunks;
+          const KvReq& rq = P.reqs[g.req];
           KvMergeItem m{};
-          m.req = (int16_t)g.req; m.head = (int16_t)h; m.qtile = (int16_t)(g.qt + t);
+          m.head = (int16_t)h;
+          m.rows = (int16_t)std::min(kTile, rq.T - (g.qt + t) * kTile);
           m.n = (int16_t)chunks; m.slot0 = slot0[t];
+          m.row0 = rq.q_row0 + (g.qt + t) * kTile;
           P.merges.push_back(m);
           ++P.n_split_units;
         }
