@@ -56,7 +56,7 @@ enum {
   KV_ERR_ORDER = -3,        /* call out of order (frame step rule above) */
   KV_ERR_NO_PENDING = -4,   /* commit or rollback without a deferred frame */
   KV_ERR_NOT_APPENDED = -5, /* kv_run for a block not appended in the current step */
-  KV_ERR_EMPTY = -6,        /* kv_plan before the first frame */
+  KV_ERR_EMPTY = -6,        /* kv_plan before the first frame, or with no visible token */
   KV_ERR_CUDA = -7,         /* a CUDA runtime or driver call failed */
   KV_ERR_DEVICE_CHECK = -8, /* a kernel set the device error word (bounded wait expired
                                or an index check failed) */
@@ -193,7 +193,12 @@ size_t kv_workspace_bytes(kv_cache_t* const* caches, int n_streams);
  * [P3] "Visible Page Table Attention"). For each cache, build the visible page
  * table ([P1] "Building the Visible Page Table"): scale pages in frame order,
  * window pages oldest to newest, the pending page, then the special pages,
- * and paged_kv_last_page_len = fill of the last special page (1..page_size).
+ * and paged_kv_last_page_len = tokens written to the table's final page
+ * (1..page_size; [P1] "Frequently Asked Questions": the exact count of valid
+ * tokens in the final page). The final page is the special stream's last page
+ * unless cross-frame special retention is off and hides all of its tokens;
+ * the tokens that retention off hides inside a listed page are not expressible
+ * in (indices, last_page_len) and are left out of the K/V tiles.
  * Split the 128-token K/V tiles over CTAs (tiles_per_split = 0: automatic
  * schedule for the SM count; > 0: at most that many tiles per CTA, which
  * forces split-KV for tests) and copy the tables into `workspace` on
@@ -203,7 +208,8 @@ size_t kv_workspace_bytes(kv_cache_t* const* caches, int n_streams);
  * workspace == NULL builds a host-only plan (kv_get_page_table works, kv_run
  * does not). All caches must share page_size, H, D, NS, num_blocks and dtype.
  * The plan stays valid, for every block, until a cache's page state changes.
- * Errors: KV_ERR_ARG, KV_ERR_EMPTY (a cache with no frame), KV_ERR_CAPACITY
+ * Errors: KV_ERR_ARG, KV_ERR_EMPTY (a cache with no frame, or none of whose
+ * tokens is visible: scale_frames = window = 0 with retention off), KV_ERR_CAPACITY
  * (workspace smaller than kv_workspace_bytes, > KV_MAX_STREAMS), KV_ERR_CUDA. */
 int kv_plan(kv_plan_t** out, kv_cache_t* const* caches, int n_streams, int tiles_per_split,
             void* workspace, size_t workspace_bytes, void* stream);

@@ -20,7 +20,7 @@ lives on page Np + j // page_size at slot j % page_size.
 Visible page table ([P1] "Building the Visible Page Table"; [P3] "Visible Page
 Table Attention"): scale pages in frame order, window pages oldest to newest,
 then the pending page if any, then special pages Np .. Np+k-1. Only the last
-page may be partial; last_page_len is the fill of the last special page.
+page may be partial; last_page_len is the fill of the table's final page.
 
 Without cross-frame special retention ([P2] "Configuration Parameters"), the
 special tokens of evicted frames drop out: the visible special tokens are the
@@ -144,15 +144,26 @@ class PageModel:
         return [j for j in range(self.sp_len) if self.sp_owner[j][0] in live]
 
     def page_table(self) -> tuple[list[int], int]:
-        """(kv_indices, last_page_len) of the visible page table."""
+        """(kv_indices, last_page_len) of the visible page table.
+
+        last_page_len is the number of tokens written to the table's final
+        page ([P1] "Frequently Asked Questions": the exact count of valid
+        tokens in the final page). The final page is a special page; only
+        with cross-frame special retention off can it be an earlier one than
+        the stream's last, whose specials are then all hidden. Hidden tokens
+        inside a listed page are not expressible by (indices, last_page_len)
+        and are read off visible_special_index instead.
+        """
         if self.committed == 0 and self.pending is None:
-            raise OracleError("EMPTY")
+            raise OracleError("EMPTY", "no frame")
         patch = [p for _, p in self.patch_pages_visible()]
-        k = -(-self.sp_len // self.ps)
         pages = sorted({j // self.ps for j in self.visible_special_index()})
         special = [self.Np + i for i in pages]
-        last = self.sp_len - self.ps * (k - 1) if k else self.ps
-        return patch + special, last
+        table = patch + special
+        if not table:   # scale_frames = window = 0 with retention off
+            raise OracleError("EMPTY", "no visible token")
+        last = min(self.ps, self.sp_len - self.ps * pages[-1]) if pages else self.ps
+        return table, last
 
     def visible_token_count(self) -> int:
         return len(self.patch_pages_visible()) * self.ps + len(self.visible_special_index())
@@ -174,6 +185,8 @@ class PageModel:
         """Visible tokens in the frame simulator's ('p', frame, t) / ('s', frame,
         slot) form, read back through the page table: each listed page and
         slot is mapped to the frame that wrote it."""
+        if self.visible_token_count() == 0:
+            return set()
         table, last = self.page_table()
         owner = {p: f for f, p in self.patch_pages_visible()}
         vis = set(self.visible_special_index())

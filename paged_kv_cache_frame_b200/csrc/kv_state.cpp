@@ -197,12 +197,16 @@ int PageState::page_table(std::vector<int>* idx, int* last_page_len) const {
   std::vector<PageRun> runs;
   const int rc = visible_runs(&runs);
   if (rc != KV_OK) return rc;
+  // nothing visible: no scale frame, no window and retention off
+  if (runs.empty()) return KV_ERR_EMPTY;
   idx->clear();
   for (const PageRun& r : runs)
     if (idx->empty() || idx->back() != r.page) idx->push_back(r.page);
+  // tokens written to the table's final page: the special stream's last page
+  // unless retention off hides all of its tokens
   const int ps = cfg.page_size;
-  const int k = ceil_div(sp_len, ps);
-  *last_page_len = k ? sp_len - ps * (k - 1) : ps;
+  const int last = idx->back();
+  *last_page_len = last >= cfg.Np ? std::min(ps, sp_len - ps * (last - cfg.Np)) : ps;
   return KV_OK;
 }
 
@@ -279,7 +283,8 @@ int build_plan(const std::vector<const PageState*>& st, const PlanInputs& in, Ho
     int lpl = 0;
     const int rc = s->page_table(&table, &lpl);
     if (rc != KV_OK) {
-      *why = "plan: a stream has no frame yet";
+      *why = s->committed == 0 && !s->has_pending ? "plan: a stream has no frame yet"
+                                                  : "plan: a stream has no visible token";
       return rc;
     }
     std::vector<PageRun> runs;

@@ -66,6 +66,21 @@ def table(pkv, caches):
         pkv.kv_plan_free(p)
 
 
+def assert_same_table(pkv, h, m):
+    """The library's page table equals the oracle's; where the oracle finds
+    nothing to attend to (no frame, or no visible token), kv_plan refuses
+    with KV_ERR_EMPTY."""
+    try:
+        want = m.page_table()
+    except OracleError as e:
+        assert e.code == "EMPTY"
+        with pytest.raises(pkv.KVError) as ce:
+            table(pkv, [h])
+        assert ce.value.code == pkv.capi.KV_ERR_EMPTY
+        return
+    assert table(pkv, [h])[0] == want
+
+
 def test_stats_example_through_capi(pkv):
     g = json.load(open(os.path.join(ROOT, "tests", "golden", "cache_stats_12_frames.json")))
     c = g["config"]
@@ -197,7 +212,7 @@ def test_state_machine_bit_exact_vs_oracle(pkv, ops, S, W, ps, B, xs):
                 m.set_defer(True); pkv.kv_defer_eviction(h, True)
                 m.append(f); m.evict()
                 step(pkv, h, B)
-                assert table(pkv, [h])[0] == m.page_table()
+                assert_same_table(pkv, h, m)
                 if op == "defer_keep":
                     m.commit(); pkv.kv_commit_frame(h)
                 else:
@@ -217,8 +232,7 @@ def test_state_machine_bit_exact_vs_oracle(pkv, ops, S, W, ps, B, xs):
                 assert e.value.code == E.KV_ERR_NO_PENDING
             assert pkv.kv_get_free_list(h) == m.free
             assert pkv.kv_get_stats(h) == m.stats()
-            if m.committed or m.pending is not None:
-                assert table(pkv, [h])[0] == m.page_table()
+            assert_same_table(pkv, h, m)
     finally:
         pkv.kv_destroy(h)
 
@@ -235,6 +249,50 @@ def test_rollback_restores_state_through_capi(pkv, n, S, W):
     pkv.kv_rollback_last_frame(h)
     after = (pkv.kv_get_free_list(h), pkv.kv_get_stats(h), table(pkv, [h]) if n else None)
     assert before == after
+    pkv.kv_destroy(h)
+
+
+def test_last_page_len_when_retention_off_hides_the_last_special_page(pkv):
+    """One scale frame, no window, retention off, 3 frames, page size 16:
+    frames 1 and 2 are evicted as soon as they are appended, so their
+    specials (stream tokens 6-17) are hidden and special page 1 (tokens
+    16-17) holds nothing visible. The table is frame 0's patch page and
+    special page 0, which is full: last_page_len = 16, not the fill of the
+    stream's last page (2). Only tokens 0-5 of special page 0 are tiled."""
+    S, W, ps, max_pages = 1, 0, 16, 6
+    Np = S + W + 1
+    h = mk(pkv, S, W, ps, max_pages)
+    pkv.kv_set_cross_frame_special(h, False)
+    for _ in range(3):
+        step(pkv, h)
+    p = pkv.kv_plan([h])
+    assert pkv.kv_get_page_table(p) == ([0, Np], 16)
+    got = tile_cover(pkv.kv_get_kv_tiles(p), ps)
+    assert sorted(got) == sorted([(0, t) for t in range(ps)] + [(Np, t) for t in range(6)])
+    pkv.kv_plan_free(p)
+    # retention on: every special is visible; the last page holds 2 tokens
+    pkv.kv_set_cross_frame_special(h, True)
+    p = pkv.kv_plan([h])
+    assert pkv.kv_get_page_table(p) == ([0, Np, Np + 1], 2)
+    pkv.kv_plan_free(p)
+    pkv.kv_destroy(h)
+
+
+def test_plan_refuses_a_stream_with_no_visible_token(pkv):
+    """No scale frame, no window, retention off: every frame is evicted as it
+    is appended and its specials go with it, so nothing is left to attend
+    to; kv_plan reports KV_ERR_EMPTY instead of planning an empty softmax."""
+    h = mk(pkv, 0, 0, 16, 4)
+    pkv.kv_set_cross_frame_special(h, False)
+    step(pkv, h)
+    with pytest.raises(pkv.KVError) as e:
+        pkv.kv_plan([h])
+    assert e.value.code == pkv.capi.KV_ERR_EMPTY
+    assert "no visible token" in str(e.value)
+    pkv.kv_set_cross_frame_special(h, True)   # the specials are visible again
+    p = pkv.kv_plan([h])
+    assert pkv.kv_get_page_table(p) == ([1], 6)
+    pkv.kv_plan_free(p)
     pkv.kv_destroy(h)
 
 

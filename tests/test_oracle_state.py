@@ -134,6 +134,38 @@ def test_capacity_errors():
     assert e.value.code == "EMPTY"
 
 
+def test_last_page_len_is_the_fill_of_the_tables_final_page():
+    """[P1] "Frequently Asked Questions": last_page_len counts the valid tokens
+    in the table's final page. One scale frame, no window, retention off,
+    three frames of page size 16: frames 1 and 2 are evicted on arrival, so
+    stream tokens 6-17 are hidden and special page 1 (tokens 16-17) drops out
+    of the table; its final page is special page 0, written in full."""
+    m = PageModel(1, 0, 16, max_pages=6, NS=6, cross_frame_special=False)
+    sim = FrameListSim(1, 0, 6, cross_frame_special=False)
+    for f in range(3):
+        m.append(f); m.evict()
+        sim.append(f); sim.evict()
+    assert m.page_table() == ([0, 2], 16)
+    assert m.visible_special_index() == list(range(6))
+    assert m.visible_tokens() == sim.visible_tokens(16)
+    # with retention on the final page is the stream's last: 18 - 16 = 2 tokens
+    m.cross_frame_special = True
+    assert m.page_table() == ([0, 2, 3], 2)
+
+
+def test_nothing_visible_is_an_empty_table():
+    """No scale frame, no window, retention off: a frame is evicted as it is
+    appended and its specials hide with it, so the table would be empty."""
+    m = PageModel(0, 0, 16, max_pages=4, NS=6, cross_frame_special=False)
+    sim = FrameListSim(0, 0, 6, cross_frame_special=False)
+    m.append(0); m.evict()
+    sim.append(0); sim.evict()
+    assert sim.visible_tokens(16) == set() == m.visible_tokens()
+    with pytest.raises(OracleError) as e:
+        m.page_table()
+    assert e.value.code == "EMPTY"
+
+
 def _invariants(m: PageModel):
     used = [p for _, p in m.scale] + [p for _, p in m.window]
     if m.pending is not None:
