@@ -201,13 +201,41 @@ def workspace_bytes(caches) -> int:
 
 
 # ---------------------------------------------------------------- objects
+def _is_fp16(dtype) -> bool:
+    return dtype in ("fp16", "float16") or str(dtype) == "torch.float16"
+
+
+def _torch_dtype(fp16: bool):
+    import torch
+    return torch.float16 if fp16 else torch.bfloat16
+
+
+def _check_tensor(x, name, shape, fp16):
+    """The library sees only a tensor's address and touches exactly `shape`
+    elements of the cache dtype there, so the shape, dtype, layout and device
+    are checked here, before the call. Raw int addresses are the caller's
+    responsibility."""
+    if x is None or isinstance(x, int):
+        return
+    want = _torch_dtype(fp16)
+    if tuple(x.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(x.shape)}, expected {tuple(shape)}")
+    if x.dtype != want:
+        raise ValueError(f"{name}: dtype {x.dtype}, expected {want}")
+    if not x.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if x.device.type != "cuda":
+        raise ValueError(f"{name}: must be a CUDA tensor, not on {x.device}")
+
+
 class PagedKVCache:
     """One video stream's paged cache (all transformer blocks)."""
 
     def __init__(self, max_pages, page_size, num_heads, head_dim, scale_frames=8, window=64,
                  num_blocks=1, num_special=6, dtype="bf16", patch_pages=0, cross_frame_special=True):
         self.dtype = dtype
-        code = KV_FP16 if dtype in ("fp16", "float16") or str(dtype) == "torch.float16" else KV_BF16
+        self.fp16 = _is_fp16(dtype)
+        code = KV_FP16 if self.fp16 else KV_BF16
         self.handle = kv_init(max_pages, page_size, num_heads, head_dim, scale_frames, window,
                               num_blocks, num_special, code, patch_pages)
         self.max_pages, self.page_size = max_pages, page_size
@@ -230,13 +258,19 @@ class PagedKVCache:
         return kv_pool_bytes(self.handle)
 
     def bind_pool(self, block, pool, stream=None):
+        if pool is not None and not isinstance(pool, int):
+            nbytes = pool.numel() * pool.element_size()
+            if nbytes < self.pool_bytes():
+                raise ValueError(f"pool: {nbytes} bytes, the cache needs {self.pool_bytes()}")
+            if not pool.is_contiguous() or pool.device.type != "cuda":
+                raise ValueError("pool: must be a contiguous CUDA tensor")
         kv_bind_pool(self.handle, block, pool, stream)
         self.pools[block] = pool
 
     def allocate_pools(self, device="cuda", stream=None):
         """Allocate each block's pool [max_pages, 2, page_size, H, D] with torch and bind it."""
         import torch
-        dt = torch.float16 if self.dtype in ("fp16", "float16") else torch.bfloat16
+        dt = _torch_dtype(self.fp16)
         for b in range(self.num_blocks):
             pool = torch.empty((self.max_pages, 2, self.page_size, self.H, self.D), dtype=dt,
                                device=device)
@@ -244,6 +278,11 @@ class PagedKVCache:
         return self.pools
 
     def append_frame(self, block, k, v, stream=None):
+        """k, v: [T, H, D] of the cache dtype (tokens 0..NS-1 special), or both
+        None to advance the page state only."""
+        shape = (self.T, self.H, self.D)
+        _check_tensor(k, "k", shape, self.fp16)
+        _check_tensor(v, "v", shape, self.fp16)
         kv_append_frame(self.handle, block, k, v, stream)
 
     def evict_frames(self):
@@ -278,7 +317,7 @@ class Plan:
                               stream=stream)
         c0 = self.caches[0]
         self.rows = sum(c.T for c in self.caches)
-        self.H, self.D, self.dtype = c0.H, c0.D, c0.dtype
+        self.H, self.D, self.dtype, self.fp16 = c0.H, c0.D, c0.dtype, c0.fp16
 
     def __del__(self):
         h = getattr(self, "handle", None)
@@ -290,9 +329,13 @@ class Plan:
                 pass
 
     def run(self, block, q, out=None, stream=None):
+        """q (and out): [sum of the streams' T, H, D] of the cache dtype."""
+        shape = (self.rows, self.H, self.D)
+        _check_tensor(q, "q", shape, self.fp16)
         if out is None:
             import torch
             out = torch.empty_like(q)
+        _check_tensor(out, "out", shape, self.fp16)
         kv_run(self.handle, block, q, out, stream)
         return out
 

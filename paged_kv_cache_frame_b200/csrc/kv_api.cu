@@ -47,17 +47,17 @@ int cuda_fail(cudaError_t e, const char* where) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Looked up once; the initialisation of a function-local static is
+// thread-safe, so concurrent first calls from several threads are fine.
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
+      return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    return nullptr;
+  }();
   return fn;
 }
 
@@ -98,7 +98,7 @@ const char* kv_strerror(int status) {
     case KV_ERR_ORDER: return "call out of order";
     case KV_ERR_NO_PENDING: return "no pending (deferred) frame";
     case KV_ERR_NOT_APPENDED: return "block not appended in this frame step";
-    case KV_ERR_EMPTY: return "cache holds no frame";
+    case KV_ERR_EMPTY: return "cache holds no frame or no visible token";
     case KV_ERR_CUDA: return "CUDA error";
     case KV_ERR_DEVICE_CHECK: return "device-side check failed";
     case KV_ERR_UNSUPPORTED: return "unsupported shape or dtype";

@@ -42,17 +42,36 @@ def assert_close(out, want, what=""):
     return mx, mean
 
 
-def dense_fp32(cache, plan, block, q, stream_idx=0):
+def dense_fp32(cache, plan, block, q, so, Np, stream_idx=0):
     """Every row and head of the frame's attention in fp32 on the GPU: the
-    visible pages of `plan`'s table gathered densely from the block's pool
-    (a check on the kernel at full size, next to the oracle's sampled rows)."""
+    pages of `plan`'s table gathered densely from the block's pool (a check on
+    the kernel at full size, next to the oracle's sampled rows).
+
+    Patch pages are read whole. On special pages, stream token j (page
+    Np + j // page_size, slot j % page_size) is read when the oracle's frame
+    simulator `so.sim` holds it visible: all written tokens with cross-frame
+    special retention on, only live frames' tokens with it off (the table
+    cannot express those gaps). last_page_len must equal the number of
+    tokens written to the table's final page."""
     pool = cache.pools[block]                       # [max_pages, 2, page_size, H, D]
+    ps = cache.page_size
     table, lpl = plan.page_table(stream_idx)
-    idx = torch.as_tensor(table, device=pool.device, dtype=torch.long)
-    kv = pool.index_select(0, idx).float()          # [n_pages, 2, page_size, H, D]
-    n = len(table)
-    k = kv[:, 0].reshape(n * cache.page_size, cache.H, cache.D)[: (n - 1) * cache.page_size + lpl]
-    v = kv[:, 1].reshape(n * cache.page_size, cache.H, cache.D)[: (n - 1) * cache.page_size + lpl]
+    sp = so.sim.SP                                  # special stream, in append order
+    vis = set(so.sim.visible_specials())
+    rows = []
+    for p in table:
+        if p < Np:
+            rows.extend(p * 2 * ps + t for t in range(ps))
+        else:
+            i = p - Np
+            rows.extend(p * 2 * ps + t for t in range(ps)
+                        if i * ps + t < len(sp) and sp[i * ps + t] in vis)
+    last = table[-1]
+    assert last >= Np and lpl == min(ps, len(sp) - ps * (last - Np)), "last_page_len"
+    idx = torch.as_tensor(rows, device=pool.device, dtype=torch.long)
+    flat = pool.view(-1, cache.H, cache.D)          # row (page * 2 + kv) * page_size + slot
+    k = flat.index_select(0, idx).float()
+    v = flat.index_select(0, idx + ps).float()
     out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
     scale = cache.D ** -0.5
     for h in range(cache.H):   # one head at a time keeps the score matrix small
@@ -108,7 +127,8 @@ def run_stream(pkv, wl, seed, n_frames, check, rows=None, defer=None, keep=None,
             sel = slice(None) if rows is None else torch.as_tensor(rows)
             res[f] = assert_close(out[sel], so.expected(rows), f"frame {f}")
             if f in dense:
-                assert_close_dense(out, dense_fp32(cache, plan, 0, q), f"frame {f} (all rows, fp32 dense)")
+                want = dense_fp32(cache, plan, 0, q, so, patch_pages or wl.patch_pages)
+                assert_close_dense(out, want, f"frame {f} (all rows, fp32 dense)")
             if collect is not None:
                 collect[f] = out.clone()
         if d:

@@ -429,3 +429,33 @@ def test_cross_frame_special_setting_changes_the_visible_rows(pkv):
     want += [(m.Np + j // 16, j % 16) for j in m.visible_special_index()]
     assert sorted(cover_off) == sorted(want)
     pkv.kv_destroy(h)
+
+
+def test_object_api_checks_tensors_before_the_call(pkv):
+    """The library sees only addresses, so PagedKVCache and Plan check each
+    tensor's shape, dtype, layout and device first; a refused call leaves the
+    page state untouched."""
+    import torch
+    T, H, D = 16 + 6, 2, 64
+    c = pkv.PagedKVCache(8, 16, H, D, scale_frames=1, window=2, num_blocks=1)
+    on_cpu = torch.zeros(T, H, D, dtype=torch.bfloat16)
+    for bad, what in [(torch.zeros(T - 1, H, D, dtype=torch.bfloat16), "shape"),
+                      (torch.zeros(T, H, D, dtype=torch.float16), "dtype"),
+                      (torch.zeros(H, T, D, dtype=torch.bfloat16).transpose(0, 1), "contiguous"),
+                      (on_cpu, "CUDA")]:
+        with pytest.raises(ValueError, match=what):
+            c.append_frame(0, bad, bad)
+    assert c.get_stats()["frame_count"] == 0
+    with pytest.raises(ValueError, match="bytes"):
+        c.bind_pool(0, torch.zeros(16, dtype=torch.uint8))
+    c.append_frame(0, None, None)
+    p = pkv.Plan([c])
+    with pytest.raises(ValueError, match="shape"):
+        p.run(0, torch.zeros(T + 1, H, D, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="CUDA"):
+        p.run(0, on_cpu)
+    # a torch dtype selects the same kernels and pool dtype as its name
+    f16 = pkv.PagedKVCache(8, 16, H, D, 1, 2, num_blocks=1, dtype=torch.float16)
+    with pytest.raises(ValueError, match="dtype"):
+        f16.append_frame(0, on_cpu, on_cpu)
+    assert f16.fp16 and not c.fp16
