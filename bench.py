@@ -357,10 +357,10 @@ def run_gpu(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)   # before the process group, so NCCL binds this GPU
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    torch.cuda.set_device(local)
     from paged_kv_cache_frame_b200 import build
     build.build()
     wl = workload.WORKLOADS[args.workload]
@@ -378,7 +378,7 @@ def run_gpu(args):
 
     def barrier():
         if world > 1:
-            dist.barrier()
+            dist.barrier(device_ids=[local])
 
     for _ in range(args.warmup):
         runner.one_pass()
@@ -465,10 +465,9 @@ def run_gpu(args):
 
     if rank == 0:
         metric = metric_name(args.workload, wl)
-        config = workload_config(wl, world)
+        config = arm_config(wl, world, args.seed)
         if wl.streams > 1:
-            config.update({"streams": wl.streams, "stream_ages": [int(x) for x in runner.ages],
-                           "frame_steps_per_pass": runner.steps, "frames": None})
+            assert config["stream_ages"] == [int(x) for x in runner.ages]
         line = {
             "metric": metric,
             "profiling_case_not_a_bench_value": profiling_case or None,
@@ -517,6 +516,17 @@ def metric_name(workload_id, wl):
     if wl.streams > 1:
         return f"frames/s ({wl.streams} streams x {wl.blocks}-block stack), {wl.name}"
     return f"frames/s ({wl.blocks}-block stack), {wl.name}"
+
+
+def arm_config(wl, world, seed):
+    """The config object of a bench line, identical in both arms: a batched
+    workload adds rank 0's seeded stream ages (the ones BatchRunner draws)."""
+    config = workload_config(wl, world)
+    if wl.streams > 1:
+        ages = workload.stream_ages(wl, replica_seed(seed, 0))
+        config.update({"streams": wl.streams, "stream_ages": [int(x) for x in ages],
+                       "frame_steps_per_pass": wl.steps, "frames": None})
+    return config
 
 
 def workload_config(wl, world):
@@ -578,7 +588,8 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    wl = workload.WORKLOADS[args.workload]
+    arm = workload.WORKLOADS[args.workload]   # metric and config: the same as the GPU arm's
+    wl = arm
     if wl.streams > 1:
         # the oracle runs one stream; a stream as old as the oldest in the batch
         import dataclasses
@@ -595,11 +606,11 @@ def run_reference(args):
     el = time.perf_counter() - t
     v = statistics.median(x["value"] for x in vals)
     line = {
-        "impl": "reference", "metric": metric_name(args.workload, wl),
+        "impl": "reference", "metric": metric_name(args.workload, arm),
         "value": v, "unit": "frames/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(el * 1e3 / max(1, args.steps), 1), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(wl, world),
+        "config": arm_config(arm, world, args.seed),
         "cpu_baseline": {"value": v, "unit": "frames/s", "cores": oracle_threads(), "kind": "oracle",
                          "sample": vals[-1]["sample"]},
         "e2e": {"value": v, "unit": "frames/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

@@ -1,0 +1,40 @@
+"""bench.py's two arms report the same metric, unit and config.
+
+The reference arm times the oracle on a bounded sample (for a batched
+workload: one stream as old as the oldest of the batch), but its JSON line
+must name the workload exactly as the GPU arm does. The oracle timing is
+stubbed here, so this checks only the reporting, on the CPU.
+"""
+import json
+import types
+
+import pytest
+
+import bench
+import workload
+
+
+@pytest.mark.parametrize("w", [1, 2, 3, 4, 5])
+def test_reference_arm_reports_the_gpu_arms_metric_and_config(w, monkeypatch, capsys):
+    monkeypatch.setattr(bench, "cpu_baseline", lambda *a, **k: {"value": 1.0, "sample": "stub"})
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    monkeypatch.setenv("RANK", "0")
+    bench.run_reference(types.SimpleNamespace(workload=w, seed=1, steps=1, warmup=0))
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    wl = workload.WORKLOADS[w]
+    assert line["impl"] == "reference"
+    assert line["metric"] == bench.metric_name(w, wl)     # what the GPU arm prints
+    assert line["config"] == bench.arm_config(wl, 1, 1)
+    assert line["unit"] == "frames/s" and line["higher_is_better"] is True
+    assert line["e2e"] == {"value": 1.0, "unit": "frames/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+    if wl.streams > 1:
+        assert len(line["config"]["stream_ages"]) == wl.streams
+
+
+def test_reference_arm_prints_on_rank_0_only(monkeypatch, capsys):
+    monkeypatch.setattr(bench, "cpu_baseline", lambda *a, **k: {"value": 1.0, "sample": "stub"})
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setenv("RANK", "1")
+    bench.run_reference(types.SimpleNamespace(workload=1, seed=1, steps=1, warmup=0))
+    assert capsys.readouterr().out == ""
