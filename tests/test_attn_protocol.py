@@ -1,0 +1,298 @@
+"""A randomised model of the attention kernel's mbarrier protocol (head_dim 64).
+
+The kernel's warps meet only at mbarriers and at the tensor pipe, so the
+protocol can be checked on the CPU: this model runs the MMA issuer's poll
+loop, every softmax warp (with valid rows or not), the TMA producer, the tail
+warps' stage releases and an in-order tensor pipe whose commit arrives once
+every earlier MMA has run, in random interleavings. It checks:
+
+  * every parity wait polls only while its barrier has completed k or k + 1
+    phases, k being the phase it waits for (otherwise the parity is
+    ambiguous);
+  * each TMEM buffer is read while it still holds the scores S being read,
+    PV_n runs after every warp with valid rows stored P_n, and new scores
+    are written into a buffer only after the PV that reads its P ran;
+  * O_t is rescaled at tile j after PV_t(j-1) ran and before PV_t(j) runs;
+  * a K/V stage is reloaded only after every MMA reading it ran;
+  * nothing deadlocks.
+
+Two schedules are modelled. "current" is the kernel's: scores S_t, 16-bit
+P_t in separate TMEM columns, S_t(j+1) issued once softmax t has read S_t(j).
+"three_buffer" is a successor under consideration: P stored over its S,
+three S/P buffers taken in turn, S number n issued once PV number n-3 has
+been issued. The model shows that the three-buffer schedule needs two rules
+(each test below drops one and finds the failure).
+
+A model is not the kernel: it checks the protocol's logic only.
+"""
+import random
+
+import pytest
+
+ST = 4   # K/V stages
+
+
+class Violation(Exception):
+    pass
+
+
+class Bar:
+    def __init__(self, name, count):
+        self.name, self.count, self.done, self.pend = name, count, 0, 0
+
+    def arrive(self, n=1):
+        for _ in range(n):
+            self.pend += 1
+            if self.pend == self.count:
+                self.done += 1
+                self.pend = 0
+
+    def test(self, k, who):
+        """Parity test for the completion of phase k."""
+        if not (k <= self.done <= k + 1):
+            raise Violation(f"{who} waits for phase {k} of {self.name}, {self.done} completed")
+        return self.done == k + 1
+
+
+def run(schedule, nq, n_tiles, active, tail, seed, gate_on_taken=True, idle_warps_wait=True):
+    rng = random.Random(seed)
+    three = schedule == "three_buffer"
+    s_full = [Bar(f"s_full{t}", 1) for t in range(2)]
+    s_free = [Bar(f"s_free{t}", 128) for t in range(2)]
+    p_full = [Bar(f"p_full{t}", 128) for t in range(2)]
+    pv_done = [Bar(f"pv_done{t}", 1) for t in range(2)]
+    kv_full = [Bar(f"kv_full{s}", 1) for s in range(ST)]
+    kv_empty = [Bar(f"kv_empty{s}", 1 + (2 if tail else 0)) for s in range(ST)]
+    o_final = Bar("o_final", 1)
+    pipe, ran, holds, p_written, stage = [], set(), {}, {}, {}
+    number = lambda t, j: j * nq + t
+    buffer = lambda t, j: number(t, j) % 3 if three else t
+
+    def execute(op):
+        if op[0] == "commit":
+            op[1].arrive()
+            return
+        kind, t, j = op
+        n = number(t, j)
+        if stage.get(j % ST) != j:
+            raise Violation(f"{kind}_{t}({j}) runs without its K/V tile")
+        if kind == "S":
+            if three and n >= 3 and ("PV", (n - 3) % nq, (n - 3) // nq) not in ran:
+                raise Violation(f"S number {n} overwrites P before PV number {n - 3} ran")
+            holds[buffer(t, j)] = n
+        else:
+            if p_written.get(n, set()) != {w for w in range(4) if active[t][w]}:
+                raise Violation(f"PV_{t}({j}) runs before P_{t}({j}) is written")
+        ran.add((kind, t, j))
+
+    def issuer():
+        st = {"started": False, "done": False, "ns": [1, 1], "np": [0, 0], "ne": 0, "kv": 0}
+        if nq < 2:
+            st["ns"][1] = st["np"][1] = n_tiles
+
+        def issue(kind, t, j, bar):
+            pipe.append((kind, t, j))
+            pipe.append(("commit", bar))
+
+        def step():
+            if st["done"]:
+                return None
+            if not st["started"]:
+                if not kv_full[0].test(0, "issuer"):
+                    return False
+                for t in range(nq):
+                    issue("S", t, 0, s_full[t])
+                st["started"] = True
+                return True
+            moved = False
+            ns, np_ = st["ns"], st["np"]
+            for t in range(2):
+                j = ns[t]
+                if j >= n_tiles:
+                    continue
+                if three:
+                    m = number(t, j) - 3
+                    if m >= 0 and np_[m % nq] <= m // nq:
+                        continue
+                if (not three or gate_on_taken) and not s_free[t].test(j - 1, "issuer"):
+                    continue
+                if j > st["kv"]:
+                    if not kv_full[j % ST].test(j // ST, "issuer"):
+                        continue
+                    st["kv"] = j
+                issue("S", t, j, s_full[t])
+                ns[t] = j + 1
+                moved = True
+            for t in range(2):
+                j = np_[t]
+                if j < n_tiles and p_full[t].test(j, "issuer"):
+                    issue("PV", t, j, pv_done[t])
+                    np_[t] = j + 1
+                    moved = True
+            while st["ne"] < min(np_):
+                pipe.append(("commit", kv_empty[st["ne"] % ST]))
+                st["ne"] += 1
+                moved = True
+            if st["ne"] >= n_tiles:
+                pipe.append(("commit", o_final))
+                st["done"] = True
+                return True
+            return moved
+        return step
+
+    def softmax_warp(t, w):
+        rows = active[t][w]
+        st = {"j": 0, "pc": 0}
+        who = f"softmax {t}.{w}"
+
+        def step():
+            j, pc = st["j"], st["pc"]
+            if j >= n_tiles:
+                if pc == 0:
+                    if not o_final.test(0, who):
+                        return False
+                    st["pc"] = 1
+                    return True
+                return None
+            n, b = number(t, j), buffer(t, j)
+            if pc == 0:                           # S_t(j) computed
+                if not s_full[t].test(j, who):
+                    return False
+                if three and gate_on_taken:
+                    s_free[t].arrive(32)          # taken: S_t(j+1) may be issued
+                st["pc"] = 1
+            elif pc == 1:                         # first half of the scores
+                if rows and holds.get(b) != n:
+                    raise Violation(f"{who} reads S number {n}, buffer holds {holds.get(b)}")
+                st["pc"] = 2 if three or j == 0 else 10
+            elif pc == 10:                        # current: P_t free once PV_t(j-1) is done
+                if not pv_done[t].test(j - 1, who):
+                    return False
+                st["pc"] = 2
+            elif pc == 2:                         # second half
+                if rows and holds.get(b) != n:
+                    raise Violation(f"{who} reads S number {n}, buffer holds {holds.get(b)}")
+                if not three:
+                    s_free[t].arrive(32)          # current: S_t(j) read
+                st["pc"] = 3
+            elif pc == 3:                         # P stores complete
+                if rows:
+                    p_written.setdefault(n, set()).add(w)
+                st["pc"] = 4
+            elif pc == 4:                         # three_buffer: O_t free once PV_t(j-1) is done
+                if three and j > 0 and (rows or idle_warps_wait):
+                    if not pv_done[t].test(j - 1, who):
+                        return False
+                st["pc"] = 5
+            elif pc == 5:                         # rare O rescale, then P_t(j) handed over
+                if rows and j > 0 and rng.random() < 0.2:
+                    if ("PV", t, j - 1) not in ran or ("PV", t, j) in ran:
+                        raise Violation(f"{who} rescales O_{t} at tile {j} while a PV may run")
+                p_full[t].arrive(32)
+                st["j"], st["pc"] = j + 1, 0
+            return True
+        return step
+
+    def producer():
+        st = {"j": 0}
+
+        def step():
+            j = st["j"]
+            if j >= n_tiles:
+                return None
+            if j >= ST:
+                if not kv_empty[j % ST].test(j // ST - 1, "producer"):
+                    return False
+                for t in range(nq):
+                    for kind in ("S", "PV"):
+                        if (kind, t, j - ST) not in ran:
+                            raise Violation(f"stage reloaded before {kind}_{t}({j - ST}) ran")
+            stage[j % ST] = j
+            kv_full[j % ST].arrive()
+            st["j"] = j + 1
+            return True
+        return step
+
+    def tail_warp():
+        st = {"j": 0}
+
+        def step():
+            j = st["j"]
+            if j >= n_tiles:
+                return None
+            if not kv_full[j % ST].test(j // ST, "tail"):
+                return False
+            kv_empty[j % ST].arrive()
+            st["j"] = j + 1
+            return True
+        return step
+
+    def tensor_pipe():
+        if not pipe:
+            return False
+        execute(pipe.pop(0))
+        return True
+
+    actors = [issuer(), producer()]
+    actors += [softmax_warp(t, w) for t in range(nq) for w in range(4)]
+    actors += [tail_warp(), tail_warp()] if tail else []
+    finished = [False] * len(actors)
+    while True:
+        if all(finished) and not pipe:
+            return
+        order = list(range(len(actors) + 1))
+        rng.shuffle(order)
+        moved = False
+        for i in order:
+            if i == len(actors):
+                moved = tensor_pipe()
+            elif not finished[i]:
+                r = actors[i]()
+                if r is None:
+                    finished[i] = True
+                moved = bool(r)
+            if moved:
+                break
+        if not moved and not all(finished):
+            raise Violation("deadlock")
+
+
+def random_case(seed):
+    rng = random.Random(seed)
+    nq = rng.choice([1, 2])
+    active = [[True] * 4 for _ in range(2)]
+    if rng.random() < 0.5:   # a short frame: some warps have no valid rows
+        active = [[True] + [rng.random() < 0.5 for _ in range(3)] for _ in range(2)]
+    return dict(nq=nq, n_tiles=rng.randint(1, 10), active=active,
+                tail=nq == 2 and rng.random() < 0.5, seed=seed)
+
+
+def violations(schedule, cases, **rules):
+    found = []
+    for seed in range(cases):
+        try:
+            run(schedule, **random_case(seed), **rules)
+        except Violation as e:
+            found.append((seed, str(e)))
+    return found
+
+
+@pytest.mark.parametrize("schedule", ["current", "three_buffer"])
+def test_schedule_is_race_free(schedule):
+    assert violations(schedule, 1500) == []
+
+
+def test_three_buffer_schedule_needs_the_taken_gate():
+    """Without it S_t(j+1) may complete before softmax t has waited for
+    S_t(j): s_full_t runs two phases ahead and its parity wait loses count."""
+    found = violations("three_buffer", 300, gate_on_taken=False)
+    assert any("s_full" in msg for _, msg in found)
+
+
+def test_three_buffer_schedule_needs_idle_warps_to_wait():
+    """p_full_t counts arrivals, not tiles: warps without valid rows that
+    skip the per-tile PV wait run a tile ahead and complete the phase
+    before the other warps have written P."""
+    found = violations("three_buffer", 300, idle_warps_wait=False)
+    assert found
+    assert all(random_case(seed)["active"] != [[True] * 4] * 2 for seed, _ in found)
