@@ -1,4 +1,4 @@
-"""A randomised model of the attention kernel's mbarrier protocol (head_dim 64).
+"""A randomised model of the attention kernel's mbarrier protocol.
 
 The kernel's warps meet only at mbarriers and at the tensor pipe, so the
 protocol can be checked on the CPU: this model runs the MMA issuer's poll
@@ -16,9 +16,12 @@ every earlier MMA has run, in random interleavings. It checks:
   * a K/V stage is reloaded only after every MMA reading it ran;
   * nothing deadlocks.
 
-Two schedules are modelled. "current" is the kernel's: scores S_t, 16-bit
-P_t in separate TMEM columns, S_t(j+1) issued once softmax t has read S_t(j).
-"three_buffer" is a successor under consideration: P stored over its S,
+Three schedules are modelled. "current" is the kernel's for head_dim 64:
+scores S_t, 16-bit P_t in separate TMEM columns, S_t(j+1) issued once
+softmax t has read S_t(j). "head_dim_128" is the kernel's for head_dim 128:
+P_t stored over S_t, PV_t(j) issued once P_t(j) is written and S_t(j+1)
+right after it into the same columns, with no tail. "three_buffer" is a
+successor under consideration for head_dim 64: P stored over its S,
 three S/P buffers taken in turn, S number n issued once PV number n-3 has
 been issued. The model shows that the three-buffer schedule needs two rules
 (each test below drops one and finds the failure).
@@ -57,6 +60,8 @@ class Bar:
 def run(schedule, nq, n_tiles, active, tail, seed, gate_on_taken=True, idle_warps_wait=True):
     rng = random.Random(seed)
     three = schedule == "three_buffer"
+    h128 = schedule == "head_dim_128"
+    tail = tail and not h128          # head_dim 128 has no tail warps
     s_full = [Bar(f"s_full{t}", 1) for t in range(2)]
     s_free = [Bar(f"s_free{t}", 128) for t in range(2)]
     p_full = [Bar(f"p_full{t}", 128) for t in range(2)]
@@ -79,6 +84,8 @@ def run(schedule, nq, n_tiles, active, tail, seed, gate_on_taken=True, idle_warp
         if kind == "S":
             if three and n >= 3 and ("PV", (n - 3) % nq, (n - 3) // nq) not in ran:
                 raise Violation(f"S number {n} overwrites P before PV number {n - 3} ran")
+            if h128 and j > 0 and ("PV", t, j - 1) not in ran:
+                raise Violation(f"S_{t}({j}) overwrites P_{t}({j - 1}) before its PV ran")
             holds[buffer(t, j)] = n
         else:
             if p_written.get(n, set()) != {w for w in range(4) if active[t][w]}:
@@ -140,6 +147,46 @@ def run(schedule, nq, n_tiles, active, tail, seed, gate_on_taken=True, idle_warp
             return moved
         return step
 
+    def issuer_128():
+        """Serialized: per tile, per query tile, PV_t(j) once P_t(j) is written
+        and S_t(j+1) right after it; then the K/V stage is released."""
+        st = {"started": False, "done": False, "j": 0, "t": 0, "pv": False}
+
+        def step():
+            if st["done"]:
+                return None
+            if not st["started"]:
+                if not kv_full[0].test(0, "issuer"):
+                    return False
+                for t in range(nq):
+                    pipe.append(("S", t, 0))
+                    pipe.append(("commit", s_full[t]))
+                st["started"] = True
+                return True
+            j, t = st["j"], st["t"]
+            if not st["pv"]:
+                if not p_full[t].test(j, "issuer"):
+                    return False
+                pipe.append(("PV", t, j))      # no commit: S_t(j+1)'s covers it
+                st["pv"] = True
+                return True
+            if j + 1 < n_tiles:
+                if not kv_full[(j + 1) % ST].test((j + 1) // ST, "issuer"):
+                    return False
+                pipe.append(("S", t, j + 1))
+                pipe.append(("commit", s_full[t]))
+            st["pv"] = False
+            if t + 1 < nq:
+                st["t"] = t + 1
+                return True
+            pipe.append(("commit", kv_empty[j % ST]))
+            st["t"], st["j"] = 0, j + 1
+            if st["j"] >= n_tiles:
+                pipe.append(("commit", o_final))
+                st["done"] = True
+            return True
+        return step
+
     def softmax_warp(t, w):
         rows = active[t][w]
         st = {"j": 0, "pc": 0}
@@ -164,7 +211,7 @@ def run(schedule, nq, n_tiles, active, tail, seed, gate_on_taken=True, idle_warp
             elif pc == 1:                         # first half of the scores
                 if rows and holds.get(b) != n:
                     raise Violation(f"{who} reads S number {n}, buffer holds {holds.get(b)}")
-                st["pc"] = 2 if three or j == 0 else 10
+                st["pc"] = 2 if three or h128 or j == 0 else 10
             elif pc == 10:                        # current: P_t free once PV_t(j-1) is done
                 if not pv_done[t].test(j - 1, who):
                     return False
@@ -172,7 +219,7 @@ def run(schedule, nq, n_tiles, active, tail, seed, gate_on_taken=True, idle_warp
             elif pc == 2:                         # second half
                 if rows and holds.get(b) != n:
                     raise Violation(f"{who} reads S number {n}, buffer holds {holds.get(b)}")
-                if not three:
+                if not three and not h128:
                     s_free[t].arrive(32)          # current: S_t(j) read
                 st["pc"] = 3
             elif pc == 3:                         # P stores complete
@@ -233,7 +280,7 @@ def run(schedule, nq, n_tiles, active, tail, seed, gate_on_taken=True, idle_warp
         execute(pipe.pop(0))
         return True
 
-    actors = [issuer(), producer()]
+    actors = [issuer_128() if h128 else issuer(), producer()]
     actors += [softmax_warp(t, w) for t in range(nq) for w in range(4)]
     actors += [tail_warp(), tail_warp()] if tail else []
     finished = [False] * len(actors)
@@ -277,7 +324,7 @@ def violations(schedule, cases, **rules):
     return found
 
 
-@pytest.mark.parametrize("schedule", ["current", "three_buffer"])
+@pytest.mark.parametrize("schedule", ["current", "head_dim_128", "three_buffer"])
 def test_schedule_is_race_free(schedule):
     assert violations(schedule, 1500) == []
 
