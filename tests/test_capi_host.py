@@ -459,3 +459,44 @@ def test_object_api_checks_tensors_before_the_call(pkv):
     with pytest.raises(ValueError, match="dtype"):
         f16.append_frame(0, on_cpu, on_cpu)
     assert f16.fp16 and not c.fp16
+
+
+def test_inspection_calls_copy_at_most_cap_and_check_ranges(pkv):
+    """kv_get_page_table / kv_get_kv_tiles / kv_get_free_list write at most
+    `cap` entries and always report the full count; stream indices are
+    range-checked; a batch may hold at most KV_MAX_STREAMS streams."""
+    import ctypes
+    lib, E = pkv.capi.lib(), pkv.capi
+    h = mk(pkv, 2, 3, 16, 12)
+    for _ in range(7):
+        step(pkv, h)
+    p = pkv.kv_plan([h])
+    full, lpl_full = pkv.kv_get_page_table(p)
+    assert len(full) > 3
+    buf = (ctypes.c_int * 8)(*([-7] * 8))
+    n, lpl = ctypes.c_int(), ctypes.c_int()
+    assert lib.kv_get_page_table(p, 0, buf, 2, ctypes.byref(n), ctypes.byref(lpl)) == 0
+    assert n.value == len(full) and lpl.value == lpl_full
+    assert list(buf[:2]) == full[:2] and list(buf[2:]) == [-7] * 6
+    tiles = pkv.kv_get_kv_tiles(p)
+    row, lo, hi = ((ctypes.c_int * 4)(*([-7] * 4)) for _ in range(3))
+    assert lib.kv_get_kv_tiles(p, 0, row, lo, hi, 1, ctypes.byref(n)) == 0
+    assert n.value == len(tiles) and (row[0], lo[0], hi[0]) == tiles[0] and row[1] == -7
+    free = pkv.kv_get_free_list(h)
+    fb = (ctypes.c_int * 4)(*([-7] * 4))
+    assert lib.kv_get_free_list(h, fb, 1, ctypes.byref(n)) == 0
+    assert n.value == len(free) and fb[1] == -7
+    for bad in (-1, 1):
+        with pytest.raises(pkv.KVError) as e:
+            pkv.kv_get_page_table(p, bad)
+        assert e.value.code == E.KV_ERR_ARG
+        with pytest.raises(pkv.KVError) as e:
+            pkv.kv_get_kv_tiles(p, bad)
+        assert e.value.code == E.KV_ERR_ARG
+    pkv.kv_plan_free(p)
+    many = [h] * (pkv.KV_MAX_STREAMS + 1)
+    with pytest.raises(pkv.KVError) as e:
+        pkv.kv_plan(many)
+    assert e.value.code == E.KV_ERR_CAPACITY
+    assert pkv.kv_workspace_bytes(many) == 0
+    pkv.kv_destroy(h)
