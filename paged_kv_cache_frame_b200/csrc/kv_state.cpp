@@ -4,6 +4,7 @@
 #include <algorithm>
 #include <cstring>
 #include <functional>
+#include <queue>
 
 #include "../../include/kv.h"
 
@@ -350,12 +351,17 @@ int build_plan(const std::vector<const PageState*>& st, const PlanInputs& in, Ho
       }
       if ((int)costs.size() > target + n_base) break;
       std::sort(costs.begin(), costs.end(), std::greater<double>());
-      std::vector<double> slot(std::min<size_t>(target, costs.size()), 0.0);
+      // least-loaded slot first (a min-heap; tied slots are interchangeable,
+      // so the loads, and the makespan, do not depend on which one is taken)
+      std::priority_queue<double, std::vector<double>, std::greater<double>> slot;
+      for (size_t i = 0; i < std::min<size_t>(target, costs.size()); ++i) slot.push(0.0);
+      double makespan = 0.0;
       for (double x : costs) {
-        auto it = std::min_element(slot.begin(), slot.end());
-        *it += x;
+        const double load = slot.top() + x;
+        slot.pop();
+        slot.push(load);
+        makespan = std::max(makespan, load);
       }
-      const double makespan = *std::max_element(slot.begin(), slot.end());
       if (makespan < best * 0.995) {
         best = makespan;
         L = cand;
