@@ -148,7 +148,9 @@ int kv_bind_pool(kv_cache_t* c, int block, void* pool, void* stream);
  * themselves, and host-side tests).
  * Errors: KV_ERR_ARG, KV_ERR_ORDER (block appended twice in a step, or a
  * pending frame from an earlier step), KV_ERR_CAPACITY (no free patch page or
- * special stream full; the state is left unchanged), KV_ERR_CUDA. */
+ * special stream full; the state is left unchanged), KV_ERR_CUDA (the scatter
+ * launch failed after the page state advanced: the block counts as appended
+ * but its K/V are not in the pool; roll the frame back, or reset the cache). */
 int kv_append_frame(kv_cache_t* c, int block, const void* k, const void* v, void* stream);
 
 /* kv_evict_frames -- evict_frames ([P1] "Evicting Stale Frames"; [P2]
