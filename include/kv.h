@@ -150,7 +150,8 @@ int kv_bind_pool(kv_cache_t* c, int block, void* pool, void* stream);
  * pending frame from an earlier step), KV_ERR_CAPACITY (no free patch page or
  * special stream full; the state is left unchanged), KV_ERR_CUDA (the scatter
  * launch failed after the page state advanced: the block counts as appended
- * but its K/V are not in the pool; roll the frame back, or reset the cache). */
+ * but its K/V are not in the pool: roll a deferred frame back, else reset the
+ * cache). */
 int kv_append_frame(kv_cache_t* c, int block, const void* k, const void* v, void* stream);
 
 /* kv_evict_frames -- evict_frames ([P1] "Evicting Stale Frames"; [P2]
