@@ -88,6 +88,14 @@ typedef struct kv_stats {
   int special_tokens;
 } kv_stats;
 
+/* A cache's configuration as kv_init fixed it (patch_pages resolved). */
+typedef struct kv_config {
+  int max_pages, page_size, num_heads, head_dim, scale_frames, window, num_blocks, num_special, dtype;
+  int patch_pages;          /* patch pages [0, patch_pages); special pages after them */
+  int tokens_per_frame;     /* T = page_size + num_special: rows of k, v, q and out */
+  int cross_frame_special;  /* 1 while the special tokens of evicted frames stay visible */
+} kv_config;
+
 /* Execution-plan summary, for tests and benchmarks. */
 typedef struct kv_plan_stats {
   int n_streams;      /* requests in the plan */
@@ -148,10 +156,9 @@ int kv_bind_pool(kv_cache_t* c, int block, void* pool, void* stream);
  * themselves, and host-side tests).
  * Errors: KV_ERR_ARG, KV_ERR_ORDER (block appended twice in a step, or a
  * pending frame from an earlier step), KV_ERR_CAPACITY (no free patch page or
- * special stream full; the state is left unchanged), KV_ERR_CUDA (the scatter
- * launch failed after the page state advanced: the block counts as appended
- * but its K/V are not in the pool: roll a deferred frame back, else reset the
- * cache). */
+ * special stream full), KV_ERR_CUDA (the scatter launch failed). On every
+ * error the page state is left unchanged: the scatter is launched before the
+ * state advances, so after a failed launch the same call can be retried. */
 int kv_append_frame(kv_cache_t* c, int block, const void* k, const void* v, void* stream);
 
 /* kv_evict_frames -- evict_frames ([P1] "Evicting Stale Frames"; [P2]
@@ -183,6 +190,10 @@ int kv_rollback_last_frame(kv_cache_t* c);
 
 /* kv_get_stats -- get_cache_stats ([P3] "Monitoring Cache Statistics"). */
 int kv_get_stats(const kv_cache_t* c, kv_stats* out);
+
+/* kv_get_config -- the cache's configuration, for callers that size q, k, v
+ * and out ([T, H, D] per stream) from a cache handle. Errors: KV_ERR_ARG. */
+int kv_get_config(const kv_cache_t* c, kv_config* out);
 
 /* kv_get_free_list -- the free list bottom to top (the next page handed out is
  * ids[n-1]). Writes at most `cap` ids; *n gets the full length. */
@@ -277,9 +288,8 @@ int kv_set_cross_frame_special(kv_cache_t* cache, int on);
  * workspace.
  *
  * Arguments are as for kv_plan followed by kv_run. check != 0 also
- * synchronises `stream` and reads the kernels' error word, returning
- * KV_ERR_DEVICE_CHECK if a wait timed out. `stream` must belong to the
- * current device.
+ * synchronises `stream` and reads the kernels' error word (below).
+ * `stream` must belong to the current device.
  *
  * Memory and set-up:
  *   - The array is reserved on every device where the library's code is
@@ -287,8 +297,18 @@ int kv_set_cross_frame_special(kv_cache_t* cache, int on);
  *   - On the first call on a device, with that device current, the library
  *     looks up the array's device address. Make that first call before any
  *     stream capture on the device.
- *   - Each call rewrites the tables, and with them the zeroed error word, at
- *     the start of the array. Partials are written before they are read.
+ *   - Each call rewrites the tables at the start of the array. Partials are
+ *     written before they are read.
+ *   - The array's address is looked up once per device and kept. Do not call
+ *     kv_run_static on a device after cudaDeviceReset (or any other
+ *     destruction of its primary context) in the same process.
+ *
+ * Error word: the kernels of every call on a device OR their error bits into
+ * one word of the array, which starts at zero when the library is loaded.
+ * No call clears it except a call with check != 0, which reads it after
+ * synchronising `stream`, returns KV_ERR_DEVICE_CHECK if it is non-zero and
+ * then clears it. So an error raised by a call made with check == 0 is
+ * reported by the next call made with check != 0.
  *
  * Concurrency: every call on a device shares the array. Two calls that
  * overlap on the GPU (for example on two streams with no ordering between
@@ -301,6 +321,12 @@ int kv_set_cross_frame_special(kv_cache_t* cache, int on);
  * about 15 MB with automatic splitting. */
 int kv_run_static(kv_cache_t* const* caches, int n_streams, int block, int tiles_per_split,
                   const void* q, void* out, int check, void* stream);
+
+/* kv_testing_fail_launches -- for tests of the error paths only: the next n
+ * kernel launches the library makes (any call, any thread) return
+ * cudaErrorLaunchFailure, and so KV_ERR_CUDA, without launching anything.
+ * n <= 0 cancels. No device state is touched, so no GPU fault is involved. */
+void kv_testing_fail_launches(int n);
 
 /* kv_strerror -- static text for a status code. */
 const char* kv_strerror(int status);

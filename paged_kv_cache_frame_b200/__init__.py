@@ -28,9 +28,9 @@ __all__ = [
     "PagedKVCache", "Plan", "KVError", "workspace_bytes", "KV_BF16", "KV_FP16", "KV_MAX_STREAMS",
     "kv_init", "kv_destroy", "kv_reset", "kv_pool_bytes", "kv_bind_pool", "kv_append_frame",
     "kv_evict_frames", "kv_defer_eviction", "kv_commit_frame", "kv_rollback_last_frame",
-    "kv_get_stats", "kv_get_free_list", "kv_workspace_bytes", "kv_plan", "kv_run",
+    "kv_get_stats", "kv_get_config", "kv_get_free_list", "kv_workspace_bytes", "kv_plan", "kv_run",
     "kv_plan_free", "kv_get_page_table", "kv_get_kv_tiles", "kv_plan_get_stats",
-    "kv_check_device", "kv_strerror", "kv_last_error", "kv_run_static", "kv_set_cross_frame_special",
+    "kv_check_device", "kv_testing_fail_launches", "kv_strerror", "kv_last_error", "kv_run_static", "kv_set_cross_frame_special",
 ]
 
 
@@ -111,6 +111,12 @@ def kv_get_stats(c) -> dict:
     return {f: getattr(s, f) for f, _ in s._fields_}
 
 
+def kv_get_config(c) -> dict:
+    s = capi.kv_config()
+    capi.check(capi.lib().kv_get_config(c, ctypes.byref(s)), "kv_get_config")
+    return {f: getattr(s, f) for f, _ in s._fields_}
+
+
 def kv_get_free_list(c) -> list[int]:
     n = ctypes.c_int()
     capi.check(capi.lib().kv_get_free_list(c, None, 0, ctypes.byref(n)), "kv_get_free_list")
@@ -183,9 +189,28 @@ def kv_run_static(caches, block, q, out, tiles_per_split=0, check=False, stream=
     """kv_plan + kv_run for one block without any allocation: the plan tables
     and split-KV partials go to the library's static device array
     (KV_STATIC_SCRATCH_BYTES). For callers that cannot allocate device memory;
-    calls that overlap on the GPU share that array and race."""
-    capi.check(capi.lib().kv_run_static(_handles(caches), len(caches), block, tiles_per_split, _ptr(q),
+    calls that overlap on the GPU share that array and race.
+
+    caches: PagedKVCache objects or raw handles. Tensor q and out are checked
+    against the caches' configuration ([sum of T, H, D], the cache dtype,
+    contiguous, on a CUDA device) before the call, since the library would
+    read and write exactly that many rows at their addresses."""
+    handles = [c.handle if isinstance(c, PagedKVCache) else c for c in caches]
+    if handles:
+        cfgs = [kv_get_config(h) for h in handles]
+        c0 = cfgs[0]
+        shape = (sum(c["tokens_per_frame"] for c in cfgs), c0["num_heads"], c0["head_dim"])
+        fp16 = c0["dtype"] == KV_FP16
+        _check_tensor(q, "q", shape, fp16)
+        _check_tensor(out, "out", shape, fp16)
+    capi.check(capi.lib().kv_run_static(_handles(handles), len(handles), block, tiles_per_split, _ptr(q),
                                         _ptr(out), int(bool(check)), _stream(stream)), "kv_run_static")
+
+
+def kv_testing_fail_launches(n) -> None:
+    """Error-path tests only: the library's next n kernel launches fail with
+    KV_ERR_CUDA without launching (a fake of a failing launch)."""
+    capi.lib().kv_testing_fail_launches(int(n))
 
 
 def kv_strerror(status) -> str:

@@ -9,9 +9,7 @@ from __future__ import annotations
 import ctypes
 import os
 
-# PKV_LIB selects another build of the same library (e.g. an instrumented one).
-LIB_PATH = os.environ.get("PKV_LIB") or os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib",
-                                                     "libpkv.so")
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib", "libpkv.so")
 
 KV_OK = 0
 KV_ERR_ARG = -1
@@ -41,6 +39,12 @@ class kv_stats(ctypes.Structure):
     _fields_ = [("frame_count", ctypes.c_int), ("scale_pages", ctypes.c_int),
                 ("live_pages", ctypes.c_int), ("free_pages", ctypes.c_int),
                 ("special_tokens", ctypes.c_int)]
+
+
+class kv_config(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in (
+        "max_pages", "page_size", "num_heads", "head_dim", "scale_frames", "window", "num_blocks",
+        "num_special", "dtype", "patch_pages", "tokens_per_frame", "cross_frame_special")]
 
 
 class kv_plan_stats(ctypes.Structure):
@@ -75,6 +79,7 @@ SIGNATURES = {
     "kv_rollback_last_frame": (_I, [_P]),
     "kv_get_stats": (_I, [_P, ctypes.POINTER(kv_stats)]),
     "kv_get_free_list": (_I, [_P, _IP, _I, _IP]),
+    "kv_get_config": (_I, [_P, ctypes.POINTER(kv_config)]),
     "kv_workspace_bytes": (_SZ, [ctypes.POINTER(_P), _I]),
     "kv_plan": (_I, [ctypes.POINTER(_P), ctypes.POINTER(_P), _I, _I, _P, _SZ, _P]),
     "kv_run": (_I, [_P, _I, _P, _P, _P]),
@@ -85,6 +90,7 @@ SIGNATURES = {
     "kv_check_device": (_I, [_P, _P]),
     "kv_run_static": (_I, [ctypes.POINTER(_P), _I, _I, _I, _P, _P, _I, _P]),
     "kv_set_cross_frame_special": (_I, [_P, _I]),
+    "kv_testing_fail_launches": (None, [_I]),
     "kv_strerror": (ctypes.c_char_p, [_I]),
     "kv_last_error": (ctypes.c_char_p, []),
 }

@@ -6,6 +6,7 @@
 
 #include <algorithm>
 #include <cmath>
+#include <cstddef>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -14,6 +15,7 @@
 #include "../../include/kv.h"
 #include "kernels.h"
 #include "kv_state.h"
+#include "launch.cuh"
 
 struct kv_cache {
   pkv::PageState st;
@@ -88,7 +90,13 @@ int device_sms() {
 
 }  // namespace
 
+namespace pkv {
+std::atomic<int> g_fail_launches{0};
+}
+
 extern "C" {
+
+void kv_testing_fail_launches(int n) { pkv::g_fail_launches.store(n > 0 ? n : 0); }
 
 const char* kv_strerror(int status) {
   switch (status) {
@@ -171,26 +179,30 @@ int kv_append_frame(kv_cache_t* c, int block, const void* k, const void* v, void
     if (!c->bound[block]) return fail(KV_ERR_ARG, "kv_append_frame: no pool bound for this block");
     if (!aligned16(k) || !aligned16(v)) return fail(KV_ERR_ARG, "kv_append_frame: k/v not 16-byte aligned");
   }
+  // The scatter is launched before the page state advances, so a failed
+  // launch leaves the cache exactly as it was.
   int page = -1, sp0 = 0;
   std::string why;
-  const int rc = c->st.append(block, &page, &sp0, &why);
+  int rc = c->st.peek_append(block, &page, &sp0, &why);
   if (rc != KV_OK) return fail(rc, why);
-  if (!k) return KV_OK;
-  pkv::AppendArgs a;
-  a.k = k;
-  a.v = v;
-  a.pool = c->pools[block];
-  a.T = g.page_size + g.NS;
-  a.NS = g.NS;
-  a.page_size = g.page_size;
-  a.Np = g.Np;
-  a.max_pages = g.max_pages;
-  a.row_vecs = g.H * g.D * 2 / 16;
-  a.patch_page = page;
-  a.sp0 = sp0;
-  cudaError_t e = pkv::launch_append(a, (cudaStream_t)stream);
-  if (e != cudaSuccess) return cuda_fail(e, "kv_append_frame: scatter launch");
-  return KV_OK;
+  if (k) {
+    pkv::AppendArgs a;
+    a.k = k;
+    a.v = v;
+    a.pool = c->pools[block];
+    a.T = g.page_size + g.NS;
+    a.NS = g.NS;
+    a.page_size = g.page_size;
+    a.Np = g.Np;
+    a.max_pages = g.max_pages;
+    a.row_vecs = g.H * g.D * 2 / 16;
+    a.patch_page = page;
+    a.sp0 = sp0;
+    cudaError_t e = pkv::launch_append(a, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "kv_append_frame: scatter launch");
+  }
+  rc = c->st.append(block, &page, &sp0, &why);
+  return rc == KV_OK ? KV_OK : fail(rc, why);
 }
 
 int kv_evict_frames(kv_cache_t* c) {
@@ -217,6 +229,24 @@ int kv_rollback_last_frame(kv_cache_t* c) {
   std::string why;
   const int rc = c->st.rollback(&why);
   return rc == KV_OK ? rc : fail(rc, why);
+}
+
+int kv_get_config(const kv_cache_t* c, kv_config* out) {
+  if (!c || !out) return fail(KV_ERR_ARG, "kv_get_config: NULL argument");
+  const pkv::Config& g = c->st.cfg;
+  out->max_pages = g.max_pages;
+  out->page_size = g.page_size;
+  out->num_heads = g.H;
+  out->head_dim = g.D;
+  out->scale_frames = g.S;
+  out->window = g.W;
+  out->num_blocks = g.B;
+  out->num_special = g.NS;
+  out->dtype = g.dtype;
+  out->patch_pages = g.Np;
+  out->tokens_per_frame = g.page_size + g.NS;
+  out->cross_frame_special = c->st.cross_special ? 1 : 0;
+  return KV_OK;
 }
 
 int kv_get_stats(const kv_cache_t* c, kv_stats* out) {
@@ -429,7 +459,7 @@ static __device__ __align__(256) uint8_t g_static_scratch[KV_STATIC_SCRATCH_BYTE
 
 namespace {
 
-constexpr int kMaxDevices = 256;
+using pkv::kMaxDevices;
 std::mutex g_static_mu;
 void* g_static_addr[kMaxDevices] = {};   // device address of g_static_scratch, per device
 
@@ -496,13 +526,17 @@ extern "C" int kv_run_static(kv_cache_t* const* caches, int n_streams, int block
   pkv::KvPlanHeader& hd = p.hp.header;
   hd.off_part_o = (int64_t)off_o;
   hd.off_part_lse = (int64_t)off_lse;
-  hd.error = 0;   // uploaded with the tables: the kernels' error word starts at zero on every call
   std::memcpy(p.hp.image.data(), &hd, sizeof(hd));
 
   void* scratch = nullptr;
   rc = static_scratch(&scratch);
   if (rc != KV_OK) return rc;
-  cudaError_t e = pkv::upload_plan(scratch, p.hp.image.data(), p.hp.image.size(), (cudaStream_t)stream);
+  // Everything but the error word (the header's first word) is uploaded, so
+  // the word keeps the bits of earlier calls until a checking call clears it.
+  static_assert(offsetof(pkv::KvPlanHeader, error) == 0, "error word first");
+  constexpr size_t kW = sizeof(uint32_t);
+  cudaError_t e = pkv::upload_plan(static_cast<uint8_t*>(scratch) + kW, p.hp.image.data() + kW,
+                                   p.hp.image.size() - kW, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "kv_run_static: upload");
   for (int i = 0; i < n_streams; ++i) {
     p.caches.push_back(caches[i]);
@@ -521,6 +555,11 @@ extern "C" int kv_run_static(kv_cache_t* const* caches, int n_streams, int block
   uint32_t w = 0;
   e = cudaMemcpy(&w, scratch, sizeof(w), cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(e, "kv_run_static: read error word");
-  if (w) return fail(KV_ERR_DEVICE_CHECK, "kernel error word " + std::to_string(w));
+  if (w) {
+    const uint32_t zero = 0;
+    e = cudaMemcpy(scratch, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "kv_run_static: clear error word");
+    return fail(KV_ERR_DEVICE_CHECK, "kernel error word " + std::to_string(w));
+  }
   return KV_OK;
 }

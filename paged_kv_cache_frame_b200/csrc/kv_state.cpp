@@ -60,7 +60,7 @@ void PageState::commit_frame(const FramePage& fp) {
   ++committed;
 }
 
-int PageState::append(int block, int* page, int* sp0, std::string* why) {
+int PageState::peek_append(int block, int* page, int* sp0, std::string* why) const {
   if (block < 0 || block >= cfg.B) {
     *why = "append: block out of range";
     return KV_ERR_ARG;
@@ -79,6 +79,23 @@ int PageState::append(int block, int* page, int* sp0, std::string* why) {
       *why = "append: special stream full (raise max_pages)";
       return KV_ERR_CAPACITY;
     }
+    *page = free_.back();
+    *sp0 = sp_len;
+    return KV_OK;
+  }
+  if (appended[block]) {
+    *why = "append: block already appended in this frame step";
+    return KV_ERR_ORDER;
+  }
+  *page = step_page;
+  *sp0 = step_sp0;
+  return KV_OK;
+}
+
+int PageState::append(int block, int* page, int* sp0, std::string* why) {
+  const int rc = peek_append(block, page, sp0, why);
+  if (rc != KV_OK) return rc;
+  if (!step_open || n_appended == cfg.B) {
     const int pg = free_.back();
     free_.pop_back();
     step_sp0 = sp_len;
@@ -95,14 +112,9 @@ int PageState::append(int block, int* page, int* sp0, std::string* why) {
     std::fill(appended.begin(), appended.end(), 0);
     n_appended = 0;
     ++epoch;
-  } else if (appended[block]) {
-    *why = "append: block already appended in this frame step";
-    return KV_ERR_ORDER;
   }
   appended[block] = 1;
   ++n_appended;
-  *page = step_page;
-  *sp0 = step_sp0;
   return KV_OK;
 }
 

@@ -76,6 +76,10 @@ class PageState {
   // Marks `block` appended in the current step, opening a new step (and
   // taking a patch page and NS special slots) when needed.
   int append(int block, int* page, int* sp0, std::string* why);
+  // What append(block) would return (status, page, sp0), with no change to
+  // the state: lets a caller launch the scatter first and advance the state
+  // only once the launch has succeeded.
+  int peek_append(int block, int* page, int* sp0, std::string* why) const;
   int evict();
   int set_defer(int on, std::string* why);
   int commit(std::string* why);

@@ -8,14 +8,24 @@
 #pragma once
 #include <cuda_runtime.h>
 
+#include <atomic>
+#include <cstdint>
+
 namespace pkv {
 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
+// Launches still to be failed on purpose (kv_testing_fail_launches): a fake
+// of a failing launch for the host-side error-path tests.
+extern std::atomic<int> g_fail_launches;
+
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
                        Args&&... args) {
+  if (g_fail_launches.load(std::memory_order_relaxed) > 0 &&
+      g_fail_launches.fetch_sub(1, std::memory_order_relaxed) > 0)
+    return cudaErrorLaunchFailure;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -27,6 +37,24 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+constexpr int kMaxDevices = 256;
+
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) applies to the current
+// device only, so it is set once per (kernel, device). `done` is the caller's
+// per-kernel array of kMaxDevices flags. Two threads that race on a first
+// launch both set the attribute, which is harmless.
+template <typename F>
+cudaError_t ensure_dynamic_smem(F kern, int bytes, std::atomic<uint8_t>* done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done[dev].store(1, std::memory_order_release);
+  return e;
 }
 
 }  // namespace pkv

@@ -826,12 +826,9 @@ template <int D, bool kFP16, int STAGES>
 static cudaError_t launch_attn_t(const AttnMaps& maps, const AttnArgs& a, int n_units, cudaStream_t stream) {
   using L = AttnSmem<D, STAGES>;
   auto kern = paged_prefill_attn_kernel<D, kFP16, STAGES, kEmu>;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static std::atomic<uint8_t> configured[kMaxDevices];   // per device: smem attribute set
+  const cudaError_t e = ensure_dynamic_smem(kern, L::kAlloc, configured);
+  if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3(n_units), dim3(AttnRoles<D>::kThreads), L::kAlloc, stream, maps, a);
 }
 

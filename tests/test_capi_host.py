@@ -401,6 +401,42 @@ def test_run_static_argument_checks_before_any_device_work(pkv):
     pkv.kv_destroy(h)
 
 
+def test_run_static_python_checks_tensors_before_the_call(pkv):
+    """The kv_run_static binding takes q and out as tensors and checks them
+    against the caches' configuration ([sum of T, H, D], cache dtype,
+    contiguous, CUDA) before any library call, as Plan.run does: the library
+    would read and write exactly that many rows at their addresses."""
+    import torch
+    T, H, D = 16 + 6, 2, 64
+    c = pkv.PagedKVCache(8, 16, H, D, scale_frames=1, window=2, num_blocks=1)
+    c2 = pkv.PagedKVCache(8, 16, H, D, scale_frames=1, window=2, num_blocks=1)
+    for bad, what in [(torch.zeros(T + 1, H, D, dtype=torch.bfloat16), "shape"),
+                      (torch.zeros(T, H, D, dtype=torch.float16), "dtype"),
+                      (torch.zeros(H, T, D, dtype=torch.bfloat16).transpose(0, 1), "contiguous"),
+                      (torch.zeros(T, H, D, dtype=torch.bfloat16), "CUDA")]:
+        with pytest.raises(ValueError, match=what):
+            pkv.kv_run_static([c], 0, bad, bad)
+        with pytest.raises(ValueError, match=what):      # raw handles are checked the same way
+            pkv.kv_run_static([c.handle], 0, bad, bad)
+    # two streams: 2 T rows
+    with pytest.raises(ValueError, match="expected \\(44, 2, 64\\)"):
+        pkv.kv_run_static([c, c2], 0, torch.zeros(T, H, D, dtype=torch.bfloat16), None)
+
+
+def test_get_config_reports_what_init_fixed(pkv):
+    h = pkv.kv_init(90, 256, 16, 64, 8, 64, 24, num_special=6, dtype=pkv.KV_FP16)
+    cfg = pkv.kv_get_config(h)
+    assert cfg == {"max_pages": 90, "page_size": 256, "num_heads": 16, "head_dim": 64, "scale_frames": 8,
+                   "window": 64, "num_blocks": 24, "num_special": 6, "dtype": pkv.KV_FP16,
+                   "patch_pages": 73, "tokens_per_frame": 262, "cross_frame_special": 1}
+    pkv.kv_set_cross_frame_special(h, False)
+    assert pkv.kv_get_config(h)["cross_frame_special"] == 0
+    pkv.kv_destroy(h)
+    h = pkv.kv_init(100, 16, 2, 64, 2, 4, 1, patch_pages=88)
+    assert pkv.kv_get_config(h)["patch_pages"] == 88
+    pkv.kv_destroy(h)
+
+
 def test_cross_frame_special_setting_changes_the_visible_rows(pkv):
     """Switching cross-frame special retention changes what the next plan
     attends to (here: 2 patch frames of 16 plus 24 special tokens, then plus

@@ -265,3 +265,47 @@ def test_full_batched_ragged_sampled(pkv):
     for s, so in enumerate(oracles):
         got = out[s * wl.T:(s + 1) * wl.T][torch.as_tensor(rows)]
         assert_close(got, so.expected(rows), f"stream {s} age {ages[s]}")
+
+
+def test_failed_append_launch_leaves_state_unchanged(pkv):
+    """A scatter launch that fails (faked by kv_testing_fail_launches, so no
+    GPU fault is involved) leaves the page state exactly as it was, whether
+    the append would have opened a new frame step or not; the same call then
+    succeeds, and pool and attention match the oracle."""
+    wl = small(64, H=2, S=1, W=2, frames=8)
+    cache = new_cache(pkv, wl, num_blocks=2)
+    m = PageModel(wl.S, wl.W, wl.page_size, wl.max_pages, NS=wl.NS)
+    imgs = [PoolImage(m, wl.H, wl.D) for _ in range(2)]
+    frames = [Frames(wl, seed=61, block=b) for b in range(2)]
+
+    def state():
+        return cache.get_stats(), cache.free_list()
+
+    for f in range(6):
+        for b in range(2):
+            _, k, v = frames[b].get(f)
+            before = state()
+            pkv.kv_testing_fail_launches(1)
+            with pytest.raises(pkv.KVError) as e:
+                cache.append_frame(b, k.cuda(), v.cuda())
+            assert e.value.name == "CUDA"
+            assert state() == before, f"frame {f} block {b}"
+            cache.append_frame(b, k.cuda(), v.cuda())
+            if b == 0:
+                cache.evict_frames()
+                page, sp0 = m.append(f)
+                m.evict()
+            imgs[b].write(page, sp0, bits16(k), bits16(v))
+        assert cache.free_list() == m.free
+    for b in range(2):
+        pool = cache.pools[b].cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+        np.testing.assert_array_equal(pool, imgs[b].bits, err_msg=f"block {b}")
+    pkv.kv_testing_fail_launches(0)
+    so = StreamOracle(wl.S, wl.W, wl.NS, wl.P, wl.dtype, frames[1].bits)
+    for f in range(6):
+        so.begin_frame(f)
+    plan = pkv.Plan([cache], workspace(pkv, [cache]))
+    q = frames[1].get(5)[0].cuda()
+    out = plan.run(1, q)
+    plan.check_device()
+    assert_close(out, so.expected(), "after failed launches")
