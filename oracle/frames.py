@@ -27,14 +27,24 @@ Rules, each from the pages:
     committed. Commit makes it a normal frame and runs eviction; rollback
     discards it and its special tokens ([P2] "Flow-Based Keyframe Selection";
     [P4] "Deferred Eviction and Rollback Mechanism").
+  * Camera-only ([P2] "Configuration Parameters": kv_cache_camera_only
+    restricts the cache to camera tokens, excluding patches). The pages list
+    a frame's six special tokens as camera, register, scale ([P2] "Special
+    Stream (Append-Only)"); reading: slot 0 of the six is the camera token.
+    With camera-only on, attention sees no patch token and no register or
+    scale token: only the camera tokens among the special tokens that would
+    otherwise be visible. The frame lists themselves (what is cached, what
+    is evicted) do not change.
 """
 from __future__ import annotations
 
 
 class FrameListSim:
-    def __init__(self, S: int, W: int, NS: int = 6, cross_frame_special: bool = True):
+    def __init__(self, S: int, W: int, NS: int = 6, cross_frame_special: bool = True,
+                 camera_only: bool = False):
         self.S, self.W, self.NS = S, W, NS
         self.cross_frame_special = cross_frame_special
+        self.camera_only = camera_only
         self.C: list[int] = []
         self.resident: list[int] = []
         self.pending: int | None = None
@@ -83,19 +93,28 @@ class FrameListSim:
 
     # -- queries ----------------------------------------------------------
     def patch_frames(self) -> list[int]:
-        """Frames whose patch tokens are visible, oldest first."""
+        """Frames whose patch tokens are cached (resident, then pending), oldest
+        first: the visible patch frames unless camera-only is on."""
         return self.resident + ([self.pending] if self.pending is not None else [])
+
+    def attended_patch_frames(self) -> list[int]:
+        """Frames whose patch tokens attention sees: none with camera-only."""
+        return [] if self.camera_only else self.patch_frames()
 
     def visible_specials(self) -> list[tuple[int, int]]:
         """Visible special tokens as (frame, slot), in stream order."""
         if self.cross_frame_special:
-            return list(self.SP)
-        live = set(self.patch_frames())
-        return [(f, j) for (f, j) in self.SP if f in live]
+            out = list(self.SP)
+        else:
+            live = set(self.patch_frames())
+            out = [(f, j) for (f, j) in self.SP if f in live]
+        if self.camera_only:
+            out = [(f, j) for (f, j) in out if j == 0]
+        return out
 
     def visible_tokens(self, P: int) -> set:
         """Visible tokens as ('p', frame, patch_index) / ('s', frame, slot)."""
-        out = {("p", f, t) for f in self.patch_frames() for t in range(P)}
+        out = {("p", f, t) for f in self.attended_patch_frames() for t in range(P)}
         out.update(("s", f, j) for (f, j) in self.visible_specials())
         return out
 

@@ -29,6 +29,12 @@ oldest window frame, so those runs form at most two ranges of the stream
 (the scale frames' and the window's), and the table lists only special pages
 that hold a visible token.
 
+Camera-only ([P2] "Configuration Parameters"; the reading is stated in
+frames.py): the pages and free list behave as always, but attention sees only
+the camera token (slot 0) of each frame among the special tokens that would
+otherwise be visible, and no patch page; the table then lists only special
+pages holding a visible camera token.
+
 get_cache_stats keys ([P3] "Monitoring Cache Statistics"): frame_count,
 scale_pages, live_pages, free_pages, special_tokens.
 """
@@ -45,9 +51,11 @@ class OracleError(Exception):
 
 class PageModel:
     def __init__(self, S: int, W: int, page_size: int, max_pages: int,
-                 NS: int = 6, patch_pages: int | None = None, cross_frame_special: bool = True):
+                 NS: int = 6, patch_pages: int | None = None, cross_frame_special: bool = True,
+                 camera_only: bool = False):
         self.S, self.W, self.ps, self.NS = S, W, page_size, NS
         self.cross_frame_special = cross_frame_special
+        self.camera_only = camera_only
         self.Np = patch_pages if patch_pages else S + W + 1
         if self.Np < 1 or max_pages < self.Np + (1 if NS > 0 else 0):
             raise OracleError("CAPACITY", "pool too small")
@@ -136,12 +144,20 @@ class PageModel:
             out = out + [self.pending]
         return out
 
+    def attended_patch_pages(self) -> list[tuple[int, int]]:
+        """(frame, page) of the patch pages attention reads: none with camera-only."""
+        return [] if self.camera_only else self.patch_pages_visible()
+
     def visible_special_index(self) -> list[int]:
         """Stream indices j of the visible special tokens, ascending."""
         if self.cross_frame_special:
-            return list(range(self.sp_len))
-        live = {f for f, _ in self.patch_pages_visible()}
-        return [j for j in range(self.sp_len) if self.sp_owner[j][0] in live]
+            out = list(range(self.sp_len))
+        else:
+            live = {f for f, _ in self.patch_pages_visible()}
+            out = [j for j in range(self.sp_len) if self.sp_owner[j][0] in live]
+        if self.camera_only:
+            out = [j for j in out if self.sp_owner[j][1] == 0]
+        return out
 
     def page_table(self) -> tuple[list[int], int]:
         """(kv_indices, last_page_len) of the visible page table.
@@ -156,7 +172,7 @@ class PageModel:
         """
         if self.committed == 0 and self.pending is None:
             raise OracleError("EMPTY", "no frame")
-        patch = [p for _, p in self.patch_pages_visible()]
+        patch = [p for _, p in self.attended_patch_pages()]
         pages = sorted({j // self.ps for j in self.visible_special_index()})
         special = [self.Np + i for i in pages]
         table = patch + special
@@ -166,7 +182,7 @@ class PageModel:
         return table, last
 
     def visible_token_count(self) -> int:
-        return len(self.patch_pages_visible()) * self.ps + len(self.visible_special_index())
+        return len(self.attended_patch_pages()) * self.ps + len(self.visible_special_index())
 
     def stats(self) -> dict:
         pend = 1 if self.pending is not None else 0
@@ -188,7 +204,7 @@ class PageModel:
         if self.visible_token_count() == 0:
             return set()
         table, last = self.page_table()
-        owner = {p: f for f, p in self.patch_pages_visible()}
+        owner = {p: f for f, p in self.attended_patch_pages()}
         vis = set(self.visible_special_index())
         out = set()
         for n, p in enumerate(table):

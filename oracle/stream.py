@@ -31,8 +31,9 @@ def bits16(t) -> np.ndarray:
 class StreamOracle:
     """fetch(frame) -> (q, k, v) as [T, H, D] uint16 bit patterns."""
 
-    def __init__(self, S: int, W: int, NS: int, P: int, dtype: str, fetch, cross_frame_special: bool = True):
-        self.sim = FrameListSim(S, W, NS, cross_frame_special)
+    def __init__(self, S: int, W: int, NS: int, P: int, dtype: str, fetch, cross_frame_special: bool = True,
+                 camera_only: bool = False):
+        self.sim = FrameListSim(S, W, NS, cross_frame_special, camera_only)
         self.NS, self.P, self.dtype, self.fetch = NS, P, dtype, fetch
         self.patch_kv: dict[int, tuple[np.ndarray, np.ndarray]] = {}
         self.special_kv: dict[int, tuple[np.ndarray, np.ndarray]] = {}
@@ -72,7 +73,7 @@ class StreamOracle:
 
     def visible_kv(self):
         ks, vs = [], []
-        for f in self.sim.patch_frames():
+        for f in self.sim.attended_patch_frames():
             k, v = self.patch_kv[f]
             ks.append(k)
             vs.append(v)

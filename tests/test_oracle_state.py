@@ -292,3 +292,66 @@ def test_cross_frame_special_off_closed_form(S, W):
         assert len(on.visible_tokens(P)) == frames * P + NS * n
         if n <= S + W:   # nothing evicted yet: the two settings agree
             assert off.visible_tokens(P) == on.visible_tokens(P)
+
+
+def test_camera_only_worked_example():
+    """Tiny config (page 16, S=2, W=4, NS=6), 12 frames, camera-only: the
+    camera token is slot 0 of each frame's six, so the visible special stream
+    indices are the multiples of 6. With retention on: 0, 6, ..., 66 on
+    special pages 0 (0, 6, 12), 1 (18, 24, 30), 2 (36, 42), 3 (48, 54, 60)
+    and 4 (66); no patch page; the last page holds 72 - 64 = 8 written
+    tokens. With retention off only frames 0, 1 and 8..11 count: indices 0,
+    6, 48, 54, 60, 66 on special pages 0, 3, 4. Worked by hand."""
+    Np = 7
+    for xs, idx, pages in [(True, list(range(0, 72, 6)), [0, 1, 2, 3, 4]),
+                           (False, [0, 6, 48, 54, 60, 66], [0, 3, 4])]:
+        m = PageModel(2, 4, 16, max_pages=Np + 5, NS=6, cross_frame_special=xs, camera_only=True)
+        sim = FrameListSim(2, 4, 6, cross_frame_special=xs, camera_only=True)
+        for f in range(12):
+            m.append(f); m.evict()
+            sim.append(f); sim.evict()
+        table, lpl = m.page_table()
+        assert table == [Np + p for p in pages] and lpl == 8
+        assert m.visible_special_index() == idx
+        assert m.visible_token_count() == len(idx)
+        assert sim.visible_specials() == [(j // 6, 0) for j in idx]
+        assert m.visible_tokens() == sim.visible_tokens(16) == {("s", j // 6, 0) for j in idx}
+        # the cache itself is as without camera-only: same pages, stats, free list
+        plain = PageModel(2, 4, 16, max_pages=Np + 5, NS=6, cross_frame_special=xs)
+        for f in range(12):
+            plain.append(f); plain.evict()
+        assert m.snapshot() == plain.snapshot() and m.stats() == plain.stats()
+
+
+@pytest.mark.parametrize("S,W", [(0, 3), (2, 4), (8, 64)])
+def test_camera_only_closed_form(S, W):
+    """Camera-only sees exactly one token per frame whose special tokens are
+    visible: n with retention on, the visible frames with it off."""
+    for xs in (True, False):
+        sim = FrameListSim(S, W, 6, cross_frame_special=xs, camera_only=True)
+        for n in range(1, 3 * (S + W) + 5):
+            sim.append(n - 1); sim.evict()
+            frames = min(n, S) + min(max(n - S, 0), W)
+            assert len(sim.visible_tokens(16)) == (n if xs else frames)
+            assert sim.attended_patch_frames() == []
+
+
+@settings(max_examples=80, deadline=None)
+@given(ops=st.lists(st.sampled_from(["key", "key", "defer_keep", "defer_drop"]), min_size=1, max_size=40),
+       S=st.integers(0, 3), W=st.integers(0, 4), ps=st.sampled_from([5, 16, 130]), xs=st.booleans())
+def test_camera_only_page_model_matches_frame_list(ops, S, W, ps, xs):
+    m = PageModel(S, W, ps, max_pages=S + W + 1 + 6 * 40 // ps + 2, NS=6, cross_frame_special=xs,
+                  camera_only=True)
+    sim = FrameListSim(S, W, 6, cross_frame_special=xs, camera_only=True)
+    for f, op in enumerate(ops):
+        d = op != "key"
+        m.set_defer(d); sim.set_defer(d)
+        m.append(f); sim.append(f)
+        m.evict(); sim.evict()
+        assert m.visible_tokens() == sim.visible_tokens(ps)
+        if d:
+            if op == "defer_keep":
+                m.commit(); sim.commit()
+            else:
+                m.rollback(); sim.rollback()
+        assert m.visible_tokens() == sim.visible_tokens(ps)
