@@ -32,7 +32,7 @@ the pages print, closed forms, a library routine (PyTorch SDPA in float64) or
 brute force. No function here is "parity unpinned".
 """
 from .frames import FrameListSim
-from .pages import PageModel, PoolImage, OracleError
+from .pages import PageModel, PoolImage, OracleError, SharedPatchPool
 from . import attention
 
-__all__ = ["FrameListSim", "PageModel", "PoolImage", "OracleError", "attention"]
+__all__ = ["FrameListSim", "PageModel", "PoolImage", "OracleError", "SharedPatchPool", "attention"]

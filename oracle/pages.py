@@ -35,6 +35,14 @@ the camera token (slot 0) of each frame among the special tokens that would
 otherwise be visible, and no patch page; the table then lists only special
 pages holding a visible camera token.
 
+Shared pool ([P3] "Constant Memory with Two-Stream Paging": memory is bounded
+by max_patch_pages + max_special_pages). Several streams can share one pool
+per block: the patch pages [0, Np) and one LIFO free list are common, and
+each stream owns a fixed range of special pages [sp_base, sp_base + sp_pages)
+for its own special stream. Reading: a stream that is reset returns its scale
+pages (in frame order), then its window pages (oldest first), then a pending
+page to the common free list; nothing else changes for the other streams.
+
 get_cache_stats keys ([P3] "Monitoring Cache Statistics"): frame_count,
 scale_pages, live_pages, free_pages, special_tokens.
 """
@@ -49,21 +57,49 @@ class OracleError(Exception):
         self.code = code
 
 
+class SharedPatchPool:
+    """Patch pages [0, Np) and their LIFO free list, common to the page
+    models of several streams (initially [Np-1, ..., 0]: pops yield 0, 1, ...)."""
+
+    def __init__(self, Np: int):
+        self.Np = Np
+        self.free = list(range(Np - 1, -1, -1))
+
+
 class PageModel:
     def __init__(self, S: int, W: int, page_size: int, max_pages: int,
                  NS: int = 6, patch_pages: int | None = None, cross_frame_special: bool = True,
-                 camera_only: bool = False):
+                 camera_only: bool = False, shared: SharedPatchPool | None = None,
+                 sp_base: int | None = None, sp_pages: int | None = None):
+        """shared: the common patch pool of a group of streams (patch_pages is
+        then its size); sp_base, sp_pages: this stream's range of special
+        pages (default: every page after the patch pages)."""
         self.S, self.W, self.ps, self.NS = S, W, page_size, NS
         self.cross_frame_special = cross_frame_special
         self.camera_only = camera_only
-        self.Np = patch_pages if patch_pages else S + W + 1
-        if self.Np < 1 or max_pages < self.Np + (1 if NS > 0 else 0):
+        self.shared = shared
+        self.Np = shared.Np if shared else (patch_pages if patch_pages else S + W + 1)
+        self.sp_base = self.Np if sp_base is None else sp_base
+        self.sp_pages = max_pages - self.sp_base if sp_pages is None else sp_pages
+        if (self.Np < 1 or self.sp_base < self.Np or self.sp_base + self.sp_pages > max_pages
+                or self.sp_pages < (1 if NS > 0 else 0)):
             raise OracleError("CAPACITY", "pool too small")
         self.max_pages = max_pages
+        self._own_free: list[int] = []
+        self.scale, self.window, self.pending = [], [], None
         self.reset()
 
+    @property
+    def free(self) -> list[int]:
+        return self.shared.free if self.shared else self._own_free
+
     def reset(self) -> None:
-        self.free = list(range(self.Np - 1, -1, -1))
+        if self.shared:
+            # this stream's patch pages go back to the common free list
+            for _, p in self.scale + self.window + ([self.pending] if self.pending else []):
+                self.shared.free.append(p)
+        else:
+            self._own_free = list(range(self.Np - 1, -1, -1))
         self.scale: list[tuple[int, int]] = []    # (frame, page)
         self.window: list[tuple[int, int]] = []   # (frame, page), oldest first
         self.pending: tuple[int, int] | None = None
@@ -74,7 +110,7 @@ class PageModel:
 
     @property
     def special_capacity(self) -> int:
-        return (self.max_pages - self.Np) * self.ps
+        return self.sp_pages * self.ps
 
     # -- operations -------------------------------------------------------
     def append(self, f: int) -> tuple[int, int]:
@@ -174,7 +210,7 @@ class PageModel:
             raise OracleError("EMPTY", "no frame")
         patch = [p for _, p in self.attended_patch_pages()]
         pages = sorted({j // self.ps for j in self.visible_special_index()})
-        special = [self.Np + i for i in pages]
+        special = [self.sp_base + i for i in pages]
         table = patch + special
         if not table:   # scale_frames = window = 0 with retention off
             raise OracleError("EMPTY", "no visible token")
@@ -195,7 +231,7 @@ class PageModel:
         }
 
     def special_location(self, j: int) -> tuple[int, int]:
-        return self.Np + j // self.ps, j % self.ps
+        return self.sp_base + j // self.ps, j % self.ps
 
     def visible_tokens(self) -> set:
         """Visible tokens in the frame simulator's ('p', frame, t) / ('s', frame,
@@ -212,8 +248,8 @@ class PageModel:
             for t in range(cnt):
                 if p < self.Np:
                     out.add(("p", owner[p], t))
-                elif (p - self.Np) * self.ps + t in vis:
-                    out.add(("s",) + self.sp_owner[(p - self.Np) * self.ps + t])
+                elif (p - self.sp_base) * self.ps + t in vis:
+                    out.add(("s",) + self.sp_owner[(p - self.sp_base) * self.ps + t])
         return out
 
     def snapshot(self):
@@ -229,14 +265,16 @@ class PoolImage:
         self.m = model
         self.bits = np.zeros((model.max_pages, 2, model.ps, H, D), dtype=np.uint16)
 
-    def write(self, page: int, sp0: int, k_bits: np.ndarray, v_bits: np.ndarray) -> None:
+    def write(self, page: int, sp0: int, k_bits: np.ndarray, v_bits: np.ndarray, model=None) -> None:
         """k_bits, v_bits: [NS + P, H, D] uint16. Tokens 0..NS-1 are the frame's
-        special tokens, NS.. its patch tokens."""
-        NS, ps = self.m.NS, self.m.ps
+        special tokens, NS.. its patch tokens. model: the stream that appends
+        (for a pool shared by several streams), default the image's own."""
+        m = model or self.m
+        NS, ps = m.NS, m.ps
         for kv, x in ((0, k_bits), (1, v_bits)):
             self.bits[page, kv, :ps] = x[NS:NS + ps]
             for i in range(NS):
-                pg, slot = self.m.special_location(sp0 + i)
+                pg, slot = m.special_location(sp0 + i)
                 self.bits[pg, kv, slot] = x[i]
 
     def gather(self, kv_indices, last_page_len):

@@ -355,3 +355,88 @@ def test_camera_only_page_model_matches_frame_list(ops, S, W, ps, xs):
             else:
                 m.rollback(); sim.rollback()
         assert m.visible_tokens() == sim.visible_tokens(ps)
+
+
+def test_shared_pool_worked_example():
+    """Two streams A, B share 5 patch pages (S=1, W=1, page 4, NS=2); A's
+    special pages are 5-6, B's 7-8. Worked by hand, the common LIFO free
+    list starting [4, 3, 2, 1, 0]:
+      A0 takes 0, B0 takes 1, A1 takes 2, A2 takes 3 and evicts A1 (2 back),
+      B1 takes 2, B2 takes 4 and evicts B1 (2 back): free [2].
+      A's table [0, 3, 5, 6] (6 special tokens: 4 + 2), B's [1, 4, 7, 8].
+      Reset A: its scale page 0, then window page 3, go back: free [2, 0, 3].
+      B3 takes 3 and evicts B2 (4 back): free [2, 0, 4]; B's table [1, 3, 7, 8]
+      with the last page full (8 tokens). A0 again takes 4: table [4, 5]."""
+    from oracle import SharedPatchPool
+    pool = SharedPatchPool(5)
+    A = PageModel(1, 1, 4, 9, NS=2, shared=pool, sp_base=5, sp_pages=2)
+    B = PageModel(1, 1, 4, 9, NS=2, shared=pool, sp_base=7, sp_pages=2)
+
+    def step(m, f):
+        page, sp0 = m.append(f)
+        m.evict()
+        return page, sp0
+
+    assert [step(A, 0), step(B, 0), step(A, 1), step(A, 2)] == [(0, 0), (1, 0), (2, 2), (3, 4)]
+    assert pool.free == [4, 2]
+    assert [step(B, 1), step(B, 2)] == [(2, 2), (4, 4)]
+    assert pool.free == [2]
+    assert A.page_table() == ([0, 3, 5, 6], 2)
+    assert B.page_table() == ([1, 4, 7, 8], 2)
+    assert A.special_location(4) == (6, 0) and B.special_location(5) == (8, 1)
+    A.reset()
+    assert pool.free == [2, 0, 3]
+    assert step(B, 3) == (3, 6) and pool.free == [2, 0, 4]
+    assert B.page_table() == ([1, 3, 7, 8], 4)
+    assert step(A, 0) == (4, 0) and A.page_table() == ([4, 5], 2)
+    assert A.stats()["free_pages"] == B.stats()["free_pages"] == 2
+
+
+@settings(max_examples=80, deadline=None)
+@given(ops=st.lists(st.tuples(st.integers(0, 2), st.sampled_from(["key", "key", "defer_keep", "defer_drop",
+                                                                  "reset"])), min_size=1, max_size=60),
+       S=st.integers(0, 2), W=st.integers(0, 3))
+def test_shared_pool_partitions_the_patch_pages(ops, S, W):
+    """Every patch page is on the common free list or held by exactly one
+    stream (scale, window or pending page); each stream's visible set is what
+    its own frame-list simulator says; a stream alone in a pool of its own
+    size behaves exactly as a standalone page model."""
+    from oracle import SharedPatchPool
+    n, ps, Np = 3, 5, 3 * (S + W + 1)
+    pool = SharedPatchPool(Np)
+    ms = [PageModel(S, W, ps, Np + 3 * 20, NS=6, shared=pool, sp_base=Np + 20 * i, sp_pages=20) for i in range(n)]
+    sims = [FrameListSim(S, W, 6) for _ in range(n)]
+    nxt = [0] * n
+    for s_i, op in ops:
+        m, sim = ms[s_i], sims[s_i]
+        if op == "reset":
+            m.reset()
+            sims[s_i] = FrameListSim(S, W, 6)
+            nxt[s_i] = 0
+            continue
+        if m.sp_len + 6 > m.special_capacity:
+            continue
+        d = op != "key"
+        m.set_defer(d); sim.set_defer(d)
+        f = nxt[s_i]
+        m.append(f); sim.append(f)
+        m.evict(); sim.evict()
+        nxt[s_i] += 1
+        if d:
+            if op == "defer_keep":
+                m.commit(); sim.commit()
+            else:
+                m.rollback(); sim.rollback()
+                nxt[s_i] -= 1
+        held = [p for mm in ms for _, p in mm.patch_pages_visible()]
+        assert sorted(held + pool.free) == list(range(Np))
+        for mm, ss in zip(ms, sims):
+            assert mm.visible_tokens() == ss.visible_tokens(ps)
+    # one stream alone in a pool of its own size: the standalone model
+    solo_pool = SharedPatchPool(S + W + 1)
+    a = PageModel(S, W, ps, S + W + 1 + 20, NS=6, shared=solo_pool)
+    b = PageModel(S, W, ps, S + W + 1 + 20, NS=6)
+    for f in range(15):
+        for m in (a, b):
+            m.append(f); m.evict()
+        assert a.snapshot() == b.snapshot() and a.page_table() == b.page_table()
