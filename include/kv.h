@@ -91,9 +91,12 @@ typedef struct kv_stats {
 /* A cache's configuration as kv_init fixed it (patch_pages resolved). */
 typedef struct kv_config {
   int max_pages, page_size, num_heads, head_dim, scale_frames, window, num_blocks, num_special, dtype;
-  int patch_pages;          /* patch pages [0, patch_pages); special pages after them */
+  int patch_pages;          /* patch pages [0, patch_pages) (shared in a group) */
+  int special_base;         /* this stream's special pages [special_base, special_base + special_pages) */
+  int special_pages;
   int tokens_per_frame;     /* T = page_size + num_special: rows of k, v, q and out */
   int cross_frame_special;  /* 1 while the special tokens of evicted frames stay visible */
+  int camera_only;          /* 1 while attention sees only the camera tokens */
 } kv_config;
 
 /* Execution-plan summary, for tests and benchmarks. */
@@ -104,6 +107,11 @@ typedef struct kv_plan_stats {
   int n_kv_tiles;     /* 128-token K/V tiles summed over streams */
   int tiles_per_cta;  /* largest number of K/V tiles one CTA processes */
   long long visible_tokens; /* visible tokens summed over streams */
+  int fused_merge;    /* 1: split units are merged by their own CTAs (every CTA of
+                         the launch fits on the device at once), 0: by a merge launch */
+  int run_launches;   /* kernel launches of one kv_run / kv_run_append (1, or 2 with
+                         a merge launch) */
+  int upload_launches; /* kernel launches kv_plan made to upload the tables */
 } kv_plan_stats;
 
 /* kv_init -- create one stream's cache ([P1] "Implementation Example": the
@@ -125,6 +133,30 @@ typedef struct kv_plan_stats {
 int kv_init(kv_cache_t** out, int max_pages, int page_size, int num_heads, int head_dim,
             int scale_frames, int window, int num_blocks, int num_special, int dtype,
             int patch_pages);
+
+/* kv_init_group -- create n_streams caches that share one pool per block
+ * ([P3] "Constant Memory with Two-Stream Paging": memory is bounded by
+ * max_patch_pages + max_special_pages, here for all the streams together).
+ * The patch pages [0, patch_pages) and their LIFO free list are common to the
+ * streams: a stream takes a page when it appends a frame and returns it when
+ * it evicts, rolls back or resets, so pages left by one stream serve another.
+ * Stream i owns the special pages [patch_pages + i * special_pages,
+ * patch_pages + (i + 1) * special_pages) for its special stream.
+ *   out            array of n_streams handles (1 <= n_streams <= KV_MAX_STREAMS),
+ *                  each released with kv_destroy
+ *   patch_pages    0 = n_streams * (scale_frames + window + 1), enough for every
+ *                  stream at once; fewer pages give KV_ERR_CAPACITY on an append
+ *                  that finds the common list empty
+ *   special_pages  per stream; 0 = (max_pages - patch_pages) / n_streams
+ * Other arguments as kv_init. kv_bind_pool on any of the caches binds the
+ * block's pool for all of them (and zero-fills it: bind before the first
+ * append). kv_reset of one stream returns its scale pages (frame order), then
+ * its window pages (oldest first), then a pending page to the common list.
+ * Errors: KV_ERR_ARG, KV_ERR_CAPACITY (max_pages < patch_pages + n_streams *
+ * special_pages). No CUDA call is made. */
+int kv_init_group(kv_cache_t** out, int n_streams, int max_pages, int page_size, int num_heads, int head_dim,
+                  int scale_frames, int window, int num_blocks, int num_special, int dtype, int patch_pages,
+                  int special_pages);
 
 /* kv_destroy -- free the host state. Pools are not touched. NULL is ignored. */
 void kv_destroy(kv_cache_t* c);
@@ -239,6 +271,32 @@ int kv_plan(kv_plan_t** out, kv_cache_t* const* caches, int n_streams, int tiles
  * Errors: KV_ERR_ARG, KV_ERR_STALE_PLAN, KV_ERR_NOT_APPENDED, KV_ERR_CUDA. */
 int kv_run(const kv_plan_t* plan, int block, const void* q, void* out, void* stream);
 
+/* kv_begin_frame -- open a frame step without appending a block: the new
+ * frame takes its patch page and NS special slots now, as the first
+ * kv_append_frame of a step would ([P1] "Appending New Frames"). Then evict,
+ * plan, and append every block, each with kv_append_frame or kv_run_append.
+ * Errors: KV_ERR_ORDER (the open step still has blocks to append, or a
+ * pending frame of an earlier step), KV_ERR_CAPACITY (no free patch page or
+ * special stream full); the state is unchanged on error. Host only. */
+int kv_begin_frame(kv_cache_t* c);
+
+/* kv_run_append -- append_frame for block `block` followed by run() for it,
+ * in one kernel launch ([P1] "Appending New Frames", "FlashInfer Kernel
+ * Execution"). k, v, q, out: device [sum T, H, D] in the cache dtype, the
+ * streams' rows in plan order (as q for kv_run). The launch copies every
+ * stream's k, v rows into the block's pool (special tokens to the special
+ * stream, patch tokens to the frame's page, exactly as kv_append_frame does)
+ * and computes out as kv_run does, reading the frame's own K/V from k and v.
+ * The plan must have been built after the step was opened (kv_begin_frame,
+ * or a kv_append_frame of another block), and `block` must not be appended
+ * yet in that step; it counts as appended once the launch has been made.
+ * Errors: KV_ERR_ARG, KV_ERR_STALE_PLAN, KV_ERR_ORDER (no open step for the
+ * plan, or the block already appended), KV_ERR_CUDA. If the attention launch
+ * fails nothing was appended; if a merge launch after it fails, the block is
+ * appended and out is incomplete. */
+int kv_run_append(const kv_plan_t* plan, int block, const void* k, const void* v, const void* q,
+                  void* out, void* stream);
+
 /* kv_plan_free -- release a plan's host state. NULL is ignored. */
 void kv_plan_free(kv_plan_t* plan);
 
@@ -248,12 +306,20 @@ void kv_plan_free(kv_plan_t* plan);
 int kv_get_page_table(const kv_plan_t* plan, int stream_idx, int* indices, int cap, int* n,
                       int* last_page_len);
 
-/* kv_get_kv_tiles -- host copy of stream `stream_idx`'s K/V tile list, in
- * visible-table order. Tile t reads pool K rows [row[t], row[t] + 128) of the
+/* kv_get_kv_tiles -- host copy of stream `stream_idx`'s K/V tile list: the
+ * visible rows of earlier frames in visible-table order, then those of the
+ * open step's frame. Tile t reads pool K rows [row[t], row[t] + 128) of the
  * [max_pages * 2 * page_size]-row space (its V rows start page_size later);
  * columns [lo[t], hi[t]) of the tile are visible tokens, the rest are masked.
+ * krow (may be NULL): for a tile of the open step's frame, the row of the
+ * frame's k/v ([T, H, D]) that column 0 stands for (column c is row
+ * krow[t] + c; it can be negative, those columns being masked), which
+ * kv_run_append reads instead of the pool; INT32_MIN / 2 for other tiles.
+ * step (may be NULL): 1, or with camera-only NS: of [lo, hi) only columns
+ * lo, lo + step, ... are visible.
  * Writes at most `cap` entries per array; *n gets the full count. */
-int kv_get_kv_tiles(const kv_plan_t* plan, int stream_idx, int* row, int* lo, int* hi, int cap, int* n);
+int kv_get_kv_tiles(const kv_plan_t* plan, int stream_idx, int* row, int* lo, int* hi, int* krow, int* step,
+                    int cap, int* n);
 
 /* kv_plan_get_stats -- summary of the plan's schedule. */
 int kv_plan_get_stats(const kv_plan_t* plan, kv_plan_stats* out);
@@ -273,6 +339,21 @@ int kv_check_device(const kv_plan_t* plan, void* stream);
  * section is scale_frames = 0 in kv_init.
  * Errors: KV_ERR_ARG (NULL cache). */
 int kv_set_cross_frame_special(kv_cache_t* cache, int on);
+
+/* kv_set_camera_only -- kv_cache_camera_only ([P2] "Configuration
+ * Parameters": restrict the cache to camera tokens, excluding patches). The
+ * pages list a frame's six special tokens as camera, register and scale
+ * ([P2] "Special Stream (Append-Only)"); this library reads slot 0 of each
+ * frame's NS special tokens (token 0 of its k/v) as the camera token. With
+ * camera-only on (1), attention sees no patch token and only the camera
+ * tokens among the special tokens that would otherwise be visible (every
+ * frame's with cross-frame special retention on, the scale, window and
+ * pending frames' with it off); kv_get_page_table lists only the special
+ * pages that hold one. The page state is unchanged: patch pages are still
+ * taken, written and evicted as usual. Off (0) is the default. Takes effect
+ * for the next kv_plan (plans made before it become stale).
+ * Errors: KV_ERR_ARG (NULL cache). */
+int kv_set_camera_only(kv_cache_t* cache, int on);
 
 /* Size of the library-owned device array that kv_run_static uses as scratch. */
 #define KV_STATIC_SCRATCH_BYTES (32u << 20)

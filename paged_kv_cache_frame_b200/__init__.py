@@ -22,15 +22,16 @@ from __future__ import annotations
 import ctypes
 
 from . import capi
-from .capi import KVError, KV_BF16, KV_FP16, KV_MAX_STREAMS, KV_STATIC_SCRATCH_BYTES
+from .capi import KVError, KV_BF16, KV_FP16, KV_MAX_STREAMS, KV_NOT_CURRENT, KV_STATIC_SCRATCH_BYTES
 
 __all__ = [
     "PagedKVCache", "Plan", "KVError", "workspace_bytes", "KV_BF16", "KV_FP16", "KV_MAX_STREAMS",
-    "kv_init", "kv_destroy", "kv_reset", "kv_pool_bytes", "kv_bind_pool", "kv_append_frame",
+    "kv_init", "kv_init_group", "kv_destroy", "kv_reset", "kv_pool_bytes", "kv_bind_pool", "kv_append_frame",
     "kv_evict_frames", "kv_defer_eviction", "kv_commit_frame", "kv_rollback_last_frame",
     "kv_get_stats", "kv_get_config", "kv_get_free_list", "kv_workspace_bytes", "kv_plan", "kv_run",
-    "kv_plan_free", "kv_get_page_table", "kv_get_kv_tiles", "kv_plan_get_stats",
-    "kv_check_device", "kv_testing_fail_launches", "kv_strerror", "kv_last_error", "kv_run_static", "kv_set_cross_frame_special",
+    "kv_run_append", "kv_begin_frame", "kv_plan_free", "kv_get_page_table", "kv_get_kv_tiles",
+    "kv_plan_get_stats", "kv_check_device", "kv_testing_fail_launches", "kv_strerror",
+    "kv_last_error", "kv_run_static", "kv_set_cross_frame_special", "kv_set_camera_only",
 ]
 
 
@@ -62,6 +63,15 @@ def kv_init(max_pages, page_size, num_heads, head_dim, scale_frames, window, num
                                   scale_frames, window, num_blocks, num_special, dtype,
                                   patch_pages), "kv_init")
     return h.value
+
+
+def kv_init_group(n_streams, max_pages, page_size, num_heads, head_dim, scale_frames, window, num_blocks,
+                  num_special=6, dtype=KV_BF16, patch_pages=0, special_pages=0) -> list[int]:
+    hs = (ctypes.c_void_p * n_streams)()
+    capi.check(capi.lib().kv_init_group(hs, n_streams, max_pages, page_size, num_heads, head_dim, scale_frames,
+                                        window, num_blocks, num_special, dtype, patch_pages, special_pages),
+               "kv_init_group")
+    return [hs[i] for i in range(n_streams)]
 
 
 def kv_destroy(c) -> None:
@@ -103,6 +113,10 @@ def kv_rollback_last_frame(c) -> None:
 
 def kv_set_cross_frame_special(c, on) -> None:
     capi.check(capi.lib().kv_set_cross_frame_special(c, int(bool(on))), "kv_set_cross_frame_special")
+
+
+def kv_set_camera_only(c, on) -> None:
+    capi.check(capi.lib().kv_set_camera_only(c, int(bool(on))), "kv_set_camera_only")
 
 
 def kv_get_stats(c) -> dict:
@@ -150,6 +164,15 @@ def kv_run(plan, block, q, out, stream=None) -> None:
     capi.check(capi.lib().kv_run(plan, block, _ptr(q), _ptr(out), _stream(stream)), "kv_run")
 
 
+def kv_run_append(plan, block, k, v, q, out, stream=None) -> None:
+    capi.check(capi.lib().kv_run_append(plan, block, _ptr(k), _ptr(v), _ptr(q), _ptr(out), _stream(stream)),
+               "kv_run_append")
+
+
+def kv_begin_frame(c) -> None:
+    capi.check(capi.lib().kv_begin_frame(c), "kv_begin_frame")
+
+
 def kv_plan_free(plan) -> None:
     capi.lib().kv_plan_free(plan)
 
@@ -164,14 +187,19 @@ def kv_get_page_table(plan, stream_idx=0):
     return list(buf[: n.value]), lpl.value
 
 
-def kv_get_kv_tiles(plan, stream_idx=0):
+def kv_get_kv_tiles(plan, stream_idx=0, with_krow=False):
+    """[(row, lo, hi)] per tile; with_krow: [(row, lo, hi, krow, step)]
+    (krow = KV_NOT_CURRENT for tiles that are not the open step's frame; of
+    [lo, hi) only lo, lo + step, ... are visible)."""
     n = ctypes.c_int()
-    capi.check(capi.lib().kv_get_kv_tiles(plan, stream_idx, None, None, None, 0, ctypes.byref(n)),
+    capi.check(capi.lib().kv_get_kv_tiles(plan, stream_idx, None, None, None, None, None, 0, ctypes.byref(n)),
                "kv_get_kv_tiles")
     m = max(1, n.value)
-    row, lo, hi = (ctypes.c_int * m)(), (ctypes.c_int * m)(), (ctypes.c_int * m)()
-    capi.check(capi.lib().kv_get_kv_tiles(plan, stream_idx, row, lo, hi, n.value, ctypes.byref(n)),
+    row, lo, hi, kr, sp = ((ctypes.c_int * m)() for _ in range(5))
+    capi.check(capi.lib().kv_get_kv_tiles(plan, stream_idx, row, lo, hi, kr, sp, n.value, ctypes.byref(n)),
                "kv_get_kv_tiles")
+    if with_krow:
+        return [(row[i], lo[i], hi[i], kr[i], sp[i]) for i in range(n.value)]
     return [(row[i], lo[i], hi[i]) for i in range(n.value)]
 
 
@@ -257,18 +285,23 @@ class PagedKVCache:
     """One video stream's paged cache (all transformer blocks)."""
 
     def __init__(self, max_pages, page_size, num_heads, head_dim, scale_frames=8, window=64,
-                 num_blocks=1, num_special=6, dtype="bf16", patch_pages=0, cross_frame_special=True):
+                 num_blocks=1, num_special=6, dtype="bf16", patch_pages=0, cross_frame_special=True,
+                 camera_only=False, _handle=None, _pools=None):
         self.dtype = dtype
         self.fp16 = _is_fp16(dtype)
         code = KV_FP16 if self.fp16 else KV_BF16
-        self.handle = kv_init(max_pages, page_size, num_heads, head_dim, scale_frames, window,
-                              num_blocks, num_special, code, patch_pages)
+        self.handle = _handle if _handle is not None else kv_init(
+            max_pages, page_size, num_heads, head_dim, scale_frames, window, num_blocks, num_special, code,
+            patch_pages)
         self.max_pages, self.page_size = max_pages, page_size
         self.H, self.D, self.num_blocks, self.NS = num_heads, head_dim, num_blocks, num_special
         self.T = page_size + num_special
-        self.pools = [None] * num_blocks
+        # the block pools (a list shared by the caches of a group)
+        self.pools = _pools if _pools is not None else [None] * num_blocks
         if not cross_frame_special:
             kv_set_cross_frame_special(self.handle, False)
+        if camera_only:
+            kv_set_camera_only(self.handle, True)
 
     def __del__(self):
         h = getattr(self, "handle", None)
@@ -278,6 +311,21 @@ class PagedKVCache:
                 kv_destroy(h)
             except Exception:   # interpreter shutdown: the library may already be gone
                 pass
+
+    @classmethod
+    def group(cls, n_streams, max_pages, page_size, num_heads, head_dim, scale_frames=8, window=64,
+              num_blocks=1, num_special=6, dtype="bf16", patch_pages=0, special_pages=0,
+              cross_frame_special=True, camera_only=False):
+        """n_streams caches sharing one pool per block (kv_init_group): common
+        patch pages, a special-page range per stream. allocate_pools on any
+        of them allocates and binds the pools of all."""
+        code = KV_FP16 if _is_fp16(dtype) else KV_BF16
+        hs = kv_init_group(n_streams, max_pages, page_size, num_heads, head_dim, scale_frames, window,
+                           num_blocks, num_special, code, patch_pages, special_pages)
+        pools = [None] * num_blocks
+        return [cls(max_pages, page_size, num_heads, head_dim, scale_frames, window, num_blocks, num_special,
+                    dtype, cross_frame_special=cross_frame_special, camera_only=camera_only, _handle=h,
+                    _pools=pools) for h in hs]
 
     def pool_bytes(self) -> int:
         return kv_pool_bytes(self.handle)
@@ -290,7 +338,7 @@ class PagedKVCache:
             if not pool.is_contiguous() or pool.device.type != "cuda":
                 raise ValueError("pool: must be a contiguous CUDA tensor")
         kv_bind_pool(self.handle, block, pool, stream)
-        self.pools[block] = pool
+        self.pools[block] = pool   # shared list: every cache of a group sees it
 
     def allocate_pools(self, device="cuda", stream=None):
         """Allocate each block's pool [max_pages, 2, page_size, H, D] with torch and bind it."""
@@ -309,6 +357,11 @@ class PagedKVCache:
         _check_tensor(k, "k", shape, self.fp16)
         _check_tensor(v, "v", shape, self.fp16)
         kv_append_frame(self.handle, block, k, v, stream)
+
+    def begin_frame(self):
+        """Open a frame step (take the new frame's page and special slots)
+        before its blocks are appended, e.g. by Plan.run_append."""
+        kv_begin_frame(self.handle)
 
     def evict_frames(self):
         kv_evict_frames(self.handle)
@@ -362,6 +415,20 @@ class Plan:
             out = torch.empty_like(q)
         _check_tensor(out, "out", shape, self.fp16)
         kv_run(self.handle, block, q, out, stream)
+        return out
+
+    def run_append(self, block, k, v, q, out=None, stream=None):
+        """Append block `block`'s K/V of the open frame step and run its
+        attention in one launch. k, v, q (and out): [sum of the streams' T,
+        H, D] of the cache dtype, streams in plan order."""
+        shape = (self.rows, self.H, self.D)
+        for x, name in ((k, "k"), (v, "v"), (q, "q")):
+            _check_tensor(x, name, shape, self.fp16)
+        if out is None:
+            import torch
+            out = torch.empty_like(q)
+        _check_tensor(out, "out", shape, self.fp16)
+        kv_run_append(self.handle, block, k, v, q, out, stream)
         return out
 
     def page_table(self, stream_idx=0):

@@ -26,6 +26,7 @@ KV_BF16 = 0
 KV_FP16 = 1
 KV_MAX_STREAMS = 32
 KV_STATIC_SCRATCH_BYTES = 32 << 20
+KV_NOT_CURRENT = -0x40000000   # krow of a tile that is not the open step's frame
 
 ERR_NAMES = {
     KV_ERR_ARG: "ARG", KV_ERR_CAPACITY: "CAPACITY", KV_ERR_ORDER: "ORDER",
@@ -44,13 +45,16 @@ class kv_stats(ctypes.Structure):
 class kv_config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in (
         "max_pages", "page_size", "num_heads", "head_dim", "scale_frames", "window", "num_blocks",
-        "num_special", "dtype", "patch_pages", "tokens_per_frame", "cross_frame_special")]
+        "num_special", "dtype", "patch_pages", "special_base", "special_pages", "tokens_per_frame",
+        "cross_frame_special", "camera_only")]
 
 
 class kv_plan_stats(ctypes.Structure):
     _fields_ = [("n_streams", ctypes.c_int), ("n_ctas", ctypes.c_int),
                 ("n_split_units", ctypes.c_int), ("n_kv_tiles", ctypes.c_int),
-                ("tiles_per_cta", ctypes.c_int), ("visible_tokens", ctypes.c_longlong)]
+                ("tiles_per_cta", ctypes.c_int), ("visible_tokens", ctypes.c_longlong),
+                ("fused_merge", ctypes.c_int), ("run_launches", ctypes.c_int),
+                ("upload_launches", ctypes.c_int)]
 
 
 class KVError(RuntimeError):
@@ -68,6 +72,7 @@ _IP = ctypes.POINTER(ctypes.c_int)
 # name -> (restype, argtypes)
 SIGNATURES = {
     "kv_init": (_I, [ctypes.POINTER(_P), _I, _I, _I, _I, _I, _I, _I, _I, _I, _I]),
+    "kv_init_group": (_I, [ctypes.POINTER(_P), _I, _I, _I, _I, _I, _I, _I, _I, _I, _I, _I, _I]),
     "kv_destroy": (None, [_P]),
     "kv_reset": (_I, [_P]),
     "kv_pool_bytes": (_SZ, [_P]),
@@ -83,13 +88,16 @@ SIGNATURES = {
     "kv_workspace_bytes": (_SZ, [ctypes.POINTER(_P), _I]),
     "kv_plan": (_I, [ctypes.POINTER(_P), ctypes.POINTER(_P), _I, _I, _P, _SZ, _P]),
     "kv_run": (_I, [_P, _I, _P, _P, _P]),
+    "kv_run_append": (_I, [_P, _I, _P, _P, _P, _P, _P]),
+    "kv_begin_frame": (_I, [_P]),
     "kv_plan_free": (None, [_P]),
     "kv_get_page_table": (_I, [_P, _I, _IP, _I, _IP, _IP]),
-    "kv_get_kv_tiles": (_I, [_P, _I, _IP, _IP, _IP, _I, _IP]),
+    "kv_get_kv_tiles": (_I, [_P, _I, _IP, _IP, _IP, _IP, _IP, _I, _IP]),
     "kv_plan_get_stats": (_I, [_P, ctypes.POINTER(kv_plan_stats)]),
     "kv_check_device": (_I, [_P, _P]),
     "kv_run_static": (_I, [ctypes.POINTER(_P), _I, _I, _I, _P, _P, _I, _P]),
     "kv_set_cross_frame_special": (_I, [_P, _I]),
+    "kv_set_camera_only": (_I, [_P, _I]),
     "kv_testing_fail_launches": (None, [_I]),
     "kv_strerror": (ctypes.c_char_p, [_I]),
     "kv_last_error": (ctypes.c_char_p, []),

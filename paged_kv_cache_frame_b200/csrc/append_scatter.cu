@@ -5,7 +5,8 @@
 // Inference in LingBot-Map").
 //
 // k, v: [T, H, D]; token t < NS is special token sp0 + t of the stream,
-// stored at page Np + (sp0 + t) / page_size, slot (sp0 + t) % page_size;
+// stored at page sp_base + (sp0 + t) / page_size, slot (sp0 + t) % page_size
+// (sp_base: the stream's first special page);
 // token t >= NS is patch row t - NS of page `patch_page`. Pool
 // [max_pages, 2, page_size, H, D] with dimension 1 = K/V. One thread moves one
 // 16-byte vector; consecutive threads move consecutive vectors of a token row,
@@ -32,7 +33,7 @@ __global__ void __launch_bounds__(256) append_scatter_kernel(const AppendArgs a)
     int page, slot;
     if (t < a.NS) {
       const int j = a.sp0 + t;
-      page = a.Np + j / a.page_size;
+      page = a.sp_base + j / a.page_size;
       slot = j % a.page_size;
     } else {
       page = a.patch_page;

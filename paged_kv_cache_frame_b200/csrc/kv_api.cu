@@ -8,6 +8,7 @@
 #include <cmath>
 #include <cstddef>
 #include <cstring>
+#include <memory>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -17,11 +18,16 @@
 #include "kv_state.h"
 #include "launch.cuh"
 
-struct kv_cache {
-  pkv::PageState st;
+// The device pools of one cache, or of every cache of a group (shared).
+struct DevPools {
   std::vector<void*> pools;
   std::vector<CUtensorMap> maps;
   std::vector<uint8_t> bound;
+};
+
+struct kv_cache {
+  pkv::PageState st;
+  std::shared_ptr<DevPools> dev;
 };
 
 struct kv_plan {
@@ -132,10 +138,51 @@ int kv_init(kv_cache_t** out, int max_pages, int page_size, int num_heads, int h
     delete k;
     return fail(rc, why);
   }
-  k->pools.assign(num_blocks, nullptr);
-  k->maps.assign(num_blocks, CUtensorMap{});
-  k->bound.assign(num_blocks, 0);
+  k->dev = std::make_shared<DevPools>();
+  k->dev->pools.assign(num_blocks, nullptr);
+  k->dev->maps.assign(num_blocks, CUtensorMap{});
+  k->dev->bound.assign(num_blocks, 0);
   *out = k;
+  return KV_OK;
+}
+
+int kv_init_group(kv_cache_t** out, int n_streams, int max_pages, int page_size, int num_heads, int head_dim,
+                  int scale_frames, int window, int num_blocks, int num_special, int dtype, int patch_pages,
+                  int special_pages) {
+  if (!out) return fail(KV_ERR_ARG, "kv_init_group: out is NULL");
+  if (n_streams < 1 || n_streams > KV_MAX_STREAMS) return fail(KV_ERR_ARG, "kv_init_group: n_streams out of range");
+  for (int i = 0; i < n_streams; ++i) out[i] = nullptr;
+  if (head_dim % 8 != 0) return fail(KV_ERR_ARG, "kv_init_group: head_dim must be a multiple of 8");
+  if (patch_pages < 0 || special_pages < 0) return fail(KV_ERR_ARG, "kv_init_group: negative page count");
+  const int Np = patch_pages > 0 ? patch_pages : n_streams * (scale_frames + window + 1);
+  const int sp = special_pages > 0 ? special_pages : (max_pages - Np) / n_streams;
+  if ((long long)Np + (long long)n_streams * sp > max_pages || sp < (num_special > 0 ? 1 : 0))
+    return fail(KV_ERR_CAPACITY, "kv_init_group: max_pages < patch_pages + n_streams * special_pages");
+  auto pool = std::make_shared<pkv::PatchPool>();
+  pool->Np = Np;
+  pool->shared = true;
+  for (int p = Np - 1; p >= 0; --p) pool->free.push_back(p);
+  auto dev = std::make_shared<DevPools>();
+  dev->pools.assign(num_blocks, nullptr);
+  dev->maps.assign(num_blocks, CUtensorMap{});
+  dev->bound.assign(num_blocks, 0);
+  for (int i = 0; i < n_streams; ++i) {
+    pkv::Config c{max_pages, page_size, num_heads, head_dim, scale_frames, window, num_blocks, num_special, dtype,
+                  Np, Np + i * sp, sp};
+    kv_cache* k = new kv_cache();
+    std::string why;
+    const int rc = k->st.init(c, &why, pool);
+    if (rc != KV_OK) {
+      delete k;
+      for (int j = 0; j < i; ++j) {
+        delete out[j];
+        out[j] = nullptr;
+      }
+      return fail(rc, why);
+    }
+    k->dev = dev;
+    out[i] = k;
+  }
   return KV_OK;
 }
 
@@ -161,12 +208,12 @@ int kv_bind_pool(kv_cache_t* c, int block, void* pool, void* stream) {
   cudaError_t e = cudaMemsetAsync(pool, 0, kv_pool_bytes(c), (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "kv_bind_pool: memset");
   if (g.D % 64 == 0) {
-    const int rc = encode_rows_map(&c->maps[block], pool, g.H, g.D, (long long)g.max_pages * 2 * g.page_size,
+    const int rc = encode_rows_map(&c->dev->maps[block], pool, g.H, g.D, (long long)g.max_pages * 2 * g.page_size,
                                    g.dtype);
     if (rc != KV_OK) return rc;
   }
-  c->pools[block] = pool;
-  c->bound[block] = 1;
+  c->dev->pools[block] = pool;
+  c->dev->bound[block] = 1;
   return KV_OK;
 }
 
@@ -176,7 +223,7 @@ int kv_append_frame(kv_cache_t* c, int block, const void* k, const void* v, void
   const pkv::Config& g = c->st.cfg;
   if (block < 0 || block >= g.B) return fail(KV_ERR_ARG, "kv_append_frame: block out of range");
   if (k) {
-    if (!c->bound[block]) return fail(KV_ERR_ARG, "kv_append_frame: no pool bound for this block");
+    if (!c->dev->bound[block]) return fail(KV_ERR_ARG, "kv_append_frame: no pool bound for this block");
     if (!aligned16(k) || !aligned16(v)) return fail(KV_ERR_ARG, "kv_append_frame: k/v not 16-byte aligned");
   }
   // The scatter is launched before the page state advances, so a failed
@@ -189,11 +236,11 @@ int kv_append_frame(kv_cache_t* c, int block, const void* k, const void* v, void
     pkv::AppendArgs a;
     a.k = k;
     a.v = v;
-    a.pool = c->pools[block];
+    a.pool = c->dev->pools[block];
     a.T = g.page_size + g.NS;
     a.NS = g.NS;
     a.page_size = g.page_size;
-    a.Np = g.Np;
+    a.sp_base = g.sp_base;
     a.max_pages = g.max_pages;
     a.row_vecs = g.H * g.D * 2 / 16;
     a.patch_page = page;
@@ -244,8 +291,11 @@ int kv_get_config(const kv_cache_t* c, kv_config* out) {
   out->num_special = g.NS;
   out->dtype = g.dtype;
   out->patch_pages = g.Np;
+  out->special_base = g.sp_base;
+  out->special_pages = g.sp_pages;
   out->tokens_per_frame = g.page_size + g.NS;
   out->cross_frame_special = c->st.cross_special ? 1 : 0;
+  out->camera_only = c->st.camera_only ? 1 : 0;
   return KV_OK;
 }
 
@@ -256,7 +306,7 @@ int kv_get_stats(const kv_cache_t* c, kv_stats* out) {
   out->frame_count = s.committed + pend;
   out->scale_pages = (int)s.scale_.size();
   out->live_pages = (int)s.window_.size() + pend;
-  out->free_pages = (int)s.free_.size();
+  out->free_pages = (int)s.free_list().size();
   out->special_tokens = s.sp_len;
   return KV_OK;
 }
@@ -271,9 +321,19 @@ int kv_set_cross_frame_special(kv_cache_t* c, int on) {
   return KV_OK;
 }
 
+int kv_set_camera_only(kv_cache_t* c, int on) {
+  if (!c) return fail(KV_ERR_ARG, "kv_set_camera_only: NULL cache");
+  const bool v = on != 0;
+  if (c->st.camera_only != v) {
+    c->st.camera_only = v;
+    ++c->st.epoch;
+  }
+  return KV_OK;
+}
+
 int kv_get_free_list(const kv_cache_t* c, int* ids, int cap, int* n) {
   if (!c || !n || cap < 0 || (cap > 0 && !ids)) return fail(KV_ERR_ARG, "kv_get_free_list: bad argument");
-  const auto& f = c->st.free_;
+  const auto& f = c->st.free_list();
   *n = (int)f.size();
   for (int i = 0; i < (int)f.size() && i < cap; ++i) ids[i] = f[i];
   return KV_OK;
@@ -317,7 +377,7 @@ int kv_plan(kv_plan_t** out, kv_cache_t* const* caches, int n_streams, int tiles
   in.num_sms = workspace ? device_sms() : 148;
   in.ctas_per_sm = pkv::attention_ctas_per_sm(g.D);
   in.tiles_per_split = tiles_per_split;
-  in.tail_ok = pkv::attention_tail_ok(g.D);
+  in.max_tail_rows = pkv::attention_max_tail_rows(g.D);
   kv_plan_t* p = new kv_plan_t();
   std::string why;
   rc = pkv::build_plan(st, in, &p->hp, &why);
@@ -348,27 +408,52 @@ int kv_plan(kv_plan_t** out, kv_cache_t* const* caches, int n_streams, int tiles
 
 void kv_plan_free(kv_plan_t* plan) { delete plan; }
 
-int kv_run(const kv_plan_t* p, int block, const void* q, void* out, void* stream) {
-  if (!p || !q || !out) return fail(KV_ERR_ARG, "kv_run: NULL argument");
-  if (!p->ws) return fail(KV_ERR_ARG, "kv_run: host-only plan (built without a workspace)");
-  if (p->D != 64 && p->D != 128) return fail(KV_ERR_UNSUPPORTED, "kv_run: head_dim must be 64 or 128");
-  if (!aligned16(q) || !aligned16(out)) return fail(KV_ERR_ARG, "kv_run: q/out not 16-byte aligned");
+}  // extern "C"
+
+namespace {
+
+// kv_run, and kv_run_append when k and v are given: the launch then also
+// writes the open step's frame (block `block`'s K/V) into every request's pool
+// and reads that frame's tiles from k and v. Marks the block appended once
+// the attention launch has succeeded.
+int run_impl(const kv_plan_t* p, int block, const void* q, void* out, const void* k, const void* v,
+             void* stream, const char* who) {
+  const std::string w(who);
+  const bool append = k != nullptr;
+  if (!p || !q || !out) return fail(KV_ERR_ARG, w + ": NULL argument");
+  if (append != (v != nullptr)) return fail(KV_ERR_ARG, w + ": k and v must both be set");
+  if (!p->ws) return fail(KV_ERR_ARG, w + ": host-only plan (built without a workspace)");
+  if (p->D != 64 && p->D != 128) return fail(KV_ERR_UNSUPPORTED, w + ": head_dim must be 64 or 128");
+  if (!aligned16(q) || !aligned16(out)) return fail(KV_ERR_ARG, w + ": q/out not 16-byte aligned");
+  if (append && (!aligned16(k) || !aligned16(v))) return fail(KV_ERR_ARG, w + ": k/v not 16-byte aligned");
   const int B = p->caches[0]->st.cfg.B;
-  if (block < 0 || block >= B) return fail(KV_ERR_ARG, "kv_run: block out of range");
+  if (block < 0 || block >= B) return fail(KV_ERR_ARG, w + ": block out of range");
   pkv::AttnMaps maps;
   std::memset(&maps, 0, sizeof(maps));
+  pkv::AttnArgs a;
+  std::memset(&a, 0, sizeof(a));
   for (size_t r = 0; r < p->caches.size(); ++r) {
     const kv_cache* c = p->caches[r];
-    if (c->st.epoch != p->epochs[r]) return fail(KV_ERR_STALE_PLAN, "kv_run: cache state changed after kv_plan");
-    if (!c->st.is_appended(block)) return fail(KV_ERR_NOT_APPENDED, "kv_run: block not appended in this step");
-    if (!c->bound[block]) return fail(KV_ERR_ARG, "kv_run: no pool bound for this block");
-    maps.kv[r] = c->maps[block];
+    if (c->st.epoch != p->epochs[r]) return fail(KV_ERR_STALE_PLAN, w + ": cache state changed after kv_plan");
+    if (!c->dev->bound[block]) return fail(KV_ERR_ARG, w + ": no pool bound for this block");
+    if (append) {
+      // the plan's frame step must be open with this block still to append
+      const pkv::PageState& st = c->st;
+      if (!st.step_open || st.n_appended == st.cfg.B || p->hp.reqs[r].cur_page != st.step_page)
+        return fail(KV_ERR_ORDER, w + ": no open frame step for this plan (call kv_begin_frame before kv_plan)");
+      if (st.appended[block]) return fail(KV_ERR_ORDER, w + ": block already appended in this frame step");
+      a.pools[r] = c->dev->pools[block];
+    } else if (!c->st.is_appended(block)) {
+      return fail(KV_ERR_NOT_APPENDED, w + ": block not appended in this step");
+    }
+    maps.kv[r] = c->dev->maps[block];
   }
   int rc = encode_rows_map(&maps.q, q, p->H, p->D, p->total_T, p->dtype);
+  if (rc == KV_OK && append) rc = encode_rows_map(&maps.k, k, p->H, p->D, p->total_T, p->dtype);
+  if (rc == KV_OK && append) rc = encode_rows_map(&maps.v, v, p->H, p->D, p->total_T, p->dtype);
   if (rc != KV_OK) return rc;
   uint8_t* ws = static_cast<uint8_t*>(p->ws);
   const pkv::KvPlanHeader& hd = p->hp.header;
-  pkv::AttnArgs a;
   a.q = q;
   a.reqs = reinterpret_cast<const pkv::KvReq*>(ws + hd.off_reqs);
   a.units = reinterpret_cast<const pkv::KvUnit*>(ws + hd.off_units);
@@ -377,11 +462,26 @@ int kv_run(const kv_plan_t* p, int block, const void* q, void* out, void* stream
   a.part_lse = reinterpret_cast<float*>(ws + hd.off_part_lse);
   a.out = out;
   a.err = reinterpret_cast<uint32_t*>(ws);
+  a.groups = reinterpret_cast<uint32_t*>(ws + hd.off_groups);
+  a.fused_merge = hd.fused_merge;
   a.H = p->H;
   a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)p->D));
+  a.fused_append = append ? 1 : 0;
+  a.n_reqs = (int)p->caches.size();
+  a.row_vecs = p->H * p->D * 2 / 16;
+  a.k = k;
+  a.v = v;
   cudaError_t e = pkv::launch_attention(maps, a, p->D, p->dtype == KV_FP16, hd.n_units, (cudaStream_t)stream);
-  if (e != cudaSuccess) return cuda_fail(e, "kv_run: attention launch");
-  if (hd.n_merge > 0) {
+  if (e != cudaSuccess) return cuda_fail(e, (w + ": attention launch").c_str());
+  if (append) {
+    // the launch writes the frame into the pools: the block is appended
+    for (kv_cache* c : p->caches) {
+      int page = 0, sp0 = 0;
+      std::string why;
+      c->st.append(block, &page, &sp0, &why);
+    }
+  }
+  if (hd.n_merge > 0 && !hd.fused_merge) {
     pkv::MergeArgs m;
     m.items = reinterpret_cast<const pkv::KvMergeItem*>(ws + hd.off_merge);
     m.part_o = a.part_o;
@@ -390,9 +490,30 @@ int kv_run(const kv_plan_t* p, int block, const void* q, void* out, void* stream
     m.H = p->H;
     m.n_items = hd.n_merge;
     e = pkv::launch_merge(m, p->D, p->dtype == KV_FP16, (cudaStream_t)stream);
-    if (e != cudaSuccess) return cuda_fail(e, "kv_run: merge launch");
+    if (e != cudaSuccess) return cuda_fail(e, (w + ": merge launch").c_str());
   }
   return KV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int kv_run(const kv_plan_t* p, int block, const void* q, void* out, void* stream) {
+  return run_impl(p, block, q, out, nullptr, nullptr, stream, "kv_run");
+}
+
+int kv_run_append(const kv_plan_t* p, int block, const void* k, const void* v, const void* q, void* out,
+                  void* stream) {
+  if (!k || !v) return fail(KV_ERR_ARG, "kv_run_append: NULL k/v");
+  return run_impl(p, block, q, out, k, v, stream, "kv_run_append");
+}
+
+int kv_begin_frame(kv_cache_t* c) {
+  if (!c) return fail(KV_ERR_ARG, "kv_begin_frame: NULL cache");
+  std::string why;
+  const int rc = c->st.begin_frame(&why);
+  return rc == KV_OK ? rc : fail(rc, why);
 }
 
 int kv_get_page_table(const kv_plan_t* p, int stream_idx, int* indices, int cap, int* n, int* last_page_len) {
@@ -407,7 +528,8 @@ int kv_get_page_table(const kv_plan_t* p, int stream_idx, int* indices, int cap,
   return KV_OK;
 }
 
-int kv_get_kv_tiles(const kv_plan_t* p, int stream_idx, int* row, int* lo, int* hi, int cap, int* n) {
+int kv_get_kv_tiles(const kv_plan_t* p, int stream_idx, int* row, int* lo, int* hi, int* krow, int* step, int cap,
+                    int* n) {
   if (!p || !n || cap < 0 || (cap > 0 && (!row || !lo || !hi))) return fail(KV_ERR_ARG, "kv_get_kv_tiles: bad argument");
   if (stream_idx < 0 || stream_idx >= (int)p->hp.reqs.size()) return fail(KV_ERR_ARG, "kv_get_kv_tiles: stream out of range");
   int t0 = 0;
@@ -419,6 +541,8 @@ int kv_get_kv_tiles(const kv_plan_t* p, int stream_idx, int* row, int* lo, int* 
     row[i] = t.row;
     lo[i] = t.lo;
     hi[i] = t.hi;
+    if (krow) krow[i] = t.krow;
+    if (step) step[i] = t.step;
   }
   return KV_OK;
 }
@@ -431,6 +555,10 @@ int kv_plan_get_stats(const kv_plan_t* p, kv_plan_stats* out) {
   out->n_kv_tiles = (int)p->hp.tiles.size();
   out->tiles_per_cta = p->hp.max_tiles_per_cta;
   out->visible_tokens = p->hp.visible;
+  out->fused_merge = p->hp.header.fused_merge;
+  out->run_launches = (p->hp.header.n_units > 0 ? 1 : 0) +
+                      (p->hp.header.n_merge > 0 && !p->hp.header.fused_merge ? 1 : 0);
+  out->upload_launches = p->ws ? pkv::upload_launches(p->hp.image.size()) : 0;
   return KV_OK;
 }
 
@@ -498,7 +626,7 @@ extern "C" int kv_run_static(kv_cache_t* const* caches, int n_streams, int block
   if (block < 0 || block >= g.B) return fail(KV_ERR_ARG, "kv_run_static: block out of range");
   for (int i = 0; i < n_streams; ++i) {
     if (!caches[i]->st.is_appended(block)) return fail(KV_ERR_NOT_APPENDED, "kv_run_static: block not appended in this step");
-    if (!caches[i]->bound[block]) return fail(KV_ERR_ARG, "kv_run_static: no pool bound for this block");
+    if (!caches[i]->dev->bound[block]) return fail(KV_ERR_ARG, "kv_run_static: no pool bound for this block");
   }
 
   kv_plan_t p;
@@ -506,7 +634,7 @@ extern "C" int kv_run_static(kv_cache_t* const* caches, int n_streams, int block
   in.num_sms = device_sms();
   in.ctas_per_sm = pkv::attention_ctas_per_sm(g.D);
   in.tiles_per_split = tiles_per_split;
-  in.tail_ok = pkv::attention_tail_ok(g.D);
+  in.max_tail_rows = pkv::attention_max_tail_rows(g.D);
   std::string why;
   rc = pkv::build_plan(st, in, &p.hp, &why);
   if (rc != KV_OK) return fail(rc, "kv_run_static: " + why);

@@ -18,15 +18,36 @@ struct KvReq {
   int32_t T;          // query rows (tokens of the frame)
   int32_t page_size;  // tokens per page of this request's pool
   int32_t n_tiles;    // K/V tiles in the visible table
+  // where the open step's frame goes in the pool (for a launch that appends it)
+  int32_t cur_page;   // its patch page (-1: no open step)
+  int32_t cur_sp0;    // its first special token in the special stream
+  int32_t sp_base;    // the stream's first special page (special token j: page sp_base + j / page_size)
+  int32_t NS;         // special tokens per frame
 };
 
 // 128 consecutive pool rows of one page, starting at K row `row` of the
 // [pages * 2 * page_size] row space of the pool; V rows start page_size
 // later. Columns [lo, hi) of the tile are visible tokens, the rest masked.
+//
+// Tiles of the current frame (the frame the open step appended) also carry
+// krow: column c of the tile is row krow + c of the frame's own k/v
+// ([T, H, D], tokens 0..NS-1 special), so a launch that appends the frame
+// itself can read those rows from k/v instead of the pool. krow can be
+// negative when the box is anchored before the frame's first row (those
+// columns are masked, and a TMA load fills negative rows with zeros). Other
+// tiles have krow = kNotCurrent.
+//
+// With step > 1 only every step-th column from lo on is visible (lo, lo +
+// step, ... < hi): the camera tokens of the special stream when the cache is
+// camera-only.
+constexpr int32_t kNotCurrent = -0x40000000;   // INT32_MIN / 2
 struct KvTile {
   int32_t row;
   int16_t lo;
   int16_t hi;
+  int32_t krow;
+  int16_t step;
+  int16_t pad;
 };
 
 // One CTA of the attention launch: one or two consecutive 128-row query
@@ -38,10 +59,13 @@ struct KvUnit {
   int16_t qtile;       // first query tile: rows [qtile*128, qtile*128 + 128)
   int16_t nq;          // full query tiles in the unit (1 or 2)
   int16_t tail_rows;   // rows of the tail tile qtile + nq (0 = none)
+  int16_t chunk;       // this CTA's chunk of a split group (0 if not split)
+  int16_t n_chunks;    // CTAs of the group (1 = not split)
   int16_t pad;
   int32_t tile_begin;  // absolute index into the tile table
   int32_t tile_end;
   int32_t slot[3];     // per query tile (tail last): -1 = write `out`, else partial slot
+  int32_t group;       // split group (index of its two counters), -1 if not split
 };
 
 constexpr int kMaxTailRows = 16;   // tail rows computed with swapped operands (N = 16)
@@ -65,6 +89,9 @@ struct KvPlanHeader {
   int32_t off_reqs, off_units, off_merge, off_tiles;  // byte offsets from the header
   int32_t upload_bytes;
   int64_t off_part_o, off_part_lse;                    // byte offsets from the header
+  int32_t n_groups;      // split groups
+  int32_t off_groups;    // byte offset of the groups' counters: [n_groups][2] uint32, zero
+  int32_t fused_merge;   // 1: the attention CTAs of a split group merge it themselves
 };
 
 }  // namespace pkv

@@ -15,7 +15,12 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline int ceil_div(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
 }  // namespace
 
-int PageState::init(const Config& c, std::string* why) {
+int PageState::init(const Config& c0, std::string* why, std::shared_ptr<PatchPool> pool) {
+  Config c = c0;
+  if (c.sp_base == 0 && c.sp_pages == 0) {
+    c.sp_base = c.Np;
+    c.sp_pages = c.max_pages - c.Np;
+  }
   if (c.page_size < 1 || c.H < 1 || c.D < 1 || c.S < 0 || c.W < 0 || c.B < 1 || c.NS < 0 ||
       c.max_pages < 1 || (c.dtype != KV_BF16 && c.dtype != KV_FP16) || c.Np < 1) {
     *why = "kv_init: invalid argument";
@@ -25,18 +30,30 @@ int PageState::init(const Config& c, std::string* why) {
     *why = "kv_init: pool row count exceeds int32";
     return KV_ERR_ARG;
   }
-  if (c.max_pages < c.Np + (c.NS > 0 ? 1 : 0)) {
+  if (c.sp_base < c.Np || c.sp_pages < (c.NS > 0 ? 1 : 0) || c.sp_base + c.sp_pages > c.max_pages) {
     *why = "kv_init: max_pages must leave at least one special page after the patch pages";
     return KV_ERR_CAPACITY;
   }
   cfg = c;
+  if (pool) {
+    patch_ = pool;
+  } else {
+    patch_ = std::make_shared<PatchPool>();
+    patch_->Np = c.Np;
+  }
   reset();
   return KV_OK;
 }
 
 void PageState::reset() {
-  free_.clear();
-  for (int p = cfg.Np - 1; p >= 0; --p) free_.push_back(p);
+  if (patch_->shared) {
+    for (const auto& fp : scale_) patch_->free.push_back(fp.page);
+    for (const auto& fp : window_) patch_->free.push_back(fp.page);
+    if (has_pending) patch_->free.push_back(pending_.page);
+  } else {
+    patch_->free.clear();
+    for (int p = cfg.Np - 1; p >= 0; --p) patch_->free.push_back(p);
+  }
   scale_.clear();
   window_.clear();
   has_pending = false;
@@ -71,7 +88,7 @@ int PageState::peek_append(int block, int* page, int* sp0, std::string* why) con
       *why = "append: the deferred frame of the previous step must be committed or rolled back";
       return KV_ERR_ORDER;
     }
-    if (free_.empty()) {
+    if (patch_->free.empty()) {
       *why = "append: no free patch page (patch_pages too small for S + W)";
       return KV_ERR_CAPACITY;
     }
@@ -79,7 +96,7 @@ int PageState::peek_append(int block, int* page, int* sp0, std::string* why) con
       *why = "append: special stream full (raise max_pages)";
       return KV_ERR_CAPACITY;
     }
-    *page = free_.back();
+    *page = patch_->free.back();
     *sp0 = sp_len;
     return KV_OK;
   }
@@ -92,26 +109,42 @@ int PageState::peek_append(int block, int* page, int* sp0, std::string* why) con
   return KV_OK;
 }
 
+int PageState::begin_frame(std::string* why) {
+  if (step_open && n_appended < cfg.B) {
+    *why = "begin_frame: the open frame step has blocks still to append";
+    return KV_ERR_ORDER;
+  }
+  int page = 0, sp0 = 0;
+  const int rc = peek_append(0, &page, &sp0, why);   // the checks of a step-opening append
+  if (rc != KV_OK) return rc;
+  open_step();
+  return KV_OK;
+}
+
+void PageState::open_step() {
+  const int pg = patch_->free.back();
+  patch_->free.pop_back();
+  step_sp0 = sp_len;
+  sp_len += cfg.NS;
+  step_page = pg;
+  const FramePage fp{next_frame++, pg, step_sp0};
+  if (defer) {
+    has_pending = true;
+    pending_ = fp;
+  } else {
+    commit_frame(fp);
+  }
+  step_open = true;
+  std::fill(appended.begin(), appended.end(), 0);
+  n_appended = 0;
+  ++epoch;
+}
+
 int PageState::append(int block, int* page, int* sp0, std::string* why) {
   const int rc = peek_append(block, page, sp0, why);
   if (rc != KV_OK) return rc;
   if (!step_open || n_appended == cfg.B) {
-    const int pg = free_.back();
-    free_.pop_back();
-    step_sp0 = sp_len;
-    sp_len += cfg.NS;
-    step_page = pg;
-    const FramePage fp{next_frame++, pg, step_sp0};
-    if (defer) {
-      has_pending = true;
-      pending_ = fp;
-    } else {
-      commit_frame(fp);
-    }
-    step_open = true;
-    std::fill(appended.begin(), appended.end(), 0);
-    n_appended = 0;
-    ++epoch;
+    open_step();
   }
   appended[block] = 1;
   ++n_appended;
@@ -122,7 +155,7 @@ int PageState::evict() {
   if (defer) return KV_OK;
   bool any = false;
   while ((int)window_.size() > cfg.W) {
-    free_.push_back(window_.front().page);
+    patch_->free.push_back(window_.front().page);
     window_.pop_front();
     any = true;
   }
@@ -161,7 +194,7 @@ int PageState::rollback(std::string* why) {
     *why = "rollback: no deferred frame";
     return KV_ERR_NO_PENDING;
   }
-  free_.push_back(pending_.page);
+  patch_->free.push_back(pending_.page);
   sp_len -= cfg.NS;
   --next_frame;
   has_pending = false;
@@ -189,20 +222,59 @@ int PageState::visible_runs(std::vector<PageRun>* runs) const {
   if (committed == 0 && !has_pending) return KV_ERR_EMPTY;
   runs->clear();
   const int ps = cfg.page_size;
-  for (const auto& fp : scale_) runs->push_back({fp.page, 0, ps});
-  for (const auto& fp : window_) runs->push_back({fp.page, 0, ps});
-  if (has_pending) runs->push_back({pending_.page, 0, ps});
+  if (!camera_only) {
+    for (const auto& fp : scale_) runs->push_back({fp.page, 0, ps});
+    for (const auto& fp : window_) runs->push_back({fp.page, 0, ps});
+    if (has_pending) runs->push_back({pending_.page, 0, ps});
+  }
   int g0, g1;
   special_gap(&g0, &g1);
+  // camera-only: the frames' first tokens, stream indices 0, NS, 2 NS, ...
+  // (every frame's run starts at a multiple of NS, and so do g0 and g1)
+  const int step = camera_only && cfg.NS > 0 ? cfg.NS : 1;
   const int k = ceil_div(sp_len, ps);
   for (int i = 0; i < k; ++i) {
     const int a = i * ps, b = std::min(sp_len, a + ps);   // this page's tokens [a, b) of the stream
     // visible parts: [a, b) minus the hidden range [g0, g1)
     const bool gap = g1 > g0;
     const int pieces[2][2] = {{a, gap ? std::min(b, g0) : b}, {gap ? std::max(a, g1) : b, b}};
-    for (const auto& pc : pieces)
-      if (pc[1] > pc[0]) runs->push_back({cfg.Np + i, pc[0] - a, pc[1] - a});
+    for (const auto& pc : pieces) {
+      const int lo = ceil_div(pc[0], step) * step;   // first visible token of the piece
+      if (pc[1] > lo) runs->push_back({cfg.sp_base + i, lo - a, pc[1] - a, -1, step});
+    }
   }
+  return KV_OK;
+}
+
+int PageState::tile_runs(std::vector<PageRun>* runs) const {
+  std::vector<PageRun> all;
+  const int rc = visible_runs(&all);
+  if (rc != KV_OK) return rc;
+  runs->clear();
+  if (!step_open) {
+    *runs = all;
+    return KV_OK;
+  }
+  const int ps = cfg.page_size;
+  const int c0 = step_sp0, c1 = step_sp0 + cfg.NS;   // the frame's tokens of the special stream
+  std::vector<PageRun> cur;
+  for (const PageRun& r : all) {
+    if (r.page == step_page) {
+      cur.push_back({r.page, r.lo, r.hi, cfg.NS + r.lo, r.step});
+    } else if (r.page >= cfg.sp_base) {
+      // stream tokens [a, b) of this run, split around [c0, c1) (both ends
+      // are multiples of NS, so each piece still starts on a visible token)
+      const int a = (r.page - cfg.sp_base) * ps + r.lo, b = (r.page - cfg.sp_base) * ps + r.hi;
+      const int base = a - r.lo;
+      if (std::min(b, c0) > a) runs->push_back({r.page, r.lo, std::min(b, c0) - base, -1, r.step});
+      if (std::min(b, c1) > std::max(a, c0))
+        cur.push_back({r.page, std::max(a, c0) - base, std::min(b, c1) - base, std::max(a, c0) - c0, r.step});
+      if (b > std::max(a, c1)) runs->push_back({r.page, std::max(a, c1) - base, r.hi, -1, r.step});
+    } else {
+      runs->push_back(r);
+    }
+  }
+  runs->insert(runs->end(), cur.begin(), cur.end());
   return KV_OK;
 }
 
@@ -219,23 +291,27 @@ int PageState::page_table(std::vector<int>* idx, int* last_page_len) const {
   // unless retention off hides all of its tokens
   const int ps = cfg.page_size;
   const int last = idx->back();
-  *last_page_len = last >= cfg.Np ? std::min(ps, sp_len - ps * (last - cfg.Np)) : ps;
+  *last_page_len = last >= cfg.sp_base ? std::min(ps, sp_len - ps * (last - cfg.sp_base)) : ps;
   return KV_OK;
 }
 
 long long PageState::visible_tokens() const {
-  const long long patch = (long long)scale_.size() + (long long)window_.size() + (has_pending ? 1 : 0);
-  int g0, g1;
-  special_gap(&g0, &g1);
-  return patch * cfg.page_size + sp_len - (g1 - g0);
+  std::vector<PageRun> runs;
+  if (visible_runs(&runs) != KV_OK) return 0;
+  long long n = 0;
+  for (const PageRun& r : runs) n += ceil_div(r.hi - r.lo, r.step);
+  return n;
 }
 
 void build_tiles(const std::vector<PageRun>& runs, int page_size, std::vector<KvTile>* tiles) {
   for (const PageRun& r : runs) {
     const int base = r.page * 2 * page_size;
-    for (int s = r.lo; s < r.hi; s += kTile) {
+    // a tile covers rows [s, e) of the run; the next one starts at the run's
+    // next visible row (s advances by whole steps)
+    const int advance = ceil_div(kTile, r.step) * r.step;
+    for (int s = r.lo; s < r.hi; s += advance) {
       const int e = std::min(s + kTile, r.hi);
-      KvTile t;
+      KvTile t{};
       if (e - s == kTile) {
         t.row = base + s; t.lo = 0; t.hi = kTile;
       } else if (page_size >= kTile) {
@@ -249,6 +325,10 @@ void build_tiles(const std::vector<PageRun>& runs, int page_size, std::vector<Kv
         // a page shorter than one tile: the box runs past it, rows >= e masked
         t.row = base; t.lo = (int16_t)s; t.hi = (int16_t)e;
       }
+      // column c is pool row t.row + c and, for the current frame, k/v row
+      // krow + c
+      t.krow = r.krow >= 0 ? r.krow + (t.row - base) - r.lo : kNotCurrent;
+      t.step = (int16_t)r.step;
       tiles->push_back(t);
     }
   }
@@ -264,7 +344,8 @@ WorkspaceLayout workspace_layout(const std::vector<const PageState*>& st) {
     const Config& c = s->cfg;
     const int T = c.page_size + c.NS;
     units_base += (size_t)c.H * ceil_div(T, kTile);
-    tiles_cap += (size_t)c.max_pages * ceil_div(c.page_size, kTile) + 2;   // + the gap's split page
+    // + the retention gap's split page and the current frame's special runs
+    tiles_cap += (size_t)c.max_pages * ceil_div(c.page_size, kTile) + 8;
     D = c.D;
   }
   L.slot_cap = 2 * (units_base + kMaxTargetCtas);
@@ -274,6 +355,7 @@ WorkspaceLayout workspace_layout(const std::vector<const PageState*>& st) {
   off += align_up(units_cap * sizeof(KvUnit), 16);
   off += align_up(units_base * sizeof(KvMergeItem), 16);
   off += align_up(tiles_cap * sizeof(KvTile), 16);
+  off += align_up(units_base * 2 * sizeof(uint32_t), 16);   // split groups' counters
   L.table_bytes = align_up(off, 256);
   L.off_part_o = L.table_bytes;
   L.off_part_lse = align_up(L.off_part_o + L.slot_cap * kTile * (size_t)D * 4, 256);
@@ -301,7 +383,7 @@ int build_plan(const std::vector<const PageState*>& st, const PlanInputs& in, Ho
       return rc;
     }
     std::vector<PageRun> runs;
-    s->visible_runs(&runs);
+    s->tile_runs(&runs);
     tile0[r] = (int)P.tiles.size();
     build_tiles(runs, s->cfg.page_size, &P.tiles);
     KvReq rq;
@@ -309,6 +391,10 @@ int build_plan(const std::vector<const PageState*>& st, const PlanInputs& in, Ho
     rq.T = s->cfg.page_size + s->cfg.NS;
     rq.page_size = s->cfg.page_size;
     rq.n_tiles = (int)P.tiles.size() - tile0[r];
+    rq.cur_page = s->step_open ? s->step_page : -1;
+    rq.cur_sp0 = s->step_open ? s->step_sp0 : 0;
+    rq.sp_base = s->cfg.sp_base;
+    rq.NS = s->cfg.NS;
     q_row0 += rq.T;
     P.reqs.push_back(rq);
     P.tables.push_back(table);
@@ -329,7 +415,7 @@ int build_plan(const std::vector<const PageState*>& st, const PlanInputs& in, Ho
     const int T = P.reqs[r].T;
     int qtiles = ceil_div(T, kTile);
     const int last_rows = T - (qtiles - 1) * kTile;
-    const bool tail = in.tail_ok && qtiles >= 2 && last_rows <= kMaxTailRows;
+    const bool tail = qtiles >= 2 && last_rows <= in.max_tail_rows;
     if (tail) --qtiles;
     for (int qt = 0; qt < qtiles; qt += 2) {
       const int nq = std::min(2, qtiles - qt);
@@ -382,7 +468,7 @@ int build_plan(const std::vector<const PageState*>& st, const PlanInputs& in, Ho
     }
   }
   const WorkspaceLayout WL = workspace_layout(st);
-  int n_slots = 0;
+  int n_slots = 0, n_groups = 0;
   for (const Group& g : groups) {
     const int nt = g.n;
     const int chunks = std::max(1, ceil_div(nt, L));
@@ -403,10 +489,12 @@ int build_plan(const std::vector<const PageState*>& st, const PlanInputs& in, Ho
           ++P.n_split_units;
         }
       }
+      const int group = chunks > 1 ? n_groups++ : -1;
       for (int k = 0; k < chunks; ++k) {
         KvUnit u{};
         u.req = (int16_t)g.req; u.head = (int16_t)h; u.qtile = (int16_t)g.qt; u.nq = (int16_t)g.nq;
         u.tail_rows = (int16_t)g.tail;
+        u.chunk = (int16_t)k; u.n_chunks = (int16_t)chunks; u.group = group;
         u.tile_begin = tile0[g.req] + (int)((long long)k * nt / chunks);
         u.tile_end = tile0[g.req] + (int)((long long)(k + 1) * nt / chunks);
         for (int t = 0; t < 3; ++t) u.slot[t] = (chunks > 1 && t < ntiles_q) ? slot0[t] + k : -1;
@@ -444,6 +532,11 @@ int build_plan(const std::vector<const PageState*>& st, const PlanInputs& in, Ho
   Hd.off_units = (int)off;  off += align_up(P.units.size() * sizeof(KvUnit), 16);
   Hd.off_merge = (int)off;  off += align_up(P.merges.size() * sizeof(KvMergeItem), 16);
   Hd.off_tiles = (int)off;  off += align_up(P.tiles.size() * sizeof(KvTile), 16);
+  Hd.off_groups = (int)off; off += align_up((size_t)n_groups * 2 * sizeof(uint32_t), 16);
+  Hd.n_groups = n_groups;
+  // The CTAs of a split group wait for one another before merging it, which
+  // needs every CTA of the launch resident at once: one CTA per SM slot.
+  Hd.fused_merge = (n_groups > 0 && (int)P.units.size() <= target) ? 1 : 0;
   Hd.upload_bytes = (int)off;
   Hd.off_part_o = (int64_t)WL.off_part_o;
   Hd.off_part_lse = (int64_t)WL.off_part_lse;

@@ -26,6 +26,7 @@
 #pragma once
 #include <cstdint>
 #include <deque>
+#include <memory>
 #include <string>
 #include <vector>
 
@@ -40,19 +41,33 @@ struct FramePage {
 };
 
 // A visible range [lo, hi) of rows of one pool page.
+// Visible rows lo, lo + step, ... < hi of one pool page (step > 1: the
+// camera tokens of a camera-only cache, lo being one of them).
 struct PageRun {
   int page;
   int lo, hi;
+  int krow = -1;   // rows of the current frame: k/v row of row lo (>= 0), else -1
+  int step = 1;
 };
 
 struct Config {
   int max_pages, page_size, H, D, S, W, B, NS, dtype, Np;
+  int sp_base = 0;    // this stream's special pages [sp_base, sp_base + sp_pages)
+  int sp_pages = 0;   // (0, 0 at init: every page after the patch pages)
+};
+
+// Patch pages [0, Np) and their LIFO free list (back() is handed out next).
+// A stream alone in its pool owns one; the streams of a group share one.
+struct PatchPool {
+  std::vector<int> free;
+  int Np = 0;
+  bool shared = false;
 };
 
 class PageState {
  public:
   Config cfg{};
-  std::vector<int> free_;        // back() is the next page handed out
+  std::shared_ptr<PatchPool> patch_;   // patch pages and their free list
   std::vector<FramePage> scale_;
   std::deque<FramePage> window_;
   bool has_pending = false;
@@ -62,6 +77,7 @@ class PageState {
   int next_frame = 0;
   bool defer = false;
   bool cross_special = true;   // special tokens of evicted frames stay visible
+  bool camera_only = false;    // attention sees only the camera tokens (slot 0 of each frame's NS)
   // frame step
   bool step_open = false;
   std::vector<uint8_t> appended;
@@ -71,8 +87,13 @@ class PageState {
   uint64_t epoch = 1;   // bumped on every change of the visible table
 
   // Returns KV_OK or a KV_ERR_* code; `why` gets a one-line detail on error.
-  int init(const Config& c, std::string* why);
+  // `pool`: a patch pool shared with other streams (NULL: a pool of its own).
+  int init(const Config& c, std::string* why, std::shared_ptr<PatchPool> pool = nullptr);
+  // Back to the initial state. In a shared pool this stream's patch pages go
+  // back to the common free list: scale pages (frame order), then window
+  // pages (oldest first), then a pending page.
   void reset();
+  const std::vector<int>& free_list() const { return patch_->free; }
   // Marks `block` appended in the current step, opening a new step (and
   // taking a patch page and NS special slots) when needed.
   int append(int block, int* page, int* sp0, std::string* why);
@@ -90,7 +111,14 @@ class PageState {
   void special_gap(int* g0, int* g1) const;
   // The visible rows, page by page, in page-table order.
   int visible_runs(std::vector<PageRun>* runs) const;
-  int special_capacity() const { return (cfg.max_pages - cfg.Np) * cfg.page_size; }
+  // The visible rows as the K/V tiles cover them: visible_runs with the rows
+  // of the open step's frame (its patch page and its NS special tokens, those
+  // that are visible) taken out and appended at the end with their k/v rows.
+  int tile_runs(std::vector<PageRun>* runs) const;
+  // Opens a frame step without appending a block (takes the frame's patch
+  // page and NS special slots); the blocks are appended afterwards.
+  int begin_frame(std::string* why);
+  int special_capacity() const { return cfg.sp_pages * cfg.page_size; }
   bool is_appended(int block) const {
     return step_open && block >= 0 && block < cfg.B && appended[block];
   }
@@ -98,13 +126,14 @@ class PageState {
 
  private:
   void commit_frame(const FramePage& fp);
+  void open_step();   // the step-opening part of append (checks done by the caller)
 };
 
 struct PlanInputs {
   int num_sms;           // SMs of the device
   int ctas_per_sm;       // attention CTAs resident per SM
   int tiles_per_split;   // > 0: forced chunk size (tests); 0: automatic
-  bool tail_ok;          // the attention kernel computes <= 16-row tail tiles in-unit
+  int max_tail_rows;     // the attention kernel computes tail tiles of up to this many rows in-unit
 };
 
 struct HostPlan {

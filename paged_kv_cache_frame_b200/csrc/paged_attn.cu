@@ -11,26 +11,24 @@
 // Enables Long Sequence Inference in LingBot-Map", [P3] "FlashInfer Paged KV
 // Cache Performance Benefits in LingBot-Map".)
 //
-// Roles. head_dim 64: 12 warps (384 threads); head_dim 128: 10 warps (320).
+// Roles. 12 warps (384 threads).
 //   warps 0-3, 4-7   softmax warpgroups, one per 128-row query tile. Thread i
 //                    owns query row i == TMEM lane i. Per K/V tile it reads its
 //                    S row in two 64-column halves, keeps the running max/sum
-//                    in the log2 domain, writes P (16-bit) to TMEM -- the first
-//                    half as soon as the previous PV has read P, so its store
-//                    overlaps the second half -- and rescales its O row when
-//                    the running max grows by more than 2^8 (lazy rescale:
-//                    between rescales P may exceed 1, which the final division
-//                    by the same sum cancels).
-//   producer         warp 9 (head_dim 64) / 8 (head_dim 128): TMA loads, the
+//                    in the log2 domain, writes P (16-bit) over the S columns
+//                    it has read, and rescales its O row when the running max
+//                    grows by more than 2^8 (lazy rescale: between rescales P
+//                    may exceed 1, which the final division by the same sum
+//                    cancels).
+//   producer         warp 9: TMA loads, the
 //                    query tiles once, then K/V tiles of the page table into a
 //                    STAGES-deep ring. A tile is 128 pool rows of one head, one
 //                    3-D box load per 64 columns; the tile table gives each
 //                    tile's row, so pages need not be contiguous.
-//   MMA issuer       warp 11 / 9, also the TMEM allocator (tcgen05 kind::f16,
-//                    fp32 accumulators in TMEM): S_t = Q_t K^T (M=128, N=128,
-//                    K=D) and O_t += P_t V (M=128, N=D, K=128, P read from
-//                    TMEM). Each query tile advances on its own, scores first.
-//   tail             warps 8 and 10 (head_dim 64): the unit's last query tile
+//   MMA issuer       warp 11, also the TMEM allocator (tcgen05 kind::f16,
+//                    fp32 accumulators in TMEM): S = Q_t K^T (M=128, N=128,
+//                    K=D) and O_t += P V (M=128, N=D, K=128, P read from TMEM).
+//   tail             warps 8 and 10: the unit's last query tile
 //                    of at most 16 rows (262 = 2 x 128 + 6 tokens per frame).
 //                    An M = 128 tensor-core tile would be almost all padding,
 //                    so each of these warps computes the tail's scores and
@@ -39,11 +37,22 @@
 //                    the N = 8 side, reading K and V straight from the
 //                    shared-memory ring, with its own running max/sum and O in
 //                    registers. The two partial results are merged at the end.
-// TMEM. head_dim 64: S_t at [128 t, +128), P_t at [256 + 64 t, +64), O_t at
-// [384 + 64 t, +64). P has its own columns, so the tensor core computes
-// S_t(j+1) as soon as the softmax has read S_t(j), while the exponentials of
-// tile j run. head_dim 128: O_t takes [256 + 128 t, +128), so P_t is written
-// over the S_t columns it came from and S_t(j+1) follows PV_t(j).
+//
+// Schedule. Score tiles are numbered n = j * nq + t (K/V tile j, query tile t
+// of nq). S_n goes to TMEM buffer n % NB and its P is written over it. NB is 3
+// for head_dim 64 with two query tiles (3 x 128 columns and two 64-column O
+// tiles fill the 512 columns), else 2. The tensor pipe executes a CTA's MMAs
+// in issue order, so S_n may be issued as soon as PV_{n-NB}, the last reader
+// of its buffer, has been issued: the scores of the next tiles are computed
+// while the softmax works on the current one, and the softmax never waits for
+// a PV before it stores P. Both kinds of MMA are issued in order of n, which
+// gives the two facts the waits below rely on:
+//   - once S_n has completed, every PV_m with m <= n - NB has completed; as
+//     NB <= 2 nq, the O rescale at K/V tile j (after S_t(j) was read) waits
+//     only for PV_t(j-1), because PV_t(j-2) is complete already;
+//   - no barrier runs more than one phase ahead of a waiter (each waiter's
+//     previous wait covered the phase before), so every parity wait is
+//     unambiguous. Per-buffer s_full / p_full barriers carry the phases.
 // The launch overlaps the previous kernel on the stream (programmatic
 // dependent launch): everything before pdl_wait() is setup that touches no
 // data an earlier kernel may still be writing.
@@ -55,43 +64,25 @@
 
 #include "kernels.h"
 #include "launch.cuh"
+#include "merge.cuh"
 #include "sm100.cuh"
 
 namespace pkv {
 
 constexpr int kMaxSmemTiles = 512;   // tile descriptors cached in shared memory
 
-#ifdef PKV_TRACE
-// Instrumented builds only: per-tile clock64() stamps of each role of CTA 0,
-// read back with kv_debug_trace(). Layout [role 0..5][tile < 64][event < 8].
-__device__ unsigned long long g_pkv_trace[6][64][8];
-// per CTA: globaltimer at entry, after the prologue, at exit; and its SM
-__device__ unsigned long long g_pkv_cta[1024][6];
-#define PKV_TRACE_AT(role, j, ev) \
-  do { if (blockIdx.x == 0 && (j) < 64) g_pkv_trace[role][j][ev] = clock64(); } while (0)
-#define PKV_CTA_AT(ev) \
-  do { if (threadIdx.x == 0 && blockIdx.x < 1024) { \
-         g_pkv_cta[blockIdx.x][ev] = globaltimer_ns(); \
-         if ((ev) != 1) g_pkv_cta[blockIdx.x][4 + (ev) / 2] = clock64(); } } while (0)
-#else
-#define PKV_TRACE_AT(role, j, ev) do { } while (0)
-#define PKV_CTA_AT(ev) do { } while (0)
-#endif
-
 template <int D>
 struct AttnRoles {
-  static constexpr bool kTail = D == 64;
-  // head_dim 64: warps 8 and 10 are the tail (with the softmax warpgroups,
-  // three warps per SM sub-partition), 9 the producer, 11 the MMA issuer
+  // warps 8 and 10 are the tail (with the softmax warpgroups, three warps
+  // per SM sub-partition), 9 the producer, 11 the MMA issuer
   static constexpr int kTailWarps = 2;   // each takes 64 of a K/V tile's 128 columns
-  static constexpr int kProducer = kTail ? 9 : 8, kMma = kTail ? 11 : 9;
-  static constexpr int kWarps = kTail ? 12 : 10;
+  static constexpr int kProducer = 9, kMma = 11;
+  static constexpr int kWarps = 12;
   static constexpr int kThreads = 32 * kWarps;
 };
 
 template <int D, int STAGES>
 struct AttnSmem {
-  static constexpr bool kTail = AttnRoles<D>::kTail;
   static constexpr int kTileBytes = kTile * D * 2;   // one 128-row Q, K or V tile
   static constexpr int kQ = 0;                       // two query tiles
   static constexpr int kK = 2 * kTileBytes;
@@ -99,20 +90,20 @@ struct AttnSmem {
   // tail merge: per tail warp [16 rows][D] fp32 outputs, then maxima and sums
   static constexpr int kTW = AttnRoles<D>::kTailWarps;
   static constexpr int kTailO = kV + STAGES * kTileBytes;
-  static constexpr int kTailML = kTailO + (kTail ? kTW * 16 * D * 4 : 0);
-  static constexpr int kTiles = kTailML + (kTail ? 2 * kTW * 16 * 4 : 0);
-  static constexpr int kBars = kTiles + kMaxSmemTiles * 8;
+  static constexpr int kTailML = kTailO + kTW * 16 * D * 4;
+  static constexpr int kTiles = kTailML + 2 * kTW * 16 * 4;
+  static constexpr int kBars = kTiles + kMaxSmemTiles * (int)sizeof(KvTile);
   static constexpr int kBytes = kBars + 256;
   static constexpr int kAlloc = kBytes + 1024;      // slack to align the base to 1 KB
 };
 
+// TMEM columns: the S/P buffers (128 columns each) from column 0, then O_0, O_1.
 template <int D>
 struct AttnTmem {
-  static constexpr bool kSepP = D == 64;             // P in its own columns
-  __host__ __device__ static constexpr uint32_t S(int t) { return 128u * t; }
-  __host__ __device__ static constexpr uint32_t P(int t) { return kSepP ? 256u + 64u * t : 128u * t; }
-  __host__ __device__ static constexpr uint32_t O(int t) { return (kSepP ? 384u : 256u) + (uint32_t)D * t; }
-  static_assert((kSepP ? 384 : 256) + 2 * D <= 512, "TMEM budget");
+  static constexpr int kMaxBufs = D == 64 ? 3 : 2;
+  __host__ __device__ static constexpr uint32_t buf(int b) { return 128u * b; }
+  __host__ __device__ static constexpr uint32_t O(int t) { return 128u * kMaxBufs + (uint32_t)D * t; }
+  static_assert(128 * kMaxBufs + 2 * D <= 512, "TMEM budget");
 };
 
 constexpr uint32_t kTmemCols = 512;
@@ -124,6 +115,22 @@ __device__ __forceinline__ void mbar_drain_wait(uint64_t* bar, uint32_t parity) 
   while (!mbar_try_wait(bar, parity)) {
     if (globaltimer_ns() - t0 > kWaitLimitNs) return;
   }
+}
+
+// Visible columns [base, base + 64) of a K/V tile as a bit mask (bit c for
+// column base + c): [lo, hi), and with step > 1 only lo, lo + step, ...
+__device__ __forceinline__ uint64_t visible_cols(const KvTile& t, int base) {
+  const int lo = max(t.lo - base, 0), hi = min(t.hi - base, 64);
+  if (hi <= lo) return 0;
+  uint64_t m = (hi == 64 ? ~0ull : (1ull << hi) - 1) & ~((1ull << lo) - 1);
+  if (t.step > 1) {
+    int c = t.lo - base;
+    if (c < 0) c += (-c + t.step - 1) / t.step * t.step;   // first visible column of this half
+    uint64_t s = 0;
+    for (; c < 64; c += t.step) s |= 1ull << c;
+    m &= s;
+  }
+  return m;
 }
 
 template <bool kFP16>
@@ -151,10 +158,9 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
   using R = AttnRoles<D>;
   using L = AttnSmem<D, STAGES>;
   using TM = AttnTmem<D>;
-  constexpr bool kSepP = TM::kSepP;
-  constexpr bool kTail = R::kTail;
   constexpr int kThreads = R::kThreads;
   static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+  static_assert(L::kAlloc <= 227 * 1024, "shared memory per CTA");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
 
@@ -162,31 +168,32 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
   uint64_t* bar_q = bars;
   uint64_t* bar_kv_full = bars + 1;
   uint64_t* bar_kv_empty = bars + 1 + STAGES;
-  uint64_t* bar_s_full = bars + 1 + 2 * STAGES;   // [2] S_t(j) computed
-  uint64_t* bar_s_free = bar_s_full + 2;          // [2] S_t(j) read by its softmax
-  uint64_t* bar_p_full = bar_s_full + 4;          // [2] P_t(j) written (and O_t rescaled)
+  uint64_t* bar_s_full = bars + 1 + 2 * STAGES;   // [3] S_n computed into buffer n % NB
+  uint64_t* bar_p_full = bar_s_full + 3;          // [3] P_n written over it (and O_t rescaled)
   uint64_t* bar_pv_done = bar_s_full + 6;         // [2] PV_t(j) complete
   uint64_t* bar_o_final = bar_s_full + 8;
   uint64_t* bar_drain = bar_s_full + 9;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_s_full + 10);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* merge_ok = reinterpret_cast<volatile int*>(tmem_slot + 2);
   KvTile* tile_cache = reinterpret_cast<KvTile*>(smem + L::kTiles);
 
-  PKV_CTA_AT(0);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const KvUnit u = a.units[blockIdx.x];
   const KvReq rq = a.reqs[u.req];
   const int n_tiles = u.tile_end - u.tile_begin;
   const int nq = u.nq;
-  const int tail_rows = kTail ? u.tail_rows : 0;
+  const int tail_rows = u.tail_rows;
   const bool has_tail = tail_rows > 0;
   const KvTile* tiles_g = a.tiles + u.tile_begin;
-  if (n_tiles <= 0 || nq < 1 || nq > 2 || u.tail_rows < 0 || u.tail_rows > kMaxTailRows ||
-      (!kTail && u.tail_rows != 0)) {   // the planner never emits such a unit
+  if (n_tiles <= 0 || nq < 1 || nq > 2 || u.tail_rows < 0 || u.tail_rows > (D == 64 ? kMaxTailRows : 8)) {
+    // the planner never emits such a unit
     if (threadIdx.x == 0) atomicOr(a.err, 2u);
     return;
   }
+  // S/P buffers in rotation: 3 where two query tiles leave room for them
+  const int nb = (TM::kMaxBufs == 3 && nq == 2) ? 3 : 2;
 
   // Tile descriptors into shared memory (off the softmax's critical path).
   for (int i = threadIdx.x; i < min(n_tiles, kMaxSmemTiles); i += kThreads) tile_cache[i] = tiles_g[i];
@@ -199,12 +206,11 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
       // released by the MMA issuer's commit and, with a tail, by each tail warp
       mbar_init(&bar_kv_empty[s], 1 + (has_tail ? R::kTailWarps : 0));
     }
-    for (int t = 0; t < 2; ++t) {
-      mbar_init(&bar_s_full[t], 1);
-      mbar_init(&bar_s_free[t], 128);
-      mbar_init(&bar_p_full[t], 128);
-      mbar_init(&bar_pv_done[t], 1);
+    for (int b = 0; b < 3; ++b) {
+      mbar_init(&bar_s_full[b], 1);
+      mbar_init(&bar_p_full[b], 128);
     }
+    for (int t = 0; t < 2; ++t) mbar_init(&bar_pv_done[t], 1);
     mbar_init(bar_o_final, 1);
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
@@ -218,37 +224,95 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+
+  // The producer's K/V loads, one K/V tile j into ring stage j % STAGES.
+  const CUtensorMap* mkv = &maps.kv[u.req];
+  auto load_kv = [&](int j) {
+    const int s = j % STAGES;
+    const KvTile t = tile_at(j);
+    // the frame's own tiles from k, v when this launch appends it
+    const bool own = a.fused_append && t.krow != kNotCurrent;
+    const CUtensorMap* mk = own ? &maps.k : mkv;
+    const CUtensorMap* mv = own ? &maps.v : mkv;
+    const int rk = own ? rq.q_row0 + t.krow : t.row;
+    const int rv = own ? rk : t.row + rq.page_size;
+    mbar_arrive_expect_tx(&bar_kv_full[s], 2 * L::kTileBytes);
+#pragma unroll
+    for (int kb = 0; kb < D / 64; ++kb) {
+      tma_load_3d(smem + L::kK + s * L::kTileBytes + kb * 16384, mk, &bar_kv_full[s], kb * 64, u.head, rk);
+      tma_load_3d(smem + L::kV + s * L::kTileBytes + kb * 16384, mv, &bar_kv_full[s], kb * 64, u.head, rv);
+    }
+  };
+  int j_loaded = 0;   // K/V tiles whose loads the producer has issued
+  if (warp == R::kProducer && lane == 0) {
+    prefetch_tmap(&maps.q);
+    prefetch_tmap(mkv);
+    if (a.fused_append) {
+      prefetch_tmap(&maps.k);
+      prefetch_tmap(&maps.v);
+    }
+    // Earlier frames' pool rows may be read before the previous kernel on
+    // the stream has completed: that kernel is the previous block's launch,
+    // its append or the plan upload, and none of them writes those rows (a
+    // block's pool is written only by its own appends, stream-ordered long
+    // before). The first ring stages are filled with them now; the frame's
+    // own tiles, and q, wait.
+    for (; j_loaded < min(n_tiles, STAGES) && tile_at(j_loaded).krow == kNotCurrent; ++j_loaded)
+      load_kv(j_loaded);
+  }
   // The setup above overlaps the previous kernel (the frame's K/V append);
-  // the pool and q are read only after it has completed.
+  // q, k, v and the frame's own rows are read only after it has completed.
   pdl_wait();
-  PKV_CTA_AT(1);
+
+  if (a.fused_append && warp < 8) {
+    // ------------------------------------------------- append (scatter)
+    // This CTA's slice of every request's k, v rows, copied into the pool in
+    // 16-byte vectors ([P1] "Appending New Frames": special tokens 0..NS-1 to
+    // the special stream at the frame's offset, which may straddle two
+    // pages; patch tokens to the frame's page). No CTA of this launch reads
+    // those pool rows: the frame's own tiles come from k, v. The softmax
+    // warps do it while the first scores are computed.
+    const int T = rq.T, rv = a.row_vecs;
+    const long long per_kv = (long long)T * rv, per_req = 2 * per_kv;
+    const long long total = per_req * a.n_reqs;
+    const long long i0 = total * blockIdx.x / gridDim.x, i1 = total * (blockIdx.x + 1) / gridDim.x;
+    for (long long i = i0 + threadIdx.x; i < i1; i += 256) {
+      const int r = (int)(i / per_req);
+      const long long rem = i - (long long)r * per_req;
+      const int kv = rem >= per_kv;
+      const long long rr = rem - kv * per_kv;
+      const int tok = (int)(rr / rv);
+      const int c = (int)(rr - (long long)tok * rv);
+      const KvReq q = a.reqs[r];
+      int page, slot;
+      if (tok < q.NS) {
+        const int jj = q.cur_sp0 + tok;
+        page = q.sp_base + jj / q.page_size;
+        slot = jj % q.page_size;
+      } else {
+        page = q.cur_page;
+        slot = tok - q.NS;
+      }
+      const uint4* src = static_cast<const uint4*>(kv ? a.v : a.k) + (long long)(q.q_row0 + tok) * rv + c;
+      uint4* dst = static_cast<uint4*>(a.pools[r]) + (((long long)page * 2 + kv) * q.page_size + slot) * rv + c;
+      *dst = __ldg(src);
+    }
+  }
 
   if (warp == R::kProducer) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      const CUtensorMap* mkv = &maps.kv[u.req];
-      prefetch_tmap(&maps.q);
-      prefetch_tmap(mkv);
       mbar_arrive_expect_tx(bar_q, nq * L::kTileBytes);
       for (int t = 0; t < nq; ++t)
 #pragma unroll
         for (int kb = 0; kb < D / 64; ++kb)
           tma_load_3d(smem + L::kQ + t * L::kTileBytes + kb * 16384, &maps.q, bar_q, kb * 64, u.head,
                       rq.q_row0 + (u.qtile + t) * kTile);
-      int j = 0;
+      int j = j_loaded;
       for (; j < n_tiles; ++j) {
         const int s = j % STAGES;
         if (j >= STAGES && !mbar_wait(&bar_kv_empty[s], ((j / STAGES) - 1) & 1, abort_flag)) break;
-        PKV_TRACE_AT(5, j, 0);
-        const KvTile t = tile_at(j);
-        mbar_arrive_expect_tx(&bar_kv_full[s], 2 * L::kTileBytes);
-#pragma unroll
-        for (int kb = 0; kb < D / 64; ++kb) {
-          tma_load_3d(smem + L::kK + s * L::kTileBytes + kb * 16384, mkv, &bar_kv_full[s], kb * 64, u.head,
-                      t.row);
-          tma_load_3d(smem + L::kV + s * L::kTileBytes + kb * 16384, mkv, &bar_kv_full[s], kb * 64, u.head,
-                      t.row + rq.page_size);
-        }
+        load_kv(j);
       }
       // no TMA write may still be in flight when the CTA exits
       mbar_drain_wait(bar_q, 0);
@@ -267,111 +331,73 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
       const uint64_t dQ = sdesc_sw128(smem_u32(smem + L::kQ), 16, 1024);
       const uint64_t dK = sdesc_sw128(smem_u32(smem + L::kK), 16, 1024);
       const uint64_t dV = sdesc_sw128(smem_u32(smem + L::kV), 16384, 1024);
-      int kv_ready = -1;   // highest K/V tile whose load was waited for
-      auto wait_kv = [&](int j) -> bool {
-        if (j <= kv_ready) return true;
-        if (!mbar_wait(&bar_kv_full[j % STAGES], (j / STAGES) & 1, abort_flag)) return false;
-        tc_fence_after();
-        kv_ready = j;
-        return true;
-      };
       // K-major k-step kk (16 elements): +32 bytes inside a 64-column box,
       // +16 KB to the next box
       auto kofs = [](int kk) -> uint64_t { return (uint64_t)((kk >> 2) * 1024 + (kk & 3) * 2); };
-      auto issue_s = [&](int t, int j) {   // S_t = Q_t K_j^T
+      auto issue_s = [&](int t, int j, int b) {   // S_n = Q_t K_j^T into buffer b
         const uint64_t k = dK + (j % STAGES) * kStage;
         const uint64_t q = dQ + t * kStage;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          umma_f16_ss(tmem + TM::S(t), q + kofs(kk), k + kofs(kk), idS, kk > 0);
-        umma_commit(&bar_s_full[t]);
+          umma_f16_ss(tmem + TM::buf(b), q + kofs(kk), k + kofs(kk), idS, kk > 0);
+        umma_commit(&bar_s_full[b]);
       };
-      auto issue_pv = [&](int t, int j) {   // O_t += P_t V_j, P_t from TMEM
+      auto issue_pv = [&](int t, int j, int b) {   // O_t += P_n V_j, P_n in buffer b
         const uint64_t v = dV + (j % STAGES) * kStage;
-        umma_f16_ts(tmem + TM::O(t), tmem + TM::P(t), v, idO, j > 0 ? 1u : 0u);
+        umma_f16_ts(tmem + TM::O(t), tmem + TM::buf(b), v, idO, j > 0 ? 1u : 0u);
 #pragma unroll
         for (int kk = 1; kk < kTile / 16; ++kk)
-          umma_f16_ts(tmem + TM::O(t), tmem + TM::P(t) + kk * 8, v + kk * 128, idO, 1u);
-        if (kSepP) umma_commit(&bar_pv_done[t]);
+          umma_f16_ts(tmem + TM::O(t), tmem + TM::buf(b) + kk * 8, v + kk * 128, idO, 1u);
+        umma_commit(&bar_pv_done[t]);
       };
-      bool ok = mbar_wait(bar_q, 0, abort_flag) && wait_kv(0);
-      if (ok)
-        for (int t = 0; t < nq; ++t) issue_s(t, 0);
-      if (kSepP) {
-        // Each query tile advances on its own: S_t(j) once softmax t has read
-        // S_t(j-1) and K(j) has landed, PV_t(j) once P_t(j) is written. The
-        // scores come first (the softmax waits on them); a K/V stage is
-        // released once every MMA that reads it has been issued. Non-blocking
-        // polls under one bounded wait.
-        int ns[2] = {1, 1};   // next S_t to issue
-        int np[2] = {0, 0};   // next PV_t to issue
-        if (nq < 2) ns[1] = np[1] = n_tiles;
-        int ne = 0;           // next K/V stage release
-        uint64_t t0 = globaltimer_ns();
-        for (uint32_t spin = 1; ok && ne < n_tiles; ++spin) {
-          bool progress = false;
-#pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            const int j = ns[t];
-            if (j < n_tiles && mbar_test_wait(&bar_s_free[t], (j - 1) & 1)) {
-              if (j > kv_ready) {
-                if (!mbar_test_wait(&bar_kv_full[j % STAGES], (j / STAGES) & 1)) continue;
-                kv_ready = j;
-              }
-              PKV_TRACE_AT(4, j - 1, 1 + t);
-              tc_fence_after();
-              issue_s(t, j);
-              ns[t] = j + 1;
-              progress = true;
-            }
+      // S_n once PV_{n-NB} has been issued and K/V tile j has landed; PV_n
+      // once P_n is written; both in order of n. A K/V stage is released once
+      // every MMA that reads it has been issued (the commit arrives when they
+      // complete). Non-blocking polls under one bounded wait; the scores go
+      // first, since the softmax waits on them.
+      const int n_all = n_tiles * nq;
+      int ns = 0, np = 0, ne = 0;   // next S, next PV, next K/V stage release
+      int kv_ready = -1;            // highest K/V tile whose load was observed
+      bool ok = mbar_wait(bar_q, 0, abort_flag);
+      uint64_t t0 = globaltimer_ns();
+      for (uint32_t spin = 1; ok && ne < n_tiles; ++spin) {
+        bool progress = false;
+        if (ns < n_all && ns - nb < np) {
+          const int j = ns / nq;
+          bool ready = j <= kv_ready;
+          if (!ready && mbar_test_wait(&bar_kv_full[j % STAGES], (j / STAGES) & 1)) {
+            kv_ready = j;
+            ready = true;
           }
-#pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            const int j = np[t];
-            if (j < n_tiles && mbar_test_wait(&bar_p_full[t], j & 1)) {
-              PKV_TRACE_AT(4, j, 4 + t);
-              tc_fence_after();
-              issue_pv(t, j);
-              np[t] = j + 1;
-              progress = true;
-            }
-          }
-          while (ne < min(np[0], np[1])) {   // PV_t(ne) issued for every t (and so S_t(ne))
-            umma_commit(&bar_kv_empty[ne % STAGES]);
-            PKV_TRACE_AT(4, ne, 7);
-            ++ne;
+          if (ready) {
+            tc_fence_after();
+            issue_s(ns - j * nq, j, ns % nb);
+            ++ns;
             progress = true;
           }
-          if (progress) {
-            t0 = globaltimer_ns();
-          } else {
-            // back off: this warp shares its SM sub-partition with two
-            // softmax warps, whose issue slots a tight poll would take
-            __nanosleep(32);
-            if ((spin & 15u) == 0 && (*abort_flag || globaltimer_ns() - t0 > kWaitLimitNs)) {
-              *abort_flag = 1;
-              ok = false;
-            }
-          }
         }
-      } else {
-        for (int j = 0; ok && j < n_tiles; ++j) {
-          const bool more = j + 1 < n_tiles;
-          PKV_TRACE_AT(4, j, 0);
-          // P_t(j) sits in the S_t columns: S_t(j+1) follows PV_t(j)
-          for (int t = 0; t < nq; ++t) {
-            if (!mbar_wait(&bar_p_full[t], j & 1, abort_flag)) { ok = false; break; }
-            PKV_TRACE_AT(4, j, 4 + t);
-            tc_fence_after();
-            issue_pv(t, j);
-            if (more) {
-              if (!wait_kv(j + 1)) { ok = false; break; }
-              issue_s(t, j + 1);
-            }
+        if (np < ns && mbar_test_wait(&bar_p_full[np % nb], (np / nb) & 1)) {
+          const int j = np / nq;
+          tc_fence_after();
+          issue_pv(np - j * nq, j, np % nb);
+          ++np;
+          progress = true;
+        }
+        while (ne < n_tiles && np >= (ne + 1) * nq) {   // every PV of K/V tile ne issued
+          umma_commit(&bar_kv_empty[ne % STAGES]);
+          ++ne;
+          progress = true;
+        }
+        if (progress) {
+          t0 = globaltimer_ns();
+        } else {
+          // back off: this warp shares its SM sub-partition with two
+          // softmax warps, whose issue slots a tight poll would take
+          __nanosleep(32);
+          if ((spin & 15u) == 0 && (*abort_flag || globaltimer_ns() - t0 > kWaitLimitNs)) {
+            *abort_flag = 1;
+            ok = false;
           }
-          if (!ok) break;
-          umma_commit(&bar_kv_empty[j % STAGES]);
-          PKV_TRACE_AT(4, j, 7);
         }
       }
       umma_commit(bar_o_final);
@@ -389,8 +415,6 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
       const int rows_valid = min(kTile, rq.T - (u.qtile + t) * kTile);
       const bool active = sub * 32 < rows_valid;   // warp-uniform
       const uint32_t lane_base = static_cast<uint32_t>(sub * 32) << 16;
-      const uint32_t tS = tmem + TM::S(t) + lane_base;
-      const uint32_t tP = tmem + TM::P(t) + lane_base;
       const uint32_t tO = tmem + TM::O(t) + lane_base;
       const float sl2 = a.scale_log2;
       const uint64_t sl2x2 = f2_pack(sl2, sl2);
@@ -398,152 +422,146 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
       float l_run = 0.f;         // running sum of 2^(s * sl2 - m_run)
       bool ok = true;
       for (int j = 0; j < n_tiles; ++j) {
-        // every wait is made warp-uniform: tcgen05.ld/st are .sync.aligned
-        if (!__all_sync(0xffffffffu, mbar_wait(&bar_s_full[t], j & 1, abort_flag))) { ok = false; break; }
-        if (row == 0) PKV_TRACE_AT(t, j, 0);
+        const int n = j * nq + t;
+        const int b = n % nb;
+        // Every warp waits, rows or not: p_full counts 128 arrivals a phase.
+        // The waits are warp-uniform: tcgen05.ld/st are .sync.aligned.
+        if (!__all_sync(0xffffffffu, mbar_wait(&bar_s_full[b], (n / nb) & 1, abort_flag))) { ok = false; break; }
         tc_fence_after();
-        const KvTile tl = tile_at(j);
-        const bool masked = tl.lo > 0 || tl.hi < kTile;
-        float alpha = 1.f;
-        bool need = false;
-        uint32_t pa[32], pb[32];   // this row of P_t(j): columns 0-63, 64-127 as 16-bit pairs
-        uint64_t acc[4] = {0, 0, 0, 0};
-        auto load_half = [&](int h, uint32_t (&r)[64]) {
-          tmem_ld_x64_wait(tS + 64 * h, r);
-          if (masked) {
+        if (active) {
+          const uint32_t tS = tmem + TM::buf(b) + lane_base;
+          const KvTile tl = tile_at(j);
+          const bool masked = tl.lo > 0 || tl.hi < kTile || tl.step > 1;
+          float alpha = 1.f;
+          bool need = false;
+          uint64_t acc[4] = {0, 0, 0, 0};
+          auto load_half = [&](int h, uint32_t (&r)[64]) {
+            tmem_ld_x64_wait(tS + 64 * h, r);
+            if (masked) {
+              const uint64_t vis = visible_cols(tl, 64 * h);
 #pragma unroll
-            for (int c = 0; c < 64; ++c)
-              if (64 * h + c < tl.lo || 64 * h + c >= tl.hi) r[c] = 0xFF800000u;   // -inf
-          }
-        };
-        auto half_max = [&](const uint32_t (&r)[64]) -> float {
-          float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
-#pragma unroll
-          for (int c = 0; c < 64; c += 8) {
-            mx0 = fmax3(mx0, __uint_as_float(r[c + 0]), __uint_as_float(r[c + 1]));
-            mx1 = fmax3(mx1, __uint_as_float(r[c + 2]), __uint_as_float(r[c + 3]));
-            mx2 = fmax3(mx2, __uint_as_float(r[c + 4]), __uint_as_float(r[c + 5]));
-            mx3 = fmax3(mx3, __uint_as_float(r[c + 6]), __uint_as_float(r[c + 7]));
-          }
-          return fmax3(mx0, mx1, fmaxf(mx2, mx3)) * sl2;
-        };
-        // P = 2^(s * sl2 - m_run) in 16-bit pairs into pk, summed
-        // in fp32 into acc. A half can be fully masked (a short last tile of a
-        // page), so the first half may leave m_run at -inf.
-        auto exp_half = [&](const uint32_t (&sv)[64], uint32_t (&pk)[32]) {
-          // m_run is -inf only while every column so far was masked: P is 0
-          const float mu = m_run == -INFINITY ? 0.f : m_run;
-          const uint64_t negm2 = f2_pack(-mu, -mu);
-#pragma unroll
-          for (int c = 0; c < 64; c += 2) {
-            const uint64_t x = f2_fma(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sl2x2, negm2);
-            uint64_t e;
-            if ((kEmuMask >> ((c >> 1) & 7)) & 1u) {
-              e = exp2_poly2(x);
-            } else {
-              float x0, x1;
-              f2_unpack(x, x0, x1);
-              e = f2_pack(ex2_approx(x0), ex2_approx(x1));
+              for (int c = 0; c < 64; ++c)
+                if (!((vis >> c) & 1)) r[c] = 0xFF800000u;   // -inf
             }
-            acc[(c >> 1) & 3] = f2_add(acc[(c >> 1) & 3], e);
-            float e0, e1;
-            f2_unpack(e, e0, e1);
-            pk[c >> 1] = pack16<kFP16>(e0, e1);
-          }
-        };
-        if (active) {
-          uint32_t r[64];
-          load_half(0, r);
-          if (row == 0) PKV_TRACE_AT(t, j, 3);
-          const float m0 = half_max(r);
-          if (m0 > m_run + kRescaleLog2) {
-            alpha = ex2_approx(m_run - m0);   // 0 on the first tile (m_run = -inf)
-            l_run *= alpha;
-            m_run = m0;
-            need = true;
-          }
-          exp_half(r, pa);
-        }
-        if (row == 0) PKV_TRACE_AT(t, j, 1);
-        // P_t's columns and O_t are free once PV_t(j-1) is complete; the
-        // first half of P goes out now, so its store overlaps the second half
-        if (kSepP && j > 0) {
-          if (!__all_sync(0xffffffffu, mbar_wait(&bar_pv_done[t], (j - 1) & 1, abort_flag))) { ok = false; break; }
-          tc_fence_after();
-        }
-        if (row == 0) PKV_TRACE_AT(t, j, 4);
-        if (active) {
-          if (kSepP) tmem_st_x32(tP, pa);
-          uint32_t r[64];
-          load_half(1, r);
-          if (row == 0) PKV_TRACE_AT(t, j, 5);
-          const float m1 = half_max(r);
-          const bool rare = m1 > m_run + kRescaleLog2;
-          if (__any_sync(0xffffffffu, rare)) {
-            // Rare: the second half raised the max past the threshold after
-            // the first half's P was formed. Scale that half (and its sum)
-            // down to the new max; the extra rounding stays at the 16-bit
-            // level of P. The TMEM accesses are warp-collective, so the
-            // whole warp takes this branch; other rows scale by 1 (exact).
-            float a2 = 1.f;
-            if (rare) {
-              a2 = ex2_approx(m_run - m1);
-              alpha *= a2;
-              l_run *= a2;
-              m_run = m1;
+          };
+          auto half_max = [&](const uint32_t (&r)[64]) -> float {
+            float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 64; c += 8) {
+              mx0 = fmax3(mx0, __uint_as_float(r[c + 0]), __uint_as_float(r[c + 1]));
+              mx1 = fmax3(mx1, __uint_as_float(r[c + 2]), __uint_as_float(r[c + 3]));
+              mx2 = fmax3(mx2, __uint_as_float(r[c + 4]), __uint_as_float(r[c + 5]));
+              mx3 = fmax3(mx3, __uint_as_float(r[c + 6]), __uint_as_float(r[c + 7]));
+            }
+            return fmax3(mx0, mx1, fmaxf(mx2, mx3)) * sl2;
+          };
+          // P = 2^(s * sl2 - m_run) in 16-bit pairs into pk, summed in fp32
+          // into acc. A half can be fully masked (a short last tile of a
+          // page), so the first half may leave m_run at -inf.
+          auto exp_half = [&](const uint32_t (&sv)[64], uint32_t (&pk)[32]) {
+            // m_run is -inf only while every column so far was masked: P is 0
+            const float mu = m_run == -INFINITY ? 0.f : m_run;
+            const uint64_t negm2 = f2_pack(-mu, -mu);
+#pragma unroll
+            for (int c = 0; c < 64; c += 2) {
+              const uint64_t x = f2_fma(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sl2x2, negm2);
+              uint64_t e;
+              if ((kEmuMask >> ((c >> 1) & 7)) & 1u) {
+                e = exp2_poly2(x);
+              } else {
+                float x0, x1;
+                f2_unpack(x, x0, x1);
+                e = f2_pack(ex2_approx(x0), ex2_approx(x1));
+              }
+              acc[(c >> 1) & 3] = f2_add(acc[(c >> 1) & 3], e);
+              float e0, e1;
+              f2_unpack(e, e0, e1);
+              pk[c >> 1] = pack16<kFP16>(e0, e1);
+            }
+          };
+          {
+            uint32_t r[64];
+            load_half(0, r);
+            const float m0 = half_max(r);
+            if (m0 > m_run + kRescaleLog2) {
+              alpha = ex2_approx(m_run - m0);   // 0 on the first tile (m_run = -inf)
+              l_run *= alpha;
+              m_run = m0;
               need = true;
             }
-            const uint64_t a22 = f2_pack(a2, a2);
+            uint32_t pa[32];
+            exp_half(r, pa);
+            tmem_st_x32(tS, pa);   // P columns 0-31 (16-bit pairs) over S columns 0-31, read
+          }
+          {
+            uint32_t r[64];
+            load_half(1, r);
+            const float m1 = half_max(r);
+            const bool rare = m1 > m_run + kRescaleLog2;
+            if (__any_sync(0xffffffffu, rare)) {
+              // Rare: the second half raised the max past the threshold after
+              // the first half's P was stored. Scale that half (and its sum)
+              // down to the new max; the extra rounding stays at the 16-bit
+              // level of P. The TMEM accesses are warp-collective, so the
+              // whole warp takes this branch; other rows scale by 1 (exact).
+              float a2 = 1.f;
+              if (rare) {
+                a2 = ex2_approx(m_run - m1);
+                alpha *= a2;
+                l_run *= a2;
+                m_run = m1;
+                need = true;
+              }
+              const uint64_t a22 = f2_pack(a2, a2);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) acc[i] = f2_mul(acc[i], a22);
-            if (kSepP) {
+              for (int i = 0; i < 4; ++i) acc[i] = f2_mul(acc[i], a22);
+              uint32_t pa[32];
               tmem_wait_st();
-              tmem_ld_x32_wait(tP, pa);
-            }
+              tmem_ld_x32_wait(tS, pa);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              float p0, p1;
-              unpack16<kFP16>(pa[i], p0, p1);
-              pa[i] = pack16<kFP16>(p0 * a2, p1 * a2);
+              for (int i = 0; i < 32; ++i) {
+                float p0, p1;
+                unpack16<kFP16>(pa[i], p0, p1);
+                pa[i] = pack16<kFP16>(p0 * a2, p1 * a2);
+              }
+              tmem_st_x32(tS, pa);
             }
-            if (kSepP) tmem_st_x32(tP, pa);
+            uint32_t pb[32];
+            exp_half(r, pb);
+            tmem_st_x32(tS + 32, pb);   // P columns 32-63 over S columns 32-63
           }
-          if (kSepP) {   // S_t(j) fully read: the next tile's scores may overwrite it
-            tc_fence_before();
-            mbar_arrive(&bar_s_free[t]);
-          }
-          exp_half(r, pb);
           float s0, s1;
           f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), s0, s1);
           l_run += s0 + s1;
-          if (!kSepP) tmem_st_x32(tP, pa);   // over S_t, now read
-          tmem_st_x32(tP + 32, pb);
-          // rescale O_t if the running max moved
+          // Rescale O_t if the running max moved. O_t holds PV_t(0..j-1);
+          // PV_t(j-2) completed before S_t(j) did, so the wait for PV_t(j-1)
+          // cannot observe an earlier phase of pv_done.
           if (j > 0 && __any_sync(0xffffffffu, need)) {
-            const uint64_t a2 = f2_pack(alpha, alpha);
+            if (!__all_sync(0xffffffffu, mbar_wait(&bar_pv_done[t], (j - 1) & 1, abort_flag))) {
+              ok = false;
+            } else {
+              tc_fence_after();
+              const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll
-            for (int c = 0; c < D; c += 16) {
-              uint32_t o[16];
-              tmem_ld_x16_wait(tO + c, o);
+              for (int c = 0; c < D; c += 16) {
+                uint32_t o[16];
+                tmem_ld_x16_wait(tO + c, o);
 #pragma unroll
-              for (int i = 0; i < 16; i += 2) {
-                float x0, x1;
-                f2_unpack(f2_mul(f2_pack(__uint_as_float(o[i]), __uint_as_float(o[i + 1])), a2), x0, x1);
-                o[i] = __float_as_uint(x0);
-                o[i + 1] = __float_as_uint(x1);
+                for (int i = 0; i < 16; i += 2) {
+                  float x0, x1;
+                  f2_unpack(f2_mul(f2_pack(__uint_as_float(o[i]), __uint_as_float(o[i + 1])), a2), x0, x1);
+                  o[i] = __float_as_uint(x0);
+                  o[i + 1] = __float_as_uint(x1);
+                }
+                tmem_st_x16(tO + c, o);
               }
-              tmem_st_x16(tO + c, o);
             }
           }
-          if (row == 0) PKV_TRACE_AT(t, j, 6);
           tmem_wait_st();
-        } else if (kSepP) {
-          mbar_arrive(&bar_s_free[t]);
         }
         tc_fence_before();
-        if (row == 0) PKV_TRACE_AT(t, j, 2);
-        if ((row & 31) == 0) PKV_TRACE_AT(3, j, 4 * t + (row >> 5));   // each warp's arrival
-        mbar_arrive(&bar_p_full[t]);
+        mbar_arrive(&bar_p_full[b]);
+        if (!ok) break;
       }
       ok = __all_sync(0xffffffffu, ok);
       if (ok && active && __all_sync(0xffffffffu, mbar_wait(bar_o_final, 0, abort_flag))) {
@@ -580,7 +598,7 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
         if (store && slot >= 0) a.part_lse[(size_t)slot * kTile + row] = m_run + log2f(l_run);
       }
     }
-  } else if (kTail && has_tail && (warp == 8 || warp == 10)) {
+  } else if (has_tail && (warp == 8 || warp == 10)) {
     // ------------------------------------------------------------ tail
     // Tail warp w takes K/V rows [64 w, 64 w + 64) of every tile and works
     // transposed, so the few tail rows sit in the narrow dimension:
@@ -627,10 +645,10 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
       for (int j = 0; j < n_tiles; ++j) {
         const int s = j % STAGES;
         if (!__all_sync(0xffffffffu, mbar_wait(&bar_kv_full[s], (j / STAGES) & 1, abort_flag))) { ok = false; break; }
-        PKV_TRACE_AT(2, j, 0);
         const KvTile tl = tile_at(j);
         const uint32_t ks = k_base + s * L::kTileBytes;
         const uint32_t vs = v_base + s * L::kTileBytes;
+        const uint64_t vis = visible_cols(tl, kCW * w);   // this warp's 64 K/V rows
         // S^T: m-tile i = K/V rows kCW w + 16 i .. + 15 (accumulator rows g, g + 8)
         float sc[kMT][NQ][4];
 #pragma unroll
@@ -646,11 +664,10 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
 #pragma unroll
             for (int n = 0; n < NQ; ++n) mma_16816<kFP16>(sc[i][n], af, qb[n][k][0], qb[n][k][1]);
           }
-          // mask K/V rows outside [lo, hi)
+          // mask the K/V rows that are not visible
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const int kvr = kCW * w + 16 * i + g + 8 * h;
-            if (kvr < tl.lo || kvr >= tl.hi)
+            if (!((vis >> (16 * i + g + 8 * h)) & 1))
 #pragma unroll
               for (int n = 0; n < NQ; ++n) sc[i][n][2 * h] = sc[i][n][2 * h + 1] = -INFINITY;
           }
@@ -711,7 +728,6 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar_kv_empty[s]);
-        PKV_TRACE_AT(2, j, 1);
       }
       // this warp's sums per query row
 #pragma unroll
@@ -797,10 +813,12 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
     };
     if (tail_rows <= 8)
       tail_body(std::integral_constant<int, 1>{});
-    else
+    else if (D == 64)   // the planner gives head_dim 128 at most 8 tail rows
       tail_body(std::integral_constant<int, 2>{});
   }
 
+  const bool fuse = a.fused_merge && u.n_chunks > 1;
+  if (fuse) __threadfence();   // this CTA's partials, before its arrival below
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -808,15 +826,50 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
     __syncwarp();
     tmem_dealloc(tmem, kTmemCols);
   }
-  if (threadIdx.x == 0 && *abort_flag) atomicOr(a.err, 1u);
-#ifdef PKV_TRACE
-  if (threadIdx.x == 0 && blockIdx.x < 1024) {
-    uint32_t smid;
-    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
-    g_pkv_cta[blockIdx.x][3] = smid;
+  if (fuse) {
+    // ---------------------------------------------------------- fused merge
+    // The n CTAs of a split group (all resident: the planner fuses only
+    // launches of at most one CTA per SM slot) each arrive once their
+    // partials are written, wait for the others, and merge rows
+    // [k R / n, (k + 1) R / n) of the group's R query rows. The last to
+    // leave resets the two counters for the next launch of the plan.
+    uint32_t* cnt = a.groups + 2 * u.group;
+    const int n = u.n_chunks;
+    if (threadIdx.x == 0) {
+      atomicAdd(cnt, 1u);
+      int ok = 1;
+      const uint64_t t0 = globaltimer_ns();
+      while (ld_acquire_gpu(cnt) < (uint32_t)n) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) { ok = 0; break; }
+        __nanosleep(64);
+      }
+      *merge_ok = ok;
+    }
+    __syncthreads();
+    if (*merge_ok) {
+      __threadfence();   // order this thread's reads after the arrivals it saw
+      auto rows_of = [&](int t) { return t < nq ? min(kTile, rq.T - (u.qtile + t) * kTile) : tail_rows; };
+      const int group_rows = rows_of(0) + (nq > 1 ? rows_of(1) : 0) + tail_rows;
+      const int r0 = (int)((long long)u.chunk * group_rows / n);
+      const int r1 = (int)((long long)(u.chunk + 1) * group_rows / n);
+      for (int gr = r0 + warp; gr < r1; gr += R::kWarps) {
+        int t = 0, r = gr;
+        while (t < nq && r >= rows_of(t)) r -= rows_of(t++);
+        const int orow = rq.q_row0 + (u.qtile + t) * kTile + r;
+        uint16_t* out_row = reinterpret_cast<uint16_t*>(a.out) + ((size_t)orow * a.H + u.head) * D;
+        merge_row_warp<D, kFP16>(a.part_o, a.part_lse, u.slot[t] - u.chunk, n, r, out_row, lane);
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      if (!*merge_ok) atomicOr(a.err, 1u);
+      if (atomicAdd(cnt + 1, 1u) == (uint32_t)(n - 1)) {
+        atomicExch(cnt, 0u);
+        atomicExch(cnt + 1, 0u);
+      }
+    }
   }
-#endif
-  PKV_CTA_AT(2);
+  if (threadIdx.x == 0 && *abort_flag) atomicOr(a.err, 1u);
 }
 
 // Exponentials on the FMA pipe: pair positions {6, 7} of every 8 (25 %).
@@ -844,17 +897,8 @@ cudaError_t launch_attention(const AttnMaps& maps, const AttnArgs& a, int D, boo
 
 int attention_ctas_per_sm(int) { return 1; }
 
-bool attention_tail_ok(int D) { return D == 64; }
-
-#ifdef PKV_TRACE
-extern "C" int kv_debug_trace(void* host, size_t bytes) {
-  if (bytes < sizeof(g_pkv_trace)) return -1;
-  return cudaMemcpyFromSymbol(host, g_pkv_trace, sizeof(g_pkv_trace)) == cudaSuccess ? 0 : -7;
-}
-extern "C" int kv_debug_cta(void* host, size_t bytes) {
-  if (bytes < sizeof(g_pkv_cta)) return -1;
-  return cudaMemcpyFromSymbol(host, g_pkv_cta, sizeof(g_pkv_cta)) == cudaSuccess ? 0 : -7;
-}
-#endif
+// head_dim 128 keeps tails to one 8-row n-tile: its 16-row form would hold
+// 64 fp32 output accumulators per lane and spill at the 168-register cap.
+int attention_max_tail_rows(int D) { return D == 64 ? kMaxTailRows : 8; }
 
 }  // namespace pkv

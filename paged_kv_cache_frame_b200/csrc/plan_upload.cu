@@ -29,8 +29,11 @@ static cudaError_t launch_chunk(uint32_t* dst, const uint32_t* src, int n, cudaS
   return launch_pdl(plan_upload_kernel<kWords>, dim3(1), dim3(256), 0, stream, c);
 }
 
+constexpr int kMax = 7680;   // 30 KB of payload per launch (kernel parameters allow 32 KB)
+
+int upload_launches(size_t bytes) { return (int)(((bytes + 3) / 4 + kMax - 1) / kMax); }
+
 cudaError_t upload_plan(void* dst, const void* src, size_t bytes, cudaStream_t stream) {
-  constexpr int kMax = 7680;   // 30 KB of payload per launch (kernel parameters allow 32 KB)
   const uint32_t* s = static_cast<const uint32_t*>(src);
   uint32_t* d = static_cast<uint32_t*>(dst);
   size_t words = (bytes + 3) / 4;

@@ -88,11 +88,11 @@ def assert_close_dense(out, want, what=""):
     return mx, mean
 
 
-def new_cache(pkv, wl, num_blocks=1, patch_pages=0, cross_special=True):
+def new_cache(pkv, wl, num_blocks=1, patch_pages=0, cross_special=True, camera_only=False):
     max_pages = (patch_pages or wl.patch_pages) + wl.special_pages
     c = pkv.PagedKVCache(max_pages, wl.page_size, wl.H, wl.D, wl.S, wl.W, num_blocks=num_blocks,
                          num_special=wl.NS, dtype=wl.dtype, patch_pages=patch_pages,
-                         cross_frame_special=cross_special)
+                         cross_frame_special=cross_special, camera_only=camera_only)
     c.allocate_pools("cuda")
     return c
 
@@ -102,27 +102,38 @@ def workspace(pkv, caches):
 
 
 def run_stream(pkv, wl, seed, n_frames, check, rows=None, defer=None, keep=None,
-               tiles_per_split=0, patch_pages=0, collect=None, dense=(), cross_special=True):
+               tiles_per_split=0, patch_pages=0, collect=None, dense=(), cross_special=True,
+               camera_only=False, fused=False):
     """Append frames 0..n_frames-1 of block 0; at frames in `check`, plan + run
     and compare the chosen query rows with the oracle. defer[f] / keep[f]:
     frame f is appended with eviction deferred and then committed (keep) or
     rolled back. At frames in `dense`, every row is also checked against the
-    fp32 dense gather of the visible pages. Returns {frame: (max_err, mean_err)}."""
+    fp32 dense gather of the visible pages. fused: each frame goes through
+    begin_frame + plan + run_append (the append inside the attention launch)
+    instead of append_frame + plan + run. Returns {frame: (max_err, mean_err)}."""
     fr = Frames(wl, seed)
-    cache = new_cache(pkv, wl, patch_pages=patch_pages, cross_special=cross_special)
+    cache = new_cache(pkv, wl, patch_pages=patch_pages, cross_special=cross_special, camera_only=camera_only)
     ws = workspace(pkv, [cache])
-    so = StreamOracle(wl.S, wl.W, wl.NS, wl.P, wl.dtype, fr.bits, cross_frame_special=cross_special)
+    so = StreamOracle(wl.S, wl.W, wl.NS, wl.P, wl.dtype, fr.bits, cross_frame_special=cross_special,
+                      camera_only=camera_only)
     res = {}
     for f in range(n_frames):
         q, k, v = (x.cuda() for x in fr.get(f))
         d = bool(defer[f]) if defer is not None else False
         cache.defer_eviction(d)
-        cache.append_frame(0, k, v)
-        cache.evict_frames()
+        if fused:
+            cache.begin_frame()
+            cache.evict_frames()
+            plan = pkv.Plan([cache], ws, tiles_per_split=tiles_per_split)
+            out = plan.run_append(0, k, v, q)
+        else:
+            cache.append_frame(0, k, v)
+            cache.evict_frames()
         so.begin_frame(f, d)
         if f in check:
-            plan = pkv.Plan([cache], ws, tiles_per_split=tiles_per_split)
-            out = plan.run(0, q)
+            if not fused:
+                plan = pkv.Plan([cache], ws, tiles_per_split=tiles_per_split)
+                out = plan.run(0, q)
             plan.check_device()
             sel = slice(None) if rows is None else torch.as_tensor(rows)
             res[f] = assert_close(out[sel], so.expected(rows), f"frame {f}")

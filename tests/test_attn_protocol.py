@@ -9,22 +9,19 @@ every earlier MMA has run, in random interleavings. It checks:
   * every parity wait polls only while its barrier has completed k or k + 1
     phases, k being the phase it waits for (otherwise the parity is
     ambiguous);
-  * each TMEM buffer is read while it still holds the scores S being read,
-    PV_n runs after every warp with valid rows stored P_n, and new scores
-    are written into a buffer only after the PV that reads its P ran;
+  * a softmax warp reads scores S_n while their buffer still holds them;
+    PV_n runs after every warp with valid rows stored P_n; new scores are
+    written into a buffer only after the PV that reads its P ran;
   * O_t is rescaled at tile j after PV_t(j-1) ran and before PV_t(j) runs;
   * a K/V stage is reloaded only after every MMA reading it ran;
   * nothing deadlocks.
 
-Three schedules are modelled. "current" is the kernel's for head_dim 64:
-scores S_t, 16-bit P_t in separate TMEM columns, S_t(j+1) issued once
-softmax t has read S_t(j). "head_dim_128" is the kernel's for head_dim 128:
-P_t stored over S_t, PV_t(j) issued once P_t(j) is written and S_t(j+1)
-right after it into the same columns, with no tail. "three_buffer" is a
-successor under consideration for head_dim 64: P stored over its S,
-three S/P buffers taken in turn, S number n issued once PV number n-3 has
-been issued. The model shows that the three-buffer schedule needs two rules
-(each test below drops one and finds the failure).
+The schedule modelled is the kernel's: score tile n = j * nq + t goes to
+TMEM buffer n % NB (NB = 3 for head_dim 64 with two query tiles, else 2) with
+its P stored over it; per-buffer s_full / p_full barriers; the issuer issues
+S_n once PV_{n-NB} has been issued and PV_n once P_n is written, both in
+order of n; a softmax warp waits for PV_t(j-1) only when it rescales O_t. The
+negative tests drop one rule each and find the failure it prevents.
 
 A model is not the kernel: it checks the protocol's logic only.
 """
@@ -57,86 +54,66 @@ class Bar:
         return self.done == k + 1
 
 
-def run(schedule, nq, n_tiles, active, tail, seed, gate_on_taken=True, idle_warps_wait=True):
+def run(nq, n_tiles, active, tail, seed, nb=None, gate_slack=0, idle_warps_wait=True, rescale_p=0.2):
+    """nb: S/P buffers (default: the kernel's choice, 3 for two query tiles
+    else 2). gate_slack: S_n issued once PV_{n-NB+gate_slack} is issued (0 is
+    the kernel's rule, -1 one PV too early). idle_warps_wait: warps without valid rows wait for
+    their scores before they arrive (the kernel's rule)."""
     rng = random.Random(seed)
-    three = schedule == "three_buffer"
-    h128 = schedule == "head_dim_128"
-    tail = tail and not h128          # head_dim 128 has no tail warps
-    s_full = [Bar(f"s_full{t}", 1) for t in range(2)]
-    s_free = [Bar(f"s_free{t}", 128) for t in range(2)]
-    p_full = [Bar(f"p_full{t}", 128) for t in range(2)]
+    if nb is None:
+        nb = 3 if nq == 2 else 2
+    s_full = [Bar(f"s_full{b}", 1) for b in range(3)]
+    p_full = [Bar(f"p_full{b}", 128) for b in range(3)]
     pv_done = [Bar(f"pv_done{t}", 1) for t in range(2)]
     kv_full = [Bar(f"kv_full{s}", 1) for s in range(ST)]
     kv_empty = [Bar(f"kv_empty{s}", 1 + (2 if tail else 0)) for s in range(ST)]
     o_final = Bar("o_final", 1)
     pipe, ran, holds, p_written, stage = [], set(), {}, {}, {}
-    number = lambda t, j: j * nq + t
-    buffer = lambda t, j: number(t, j) % 3 if three else t
+    n_all = n_tiles * nq
 
     def execute(op):
         if op[0] == "commit":
             op[1].arrive()
             return
-        kind, t, j = op
-        n = number(t, j)
+        kind, n = op
+        j, t, b = n // nq, n % nq, n % nb
         if stage.get(j % ST) != j:
-            raise Violation(f"{kind}_{t}({j}) runs without its K/V tile")
+            raise Violation(f"{kind}_{n} runs without its K/V tile")
         if kind == "S":
-            if three and n >= 3 and ("PV", (n - 3) % nq, (n - 3) // nq) not in ran:
-                raise Violation(f"S number {n} overwrites P before PV number {n - 3} ran")
-            if h128 and j > 0 and ("PV", t, j - 1) not in ran:
-                raise Violation(f"S_{t}({j}) overwrites P_{t}({j - 1}) before its PV ran")
-            holds[buffer(t, j)] = n
+            if n >= nb and ("PV", n - nb) not in ran:
+                raise Violation(f"S_{n} overwrites buffer {b} before PV_{n - nb} read its P")
+            holds[b] = n
         else:
+            if holds.get(b) != n:
+                raise Violation(f"PV_{n} reads buffer {b} holding S_{holds.get(b)}")
             if p_written.get(n, set()) != {w for w in range(4) if active[t][w]}:
-                raise Violation(f"PV_{t}({j}) runs before P_{t}({j}) is written")
-        ran.add((kind, t, j))
+                raise Violation(f"PV_{n} runs before P_{n} is written")
+        ran.add((kind, n))
 
     def issuer():
-        st = {"started": False, "done": False, "ns": [1, 1], "np": [0, 0], "ne": 0, "kv": 0}
-        if nq < 2:
-            st["ns"][1] = st["np"][1] = n_tiles
-
-        def issue(kind, t, j, bar):
-            pipe.append((kind, t, j))
-            pipe.append(("commit", bar))
+        st = {"ns": 0, "np": 0, "ne": 0, "kv": -1, "q": False, "done": False}
 
         def step():
             if st["done"]:
                 return None
-            if not st["started"]:
-                if not kv_full[0].test(0, "issuer"):
-                    return False
-                for t in range(nq):
-                    issue("S", t, 0, s_full[t])
-                st["started"] = True
-                return True
             moved = False
             ns, np_ = st["ns"], st["np"]
-            for t in range(2):
-                j = ns[t]
-                if j >= n_tiles:
-                    continue
-                if three:
-                    m = number(t, j) - 3
-                    if m >= 0 and np_[m % nq] <= m // nq:
-                        continue
-                if (not three or gate_on_taken) and not s_free[t].test(j - 1, "issuer"):
-                    continue
-                if j > st["kv"]:
-                    if not kv_full[j % ST].test(j // ST, "issuer"):
-                        continue
-                    st["kv"] = j
-                issue("S", t, j, s_full[t])
-                ns[t] = j + 1
-                moved = True
-            for t in range(2):
-                j = np_[t]
-                if j < n_tiles and p_full[t].test(j, "issuer"):
-                    issue("PV", t, j, pv_done[t])
-                    np_[t] = j + 1
+            if ns < n_all and ns - nb + gate_slack < np_:
+                j = ns // nq
+                ready = j <= st["kv"]
+                if not ready and kv_full[j % ST].test(j // ST, "issuer"):
+                    st["kv"], ready = j, True
+                if ready:
+                    pipe.append(("S", ns))
+                    pipe.append(("commit", s_full[ns % nb]))
+                    st["ns"] = ns + 1
                     moved = True
-            while st["ne"] < min(np_):
+            if np_ < st["ns"] and p_full[np_ % nb].test(np_ // nb, "issuer"):
+                pipe.append(("PV", np_))
+                pipe.append(("commit", pv_done[np_ % nq]))
+                st["np"] = np_ + 1
+                moved = True
+            while st["ne"] < n_tiles and st["np"] >= (st["ne"] + 1) * nq:
                 pipe.append(("commit", kv_empty[st["ne"] % ST]))
                 st["ne"] += 1
                 moved = True
@@ -147,49 +124,9 @@ def run(schedule, nq, n_tiles, active, tail, seed, gate_on_taken=True, idle_warp
             return moved
         return step
 
-    def issuer_128():
-        """Serialized: per tile, per query tile, PV_t(j) once P_t(j) is written
-        and S_t(j+1) right after it; then the K/V stage is released."""
-        st = {"started": False, "done": False, "j": 0, "t": 0, "pv": False}
-
-        def step():
-            if st["done"]:
-                return None
-            if not st["started"]:
-                if not kv_full[0].test(0, "issuer"):
-                    return False
-                for t in range(nq):
-                    pipe.append(("S", t, 0))
-                    pipe.append(("commit", s_full[t]))
-                st["started"] = True
-                return True
-            j, t = st["j"], st["t"]
-            if not st["pv"]:
-                if not p_full[t].test(j, "issuer"):
-                    return False
-                pipe.append(("PV", t, j))      # no commit: S_t(j+1)'s covers it
-                st["pv"] = True
-                return True
-            if j + 1 < n_tiles:
-                if not kv_full[(j + 1) % ST].test((j + 1) // ST, "issuer"):
-                    return False
-                pipe.append(("S", t, j + 1))
-                pipe.append(("commit", s_full[t]))
-            st["pv"] = False
-            if t + 1 < nq:
-                st["t"] = t + 1
-                return True
-            pipe.append(("commit", kv_empty[j % ST]))
-            st["t"], st["j"] = 0, j + 1
-            if st["j"] >= n_tiles:
-                pipe.append(("commit", o_final))
-                st["done"] = True
-            return True
-        return step
-
     def softmax_warp(t, w):
         rows = active[t][w]
-        st = {"j": 0, "pc": 0}
+        st = {"j": 0, "pc": 0, "rescale": False}
         who = f"softmax {t}.{w}"
 
         def step():
@@ -201,41 +138,34 @@ def run(schedule, nq, n_tiles, active, tail, seed, gate_on_taken=True, idle_warp
                     st["pc"] = 1
                     return True
                 return None
-            n, b = number(t, j), buffer(t, j)
-            if pc == 0:                           # S_t(j) computed
-                if not s_full[t].test(j, who):
-                    return False
-                if three and gate_on_taken:
-                    s_free[t].arrive(32)          # taken: S_t(j+1) may be issued
-                st["pc"] = 1
-            elif pc == 1:                         # first half of the scores
-                if rows and holds.get(b) != n:
-                    raise Violation(f"{who} reads S number {n}, buffer holds {holds.get(b)}")
-                st["pc"] = 2 if three or h128 or j == 0 else 10
-            elif pc == 10:                        # current: P_t free once PV_t(j-1) is done
-                if not pv_done[t].test(j - 1, who):
-                    return False
+            n = j * nq + t
+            b = n % nb
+            if pc == 0:                           # S_n computed
+                if rows or idle_warps_wait:
+                    if not s_full[b].test(n // nb, who):
+                        return False
+                st["pc"] = 1 if rows else 5
+            elif pc == 1:                         # first half of the scores read
+                if holds.get(b) != n:
+                    raise Violation(f"{who} reads S_{n}, buffer {b} holds {holds.get(b)}")
                 st["pc"] = 2
-            elif pc == 2:                         # second half
-                if rows and holds.get(b) != n:
-                    raise Violation(f"{who} reads S number {n}, buffer holds {holds.get(b)}")
-                if not three and not h128:
-                    s_free[t].arrive(32)          # current: S_t(j) read
+            elif pc == 2:                         # second half read; P stored over the first
+                if holds.get(b) != n:
+                    raise Violation(f"{who} reads S_{n}, buffer {b} holds {holds.get(b)}")
+                st["rescale"] = j > 0 and rng.random() < rescale_p
                 st["pc"] = 3
-            elif pc == 3:                         # P stores complete
-                if rows:
-                    p_written.setdefault(n, set()).add(w)
-                st["pc"] = 4
-            elif pc == 4:                         # three_buffer: O_t free once PV_t(j-1) is done
-                if three and j > 0 and (rows or idle_warps_wait):
+            elif pc == 3:                         # O rescale: wait for PV_t(j-1) only then
+                if st["rescale"]:
                     if not pv_done[t].test(j - 1, who):
                         return False
-                st["pc"] = 5
-            elif pc == 5:                         # rare O rescale, then P_t(j) handed over
-                if rows and j > 0 and rng.random() < 0.2:
-                    if ("PV", t, j - 1) not in ran or ("PV", t, j) in ran:
+                    if ("PV", n - nq) not in ran or ("PV", n) in ran:
                         raise Violation(f"{who} rescales O_{t} at tile {j} while a PV may run")
-                p_full[t].arrive(32)
+                st["pc"] = 4
+            elif pc == 4:                         # P stores complete
+                p_written.setdefault(n, set()).add(w)
+                st["pc"] = 5
+            elif pc == 5:                         # P_n handed over
+                p_full[b].arrive(32)
                 st["j"], st["pc"] = j + 1, 0
             return True
         return step
@@ -250,10 +180,10 @@ def run(schedule, nq, n_tiles, active, tail, seed, gate_on_taken=True, idle_warp
             if j >= ST:
                 if not kv_empty[j % ST].test(j // ST - 1, "producer"):
                     return False
-                for t in range(nq):
+                for n in range((j - ST) * nq, (j - ST + 1) * nq):
                     for kind in ("S", "PV"):
-                        if (kind, t, j - ST) not in ran:
-                            raise Violation(f"stage reloaded before {kind}_{t}({j - ST}) ran")
+                        if (kind, n) not in ran:
+                            raise Violation(f"stage reloaded before {kind}_{n} ran")
             stage[j % ST] = j
             kv_full[j % ST].arrive()
             st["j"] = j + 1
@@ -280,7 +210,7 @@ def run(schedule, nq, n_tiles, active, tail, seed, gate_on_taken=True, idle_warp
         execute(pipe.pop(0))
         return True
 
-    actors = [issuer_128() if h128 else issuer(), producer()]
+    actors = [issuer(), producer()]
     actors += [softmax_warp(t, w) for t in range(nq) for w in range(4)]
     actors += [tail_warp(), tail_warp()] if tail else []
     finished = [False] * len(actors)
@@ -304,9 +234,9 @@ def run(schedule, nq, n_tiles, active, tail, seed, gate_on_taken=True, idle_warp
             raise Violation("deadlock")
 
 
-def random_case(seed):
+def random_case(seed, nq=None):
     rng = random.Random(seed)
-    nq = rng.choice([1, 2])
+    nq = nq or rng.choice([1, 2])
     active = [[True] * 4 for _ in range(2)]
     if rng.random() < 0.5:   # a short frame: some warps have no valid rows
         active = [[True] + [rng.random() < 0.5 for _ in range(3)] for _ in range(2)]
@@ -314,32 +244,45 @@ def random_case(seed):
                 tail=nq == 2 and rng.random() < 0.5, seed=seed)
 
 
-def violations(schedule, cases, **rules):
+def violations(cases, nq=None, **rules):
     found = []
     for seed in range(cases):
         try:
-            run(schedule, **random_case(seed), **rules)
+            run(**random_case(seed, nq), **rules)
         except Violation as e:
             found.append((seed, str(e)))
     return found
 
 
-@pytest.mark.parametrize("schedule", ["current", "head_dim_128", "three_buffer"])
-def test_schedule_is_race_free(schedule):
-    assert violations(schedule, 1500) == []
+@pytest.mark.parametrize("nq", [1, 2])
+def test_kernel_schedule_is_race_free(nq):
+    assert violations(1500, nq=nq) == []
 
 
-def test_three_buffer_schedule_needs_the_taken_gate():
-    """Without it S_t(j+1) may complete before softmax t has waited for
-    S_t(j): s_full_t runs two phases ahead and its parity wait loses count."""
-    found = violations("three_buffer", 300, gate_on_taken=False)
-    assert any("s_full" in msg for _, msg in found)
+def test_two_buffers_with_two_query_tiles_are_race_free():
+    """The head_dim 128 kernel: two buffers, so S_t(j+1) follows PV_t(j)."""
+    assert violations(800, nq=2, nb=2) == []
 
 
-def test_three_buffer_schedule_needs_idle_warps_to_wait():
-    """p_full_t counts arrivals, not tiles: warps without valid rows that
-    skip the per-tile PV wait run a tile ahead and complete the phase
-    before the other warps have written P."""
-    found = violations("three_buffer", 300, idle_warps_wait=False)
+def test_scores_issued_one_pv_early_overwrite_p():
+    """S_n issued once PV_{n-NB-1} is issued (one PV too early) can
+    overwrite P_{n-NB} before the PV that reads it has run."""
+    found = violations(300, gate_slack=-1, rescale_p=0.0)
+    assert any("overwrites" in msg for _, msg in found)
+
+
+def test_three_buffers_with_one_query_tile_break_the_rescale_wait():
+    """With one query tile and three buffers, S_t(j) completing no longer
+    implies PV_t(j-2) completed, so the O rescale's parity wait on pv_done
+    can see the phase before the one it waits for."""
+    found = violations(400, nq=1, nb=3, rescale_p=0.5)
+    assert any("pv_done" in msg for _, msg in found)
+
+
+def test_idle_warps_must_wait_for_their_scores():
+    """p_full counts arrivals: warps without valid rows that arrive without
+    waiting for S_n run ahead and complete a phase before the warps with
+    rows have written P."""
+    found = violations(300, idle_warps_wait=False)
     assert found
     assert all(random_case(seed)["active"] != [[True] * 4] * 2 for seed, _ in found)

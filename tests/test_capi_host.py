@@ -338,7 +338,9 @@ def test_kv_tiles_cover_visible_tokens_exactly_once(pkv, ps, n, xs):
 
 
 def test_split_schedule_covers_each_unit(pkv):
-    """Host plan for the 224x224 shape at frame 320: 159 tiles per head,
+    """Host plan for the 224x224 shape at frame 320: 160 tiles per head
+    (71 earlier patch pages x 2, the current frame's page x 2, the earlier
+    1914 special tokens in 15 tiles, the current frame's 6 in their own),
     16 heads x 3 query tiles (one pair-plus-tail unit per head); a forced
     split of 10 tiles per CTA."""
     h = pkv.kv_init(81, 256, 16, 64, 8, 64, 1, 6, pkv.KV_BF16, 0)
@@ -346,17 +348,23 @@ def test_split_schedule_covers_each_unit(pkv):
         step(pkv, h)
     p = pkv.kv_plan([h], tiles_per_split=10)
     s = pkv.kv_plan_get_stats(p)
-    assert s["n_kv_tiles"] == 159
+    assert s["n_kv_tiles"] == 160
     assert s["visible_tokens"] == 72 * 256 + 6 * 320
     assert s["n_split_units"] == 48          # every (head, query tile) is split
     # per head one unit: query tiles 0-1 plus the 6-row tail tile 2, in
     # ceil(159/10) = 16 chunks
     assert s["n_ctas"] == 16 * 16
     assert s["tiles_per_cta"] <= 10
+    assert s["fused_merge"] == 0             # 256 CTAs cannot all be resident: a merge launch
     pkv.kv_plan_free(p)
     p = pkv.kv_plan([h])                   # automatic: fills 148 SMs
     s = pkv.kv_plan_get_stats(p)
     assert 100 <= s["n_ctas"] <= 2 * 148 + 16
+    # the automatic schedule fits one CTA per SM, so each split group merges itself
+    assert s["n_ctas"] <= 148 and s["fused_merge"] == 1
+    pkv.kv_plan_free(p)
+    p = pkv.kv_plan([h], tiles_per_split=200)   # no split: nothing to merge
+    assert pkv.kv_plan_get_stats(p)["fused_merge"] == 0
     pkv.kv_plan_free(p)
     pkv.kv_destroy(h)
 
@@ -428,7 +436,8 @@ def test_get_config_reports_what_init_fixed(pkv):
     cfg = pkv.kv_get_config(h)
     assert cfg == {"max_pages": 90, "page_size": 256, "num_heads": 16, "head_dim": 64, "scale_frames": 8,
                    "window": 64, "num_blocks": 24, "num_special": 6, "dtype": pkv.KV_FP16,
-                   "patch_pages": 73, "tokens_per_frame": 262, "cross_frame_special": 1}
+                   "patch_pages": 73, "special_base": 73, "special_pages": 17, "tokens_per_frame": 262,
+                   "cross_frame_special": 1, "camera_only": 0}
     pkv.kv_set_cross_frame_special(h, False)
     assert pkv.kv_get_config(h)["cross_frame_special"] == 0
     pkv.kv_destroy(h)
@@ -515,9 +524,11 @@ def test_inspection_calls_copy_at_most_cap_and_check_ranges(pkv):
     assert n.value == len(full) and lpl.value == lpl_full
     assert list(buf[:2]) == full[:2] and list(buf[2:]) == [-7] * 6
     tiles = pkv.kv_get_kv_tiles(p)
-    row, lo, hi = ((ctypes.c_int * 4)(*([-7] * 4)) for _ in range(3))
-    assert lib.kv_get_kv_tiles(p, 0, row, lo, hi, 1, ctypes.byref(n)) == 0
-    assert n.value == len(tiles) and (row[0], lo[0], hi[0]) == tiles[0] and row[1] == -7
+    row, lo, hi, kr, sp = ((ctypes.c_int * 4)(*([-7] * 4)) for _ in range(5))
+    assert lib.kv_get_kv_tiles(p, 0, row, lo, hi, kr, sp, 1, ctypes.byref(n)) == 0
+    assert n.value == len(tiles) and (row[0], lo[0], hi[0]) == tiles[0] and row[1] == -7 and kr[1] == -7
+    assert sp[0] == 1 and sp[1] == -7
+    assert lib.kv_get_kv_tiles(p, 0, row, lo, hi, None, None, 1, ctypes.byref(n)) == 0   # krow, step optional
     free = pkv.kv_get_free_list(h)
     fb = (ctypes.c_int * 4)(*([-7] * 4))
     assert lib.kv_get_free_list(h, fb, 1, ctypes.byref(n)) == 0
@@ -536,3 +547,268 @@ def test_inspection_calls_copy_at_most_cap_and_check_ranges(pkv):
     assert e.value.code == E.KV_ERR_CAPACITY
     assert pkv.kv_workspace_bytes(many) == 0
     pkv.kv_destroy(h)
+
+
+def snapshot(pkv, h):
+    s = pkv.kv_get_stats(h)
+    free = pkv.kv_get_free_list(h)
+    try:
+        tab = table(pkv, [h])
+    except pkv.KVError as e:
+        tab = e.value.name if hasattr(e, "value") else e.name
+    return s, free, tab
+
+
+@settings(max_examples=60, deadline=None)
+@given(ops=st.lists(st.sampled_from(["key", "key", "defer_keep", "defer_drop"]), min_size=1, max_size=30),
+       S=st.integers(0, 2), W=st.integers(0, 3), B=st.integers(1, 3), xs=st.booleans())
+def test_begin_frame_is_the_step_opening_append(pkv, ops, S, W, B, xs):
+    """A step opened by kv_begin_frame, then every block appended, leaves the
+    page state a step opened by the first block's append leaves: same stats,
+    free list and page table after every operation."""
+    a = mk(pkv, S, W, 16, S + W + 1 + 20, B=B)
+    b = mk(pkv, S, W, 16, S + W + 1 + 20, B=B)
+    for h in (a, b):
+        pkv.kv_set_cross_frame_special(h, xs)
+    for op in ops:
+        defer = op != "key"
+        for h in (a, b):
+            pkv.kv_defer_eviction(h, defer)
+        pkv.kv_begin_frame(b)
+        for blk in range(B):
+            pkv.kv_append_frame(a, blk, None, None)
+            pkv.kv_append_frame(b, blk, None, None)
+            if blk == 0:
+                assert snapshot(pkv, a) == snapshot(pkv, b)
+        for h in (a, b):
+            pkv.kv_evict_frames(h)
+            if op == "defer_keep":
+                pkv.kv_commit_frame(h)
+            elif op == "defer_drop":
+                pkv.kv_rollback_last_frame(h)
+        assert snapshot(pkv, a) == snapshot(pkv, b)
+    pkv.kv_destroy(a)
+    pkv.kv_destroy(b)
+
+
+def test_begin_frame_errors_leave_the_state_unchanged(pkv):
+    E = pkv.capi
+    h = mk(pkv, 1, 1, 16, 4, B=2)               # patch pool S + W + 1 = 3 pages, 1 special page
+    pkv.kv_begin_frame(h)
+    before = snapshot(pkv, h)
+    with pytest.raises(pkv.KVError) as e:        # the open step still has blocks to append
+        pkv.kv_begin_frame(h)
+    assert e.value.code == E.KV_ERR_ORDER and snapshot(pkv, h) == before
+    pkv.kv_append_frame(h, 0, None, None)
+    with pytest.raises(pkv.KVError) as e:        # block 1 still to append
+        pkv.kv_begin_frame(h)
+    assert e.value.code == E.KV_ERR_ORDER
+    pkv.kv_append_frame(h, 1, None, None)
+    pkv.kv_evict_frames(h)
+    pkv.kv_begin_frame(h)                        # the step is complete: a new one opens
+    assert pkv.kv_get_stats(h)["frame_count"] == 2
+    for blk in range(2):
+        pkv.kv_append_frame(h, blk, None, None)
+    pkv.kv_evict_frames(h)
+    # 16-token special page: 2 frames of 6 fit, a third does not
+    before = snapshot(pkv, h)
+    with pytest.raises(pkv.KVError) as e:
+        pkv.kv_begin_frame(h)
+    assert e.value.code == E.KV_ERR_CAPACITY and snapshot(pkv, h) == before
+    # a pending frame of an earlier step must be decided first
+    h2 = mk(pkv, 1, 1, 16, 20, B=1)
+    pkv.kv_defer_eviction(h2, True)
+    pkv.kv_begin_frame(h2)
+    pkv.kv_append_frame(h2, 0, None, None)
+    with pytest.raises(pkv.KVError) as e:
+        pkv.kv_begin_frame(h2)
+    assert e.value.code == E.KV_ERR_ORDER
+    pkv.kv_rollback_last_frame(h2)
+    assert pkv.kv_get_stats(h2)["frame_count"] == 0
+    pkv.kv_destroy(h)
+    pkv.kv_destroy(h2)
+
+
+def test_run_append_argument_checks_on_the_host(pkv):
+    E = pkv.capi
+    h = mk(pkv, 1, 2, 16, 8)
+    pkv.kv_begin_frame(h)
+    p = pkv.kv_plan([h])                          # host-only plan: no workspace
+    a = 1 << 20
+    for args, code in [((p, 0, None, a, a, a), E.KV_ERR_ARG),     # NULL k
+                       ((p, 0, a, None, a, a), E.KV_ERR_ARG),     # NULL v
+                       ((p, 0, a, a, a, a), E.KV_ERR_ARG)]:       # plan without a workspace
+        with pytest.raises(pkv.KVError) as e:
+            pkv.kv_run_append(*args)
+        assert e.value.code == code
+    pkv.kv_plan_free(p)
+    pkv.kv_destroy(h)
+
+
+def test_current_frame_tiles_carry_their_k_v_rows(pkv):
+    """The open step's frame is tiled on its own, each tile with the k/v row
+    of its column 0: its patch page (rows NS.. of k/v) and its NS special
+    tokens (rows 0..NS-1); other tiles carry none. Checked through the
+    coverage: every visible token once, the frame's tokens on current tiles."""
+    ps, S, W = 256, 8, 64
+    h = mk(pkv, S, W, ps, 73 + 9, B=2)
+    for f in range(100):
+        step(pkv, h, B=2)
+    pkv.kv_begin_frame(h)                         # frame 100 opens: page and special slots 600..605
+    pkv.kv_evict_frames(h)
+    p = pkv.kv_plan([h])
+    s = pkv.kv_plan_get_stats(p)
+    tiles = pkv.kv_get_kv_tiles(p)
+    # 71 earlier patch pages (2 tiles each), the frame's page (2), the earlier
+    # 600 special tokens (5 tiles), the frame's 6 (1 tile)
+    assert s["n_kv_tiles"] == len(tiles) == 142 + 2 + 5 + 1
+    cover = tile_cover(tiles, ps)
+    assert len(cover) == len(set(cover)) == s["visible_tokens"] == 72 * ps + 606
+    # the frame's tokens are exactly the current tiles' columns, mapped to
+    # their k/v rows: special token 600 + i is row i, patch slot x row 6 + x
+    page = pkv.kv_get_free_list(h)  # noqa: F841  (the page is read from the table below)
+    frame_page = pkv.kv_get_page_table(p)[0][71]          # scale 8 + window 64, the newest last
+    Np = 73
+    got = {}
+    for row, lo, hi, kr, _ in pkv.kv_get_kv_tiles(p, with_krow=True):
+        for col in range(lo, hi):
+            tok = divmod(row + col, 2 * ps)
+            if kr == pkv.KV_NOT_CURRENT:
+                assert tok[0] != frame_page and not (tok[0] == Np + 2 and 88 <= tok[1] < 94)
+            else:
+                got[tok] = kr + col
+    want = {(frame_page, x): 6 + x for x in range(ps)}
+    want.update({(Np + 2, 88 + i): i for i in range(6)})   # tokens 600..605: page 2, slots 88..93
+    assert got == want
+    pkv.kv_plan_free(p)
+    pkv.kv_destroy(h)
+
+
+def strided_cover(tiles, ps):
+    """(page, token) pairs that (row, lo, hi, krow, step) tiles mark visible."""
+    out = []
+    for row, lo, hi, _, step in tiles:
+        for col in range(lo, hi, step):
+            page, rem = divmod(row + col, 2 * ps)
+            assert rem < ps, "a visible column must be a K row of its page"
+            out.append((page, rem))
+    return out
+
+
+@pytest.mark.parametrize("xs", [True, False])
+@pytest.mark.parametrize("ps,n", [(16, 12), (256, 320), (999, 40), (130, 150), (64, 100), (7, 30)])
+def test_camera_only_tiles_cover_the_camera_tokens(pkv, ps, n, xs):
+    """kv_set_camera_only: the tiles cover exactly the oracle's visible camera
+    tokens (slot 0 of each frame's six), each once, with the open step's own
+    camera token on a current-frame tile that maps it to k/v row 0; the page
+    table is the oracle's; the page state is as without camera-only."""
+    S, W = 8, 64
+    pages = math.ceil(6 * (n + 1) / ps) + 1
+    h = mk(pkv, S, W, ps, 73 + pages)
+    ref = mk(pkv, S, W, ps, 73 + pages)
+    for c in (h, ref):
+        pkv.kv_set_cross_frame_special(c, xs)
+    pkv.kv_set_camera_only(h, True)
+    assert pkv.kv_get_config(h)["camera_only"] == 1
+    m = PageModel(S, W, ps, 73 + pages, cross_frame_special=xs, camera_only=True)
+    for f in range(n):
+        step(pkv, h)
+        step(pkv, ref)
+        m.append(f); m.evict()
+    pkv.kv_begin_frame(h)                     # an open step: the frame's tiles are separate
+    pkv.kv_evict_frames(h)
+    m.append(n); m.evict()
+    p = pkv.kv_plan([h])
+    assert pkv.kv_get_page_table(p) == m.page_table()
+    tiles = pkv.kv_get_kv_tiles(p, with_krow=True)
+    want = sorted((m.Np + j // ps, j % ps) for j in m.visible_special_index())
+    assert sorted(strided_cover(tiles, ps)) == want
+    assert pkv.kv_plan_get_stats(p)["visible_tokens"] == m.visible_token_count() == len(want)
+    own = [(row, lo, hi, kr) for row, lo, hi, kr, _ in tiles if kr != pkv.KV_NOT_CURRENT]
+    assert len(own) == 1 and own[0][3] + own[0][1] == 0          # column lo is k/v row 0
+    assert divmod(own[0][0] + own[0][1], 2 * ps) == (m.Np + 6 * n // ps, 6 * n % ps)
+    pkv.kv_plan_free(p)
+    step(pkv, ref)
+    for blk in range(1):
+        pkv.kv_append_frame(h, blk, None, None)
+    assert pkv.kv_get_stats(h) == pkv.kv_get_stats(ref)
+    assert pkv.kv_get_free_list(h) == pkv.kv_get_free_list(ref)
+    pkv.kv_destroy(h)
+    pkv.kv_destroy(ref)
+
+
+@settings(max_examples=80, deadline=None)
+@given(ops=st.lists(st.tuples(st.integers(0, 2), st.sampled_from(["key", "key", "defer_keep", "defer_drop",
+                                                                  "reset"])), min_size=1, max_size=60),
+       S=st.integers(0, 2), W=st.integers(0, 3), ps=st.sampled_from([5, 16]),
+       short=st.booleans())
+def test_group_state_bit_exact_vs_oracle(pkv, ops, S, W, ps, short):
+    """kv_init_group: three streams over one pool. Free list (common), stats
+    and page tables after every operation equal the oracle's shared page
+    models; with a common patch pool smaller than the
+    streams' sum, an append that finds it empty fails with KV_ERR_CAPACITY
+    and changes nothing."""
+    from oracle import SharedPatchPool
+    n, sp_pages = 3, 12
+    Np = n * (S + W + 1) - (2 if short else 0)
+    if Np < 1:
+        return
+    max_pages = Np + n * sp_pages
+    hs = pkv.kv_init_group(n, max_pages, ps, 2, 64, S, W, 1, 6, pkv.KV_BF16, Np, sp_pages)
+    pool = SharedPatchPool(Np)
+    ms = [PageModel(S, W, ps, max_pages, NS=6, shared=pool, sp_base=Np + i * sp_pages, sp_pages=sp_pages)
+          for i in range(n)]
+    nxt = [0] * n
+    for s_i, op in ops:
+        h, m = hs[s_i], ms[s_i]
+        if op == "reset":
+            pkv.kv_reset(h)
+            m.reset()
+            nxt[s_i] = 0
+        elif m.sp_len + 6 <= m.special_capacity:
+            d = op != "key"
+            pkv.kv_defer_eviction(h, d)
+            m.set_defer(d)
+            if not pool.free:
+                with pytest.raises(pkv.KVError) as e:
+                    pkv.kv_append_frame(h, 0, None, None)
+                assert e.value.name == "CAPACITY"
+                pkv.kv_defer_eviction(h, False)
+                m.set_defer(False)
+            else:
+                pkv.kv_append_frame(h, 0, None, None)
+                pkv.kv_evict_frames(h)
+                m.append(nxt[s_i])
+                m.evict()
+                nxt[s_i] += 1
+                if d:
+                    if op == "defer_keep":
+                        pkv.kv_commit_frame(h); m.commit()
+                    else:
+                        pkv.kv_rollback_last_frame(h); m.rollback()
+                        nxt[s_i] -= 1
+        for hh, mm in zip(hs, ms):
+            assert pkv.kv_get_free_list(hh) == pool.free
+            assert pkv.kv_get_stats(hh) == mm.stats()
+            assert_same_table(pkv, hh, mm)
+    cfg = [pkv.kv_get_config(h) for h in hs]
+    assert [c["special_base"] for c in cfg] == [Np + i * sp_pages for i in range(n)]
+    assert all(c["patch_pages"] == Np and c["special_pages"] == sp_pages for c in cfg)
+    for h in hs:
+        pkv.kv_destroy(h)
+
+
+def test_group_argument_checks(pkv):
+    E = pkv.capi
+    with pytest.raises(pkv.KVError) as e:          # 3 x (8 + 64 + 1) patch pages + 3 x 10 special > 240
+        pkv.kv_init_group(3, 240, 256, 16, 64, 8, 64, 24, special_pages=10)
+    assert e.value.code == E.KV_ERR_CAPACITY
+    hs = pkv.kv_init_group(3, 3 * 73 + 30, 256, 16, 64, 8, 64, 24)   # defaults: 219 patch, 10 special each
+    cfg = pkv.kv_get_config(hs[2])
+    assert (cfg["patch_pages"], cfg["special_base"], cfg["special_pages"]) == (219, 239, 10)
+    assert pkv.kv_pool_bytes(hs[0]) == (3 * 73 + 30) * 2 * 256 * 16 * 64 * 2
+    with pytest.raises(pkv.KVError) as e:
+        pkv.kv_init_group(0, 100, 16, 2, 64, 1, 1, 1)
+    assert e.value.code == E.KV_ERR_ARG
+    for h in hs:
+        pkv.kv_destroy(h)

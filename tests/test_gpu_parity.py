@@ -309,3 +309,54 @@ def test_failed_append_launch_leaves_state_unchanged(pkv):
     out = plan.run(1, q)
     plan.check_device()
     assert_close(out, so.expected(), "after failed launches")
+
+
+@pytest.mark.parametrize("H", [2, 4])
+def test_more_than_32_chunks_per_split_unit(pkv, H):
+    """One K/V tile per CTA over 53 visible tiles (48 patch pages of 64 tokens
+    and 5 special pages): 53 chunks per unit, past the merge's first 32-lane
+    pass. H = 2 gives 106 CTAs, which fit on the device at once, so the CTAs
+    merge their own groups; H = 4 gives 212, which do not, so the merge runs
+    as its own launch."""
+    wl = small(64, H=H, S=8, W=40, frames=50)
+    fr = Frames(wl, seed=70)
+    cache = new_cache(pkv, wl)
+    so = StreamOracle(wl.S, wl.W, wl.NS, wl.P, wl.dtype, fr.bits)
+    for f in range(wl.frames):
+        q, k, v = (x.cuda() for x in fr.get(f))
+        cache.append_frame(0, k, v)
+        cache.evict_frames()
+        so.begin_frame(f)
+    plan = pkv.Plan([cache], workspace(pkv, [cache]), tiles_per_split=1)
+    st = plan.stats()
+    assert st["tiles_per_cta"] == 1 and st["n_kv_tiles"] == 53
+    assert st["fused_merge"] == (1 if H == 2 else 0)
+    for rep in range(2):   # the group counters must be back at zero for the second run
+        out = plan.run(0, q)
+        plan.check_device()
+        assert_close(out, so.expected(), f"H={H} run {rep}")
+
+
+
+@pytest.mark.parametrize("xs", [True, False])
+@pytest.mark.parametrize("fused", [False, True])
+def test_camera_only_tiny_every_frame(pkv, xs, fused):
+    """kv_cache_camera_only: each frame attends to the camera tokens (slot 0
+    of each frame's six) only; strided tiles over the special pages."""
+    wl = dataclasses.replace(W0, frames=30)
+    res = run_stream(pkv, wl, seed=90, n_frames=wl.frames, check=set(range(wl.frames)),
+                     cross_special=xs, camera_only=True, fused=fused)
+    assert len(res) == wl.frames
+
+
+@pytest.mark.parametrize("ps", [16, 100, 256, 999])
+def test_camera_only_page_sizes(pkv, ps):
+    wl = small(ps, H=1 if ps == 999 else 2, S=2, W=3, frames=40)
+    run_stream(pkv, wl, seed=91 + ps, n_frames=wl.frames, check={0, 5, 39}, camera_only=True)
+    run_stream(pkv, wl, seed=92 + ps, n_frames=wl.frames, check={39}, camera_only=True, tiles_per_split=1)
+
+
+def test_camera_only_224_stream(pkv):
+    wl = dataclasses.replace(workload.WORKLOADS[1], frames=200)
+    run_stream(pkv, wl, seed=93, n_frames=wl.frames, check={0, 100, 199}, rows=sample_rows(wl.T, 93),
+               camera_only=True, fused=True)
