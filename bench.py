@@ -5,10 +5,11 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 1]
     python bench.py --impl reference ...   # the CPU oracle, timed on host cores
 
-One step = the whole stream: reset, then for each of the 320 frames one plan
-and 24 x (append_frame + run) through the C-ABI, with evict_frames after each
-append. Inputs come from a ring of 16 seeded frame sets already in HBM; the
-24 block pools (1.9 GB) exceed L2, so every call reads its K/V from HBM.
+One step = the whole stream: reset, then for each of the 320 frames
+kv_begin_frame, kv_evict_frames, one kv_plan and 24 x kv_run_append through
+the C-ABI (each one launch that appends the block's K/V and computes its
+attention). Inputs come from a ring of 16 seeded frame sets already in HBM;
+the 24 block pools (1.9 GB) exceed L2, so every call reads its K/V from HBM.
 With --gpus N (torchrun) each rank runs an independent replica stream (the
 path does not shard); value = frames of all ranks / max-over-ranks time.
 """
@@ -44,7 +45,8 @@ def peaks():
 
 
 TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "paged_prefill_attn_224x224_dram.txt")
-KERNEL_SOURCES = ("paged_attn.cu", "sm100.cuh", "tmem_access.cuh", "kernels.h", "kv_layout.h")
+KERNEL_SOURCES = ("paged_attn.cu", "sm100.cuh", "tmem_access.cuh", "kernels.h", "kv_layout.h", "merge.cuh",
+                  "launch.cuh")
 
 
 def kernel_source_hash():
@@ -161,8 +163,68 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ GPU arm
+class HostIO:
+    """End-to-end inputs and outputs: every frame step's Q/K/V (all blocks)
+    go from pinned host memory to one of two device staging buffers on a copy
+    stream, and its outputs from one of two device output buffers back to
+    pinned host memory on another stream. Events order each buffer's reuse,
+    so the copies of frame f+1 and f-1 run while frame f computes."""
+
+    def __init__(self, runner):
+        torch = runner.torch
+        self.torch = torch
+        self.hring = runner.ring.cpu().pin_memory()                 # [R, B, 3, rows, H, D]
+        self.hout = torch.empty((runner.ring_n,) + tuple(runner.out.shape), dtype=runner.out.dtype).pin_memory()
+        self.stage = [torch.empty_like(runner.ring[0]) for _ in range(2)]
+        self.outb = [torch.empty_like(runner.out) for _ in range(2)]
+        self.ptr = [[[st[b, i].data_ptr() for i in range(3)] for b in range(st.shape[0])] for st in self.stage]
+        self.optr = [[o[b].data_ptr() for b in range(o.shape[0])] for o in self.outb]
+        self.h2d = torch.cuda.Stream()
+        self.d2h = torch.cuda.Stream()
+        ev = lambda: [torch.cuda.Event() for _ in range(2)]
+        self.copied, self.computed, self.drained = ev(), ev(), ev()
+        self.used = [False, False]
+        self.h2d_bytes = self.stage[0].numel() * self.stage[0].element_size()   # per frame step
+        self.d2h_bytes = self.outb[0].numel() * self.outb[0].element_size()
+
+    def begin_pass(self, compute):
+        start = self.torch.cuda.Event()
+        start.record(compute)
+        self.h2d.wait_event(start)
+        self.d2h.wait_event(start)
+        self.used = [False, False]
+
+    def inputs(self, f, r, compute):
+        i = f % 2
+        if self.used[i]:
+            self.h2d.wait_event(self.computed[i])    # frame f-2 has read stage i
+        with self.torch.cuda.stream(self.h2d):
+            self.stage[i].copy_(self.hring[r], non_blocking=True)
+            self.copied[i].record(self.h2d)
+        compute.wait_event(self.copied[i])
+        if self.used[i]:
+            compute.wait_event(self.drained[i])      # frame f-2's outputs are back on the host
+        return self.ptr[i], self.optr[i]
+
+    def outputs(self, f, r, compute):
+        i = f % 2
+        self.computed[i].record(compute)
+        self.d2h.wait_event(self.computed[i])
+        with self.torch.cuda.stream(self.d2h):
+            self.hout[r].copy_(self.outb[i], non_blocking=True)
+            self.drained[i].record(self.d2h)
+        self.used[i] = True
+
+    def end_pass(self, compute):
+        compute.wait_stream(self.h2d)
+        compute.wait_stream(self.d2h)
+
+
 class StreamRunner:
-    """One replica of the workload's stream on the current GPU."""
+    """One replica of the workload's stream on the current GPU. A frame step
+    is kv_begin_frame, kv_evict_frames, kv_plan, then kv_run_append for every
+    block (one launch that appends the block's K/V and computes its
+    attention), and the keyframe decision when frames are deferred."""
 
     def __init__(self, wl, seed, ring=16):
         import torch
@@ -178,19 +240,18 @@ class StreamRunner:
                                       cross_frame_special=wl.cross_special)
         self.cache.allocate_pools("cuda")
         self.h = self.cache.handle
+        self.cache_arr = (ctypes.c_void_p * 1)(self.h)
         self.ws = torch.empty(pkv.workspace_bytes([self.cache]), dtype=torch.uint8, device="cuda")
         self.ring = workload.qkv_ring_cuda(wl, seed, ring)            # [R, B, 3, T, H, D]
         self.out = torch.empty((wl.blocks, wl.T, wl.H, wl.D), dtype=wl.torch_dtype(), device="cuda")
         self.keep = workload.keyframe_mask(wl, seed)
         self.defer = wl.keyframes != "all"
-        elt = self.ring.element_size()
         self.ptr = [[[self.ring[r, b, i].data_ptr() for i in range(3)] for b in range(wl.blocks)]
                     for r in range(ring)]
         self.optr = [self.out[b].data_ptr() for b in range(wl.blocks)]
         self.ws_ptr, self.ws_bytes = self.ws.data_ptr(), self.ws.numel()
-        self.stats = []          # per frame: (lkv, splits)
-        self.launches = 0
-        self._elt = elt
+        self.lkv = []            # per frame step of the last pass: visible tokens
+        self.fused = []          # per frame step: the plan merged its splits in-kernel
 
     frames_per_pass = property(lambda self: self.wl.frames)
     steps_per_pass = property(lambda self: self.wl.frames)
@@ -199,68 +260,53 @@ class StreamRunner:
         if rc != 0:
             raise self.capi.KVError(rc, what, self.L.kv_last_error().decode())
 
-    def one_pass(self, events=None, host=None):
-        """One pass over the stream. events: list to receive (start, end)
-        event pairs around every kv_run. host: (pinned ring, pinned out, dev
-        staging) for the end-to-end variant that copies inputs in and outputs
-        out every frame."""
-        torch, L, wl, h, sp = self.torch, self.L, self.wl, self.h, self.sp
+    def one_pass(self, io=None):
+        """One pass over the stream; returns the library's kernel launches.
+        io: a HostIO for the end-to-end variant."""
+        L, wl, h, sp = self.L, self.wl, self.h, self.sp
         self._chk(L.kv_reset(h), "kv_reset")
         plan = ctypes.c_void_p()
-        cache_arr = (ctypes.c_void_p * 1)(h)
-        self.stats = []
+        st = self.capi.kv_plan_stats()
+        self.lkv, self.fused = [], []
         launches = 0
+        if io is not None:
+            io.begin_pass(self.stream)
         for f in range(wl.frames):
             r = f % self.ring_n
-            if host is not None:
-                hring, hout, dstage = host
-                dstage.copy_(hring[r], non_blocking=True)
-                ptr = [[dstage[b, i].data_ptr() for i in range(3)] for b in range(wl.blocks)]
-            else:
-                ptr = self.ptr[r]
+            ptr, optr = io.inputs(f, r, self.stream) if io is not None else (self.ptr[r], self.optr)
             if self.defer:
                 self._chk(L.kv_defer_eviction(h, 1), "defer")
+            self._chk(L.kv_begin_frame(h), "begin_frame")
+            self._chk(L.kv_evict_frames(h), "evict")
+            if plan.value:
+                L.kv_plan_free(plan)
+            self._chk(L.kv_plan(ctypes.byref(plan), self.cache_arr, 1, 0, self.ws_ptr, self.ws_bytes, sp), "plan")
+            L.kv_plan_get_stats(plan, ctypes.byref(st))
+            launches += st.upload_launches + wl.blocks * st.run_launches
+            self.lkv.append(st.visible_tokens)
+            self.fused.append(st.fused_merge)
             for b in range(wl.blocks):
                 q, k, v = ptr[b]
-                self._chk(L.kv_append_frame(h, b, k, v, sp), "append")
-                launches += 1
-                if b == 0:
-                    self._chk(L.kv_evict_frames(h), "evict")
-                    if plan.value:
-                        L.kv_plan_free(plan)
-                    self._chk(L.kv_plan(ctypes.byref(plan), cache_arr, 1, 0, self.ws_ptr, self.ws_bytes, sp),
-                              "plan")
-                    st = self.capi.kv_plan_stats()
-                    L.kv_plan_get_stats(plan, ctypes.byref(st))
-                    launches += 1
-                    self.stats.append((st.visible_tokens, st.n_split_units))
-                if events is not None:
-                    e0 = torch.cuda.Event(enable_timing=True)
-                    e1 = torch.cuda.Event(enable_timing=True)
-                    e0.record(self.stream)
-                self._chk(L.kv_run(plan, b, q, self.optr[b], sp), "run")
-                launches += 1 + (1 if self.stats[-1][1] else 0)
-                if events is not None:
-                    e1.record(self.stream)
-                    events.append((e0, e1))
+                self._chk(L.kv_run_append(plan, b, k, v, q, optr[b], sp), "run_append")
             if self.defer:
                 if self.keep[f]:
                     self._chk(L.kv_commit_frame(h), "commit")
                 else:
                     self._chk(L.kv_rollback_last_frame(h), "rollback")
-            if host is not None:
-                hout[r].copy_(self.out, non_blocking=True)
+            if io is not None:
+                io.outputs(f, r, self.stream)
         if plan.value:
             L.kv_plan_free(plan)
-        self.launches = launches
+        if io is not None:
+            io.end_pass(self.stream)
         return launches
 
 
 class BatchRunner:
     """Several streams of different ages planned together (one kv_plan over
     all caches per frame step, their query rows concatenated), as in the
-    batched workload. A pass is `steps` frame steps of every stream; the
-    streams keep growing from pass to pass."""
+    batched workload, sharing one pool per block. A pass is `steps` frame
+    steps of every stream; the streams keep growing from pass to pass."""
 
     def __init__(self, wl, seed, steps, passes, ring=4):
         import torch
@@ -274,23 +320,23 @@ class BatchRunner:
         self.ages = workload.stream_ages(wl, seed)
         span = int(self.ages.max()) + steps * passes
         sp_pages = max(1, math.ceil(wl.NS * span / wl.page_size))
-        self.caches = [pkv.PagedKVCache(wl.patch_pages + sp_pages, wl.page_size, wl.H, wl.D, wl.S, wl.W,
-                                        num_blocks=wl.blocks, num_special=wl.NS, dtype=wl.dtype)
-                       for _ in range(wl.streams)]
-        for c in self.caches:
-            c.allocate_pools("cuda")
+        # one pool per block for all the streams (kv_init_group): common patch
+        # pages, a special-page range per stream
+        patch = wl.streams * wl.patch_pages
+        self.caches = pkv.PagedKVCache.group(wl.streams, patch + wl.streams * sp_pages, wl.page_size, wl.H, wl.D,
+                                             wl.S, wl.W, num_blocks=wl.blocks, num_special=wl.NS, dtype=wl.dtype,
+                                             patch_pages=patch, special_pages=sp_pages)
+        self.caches[0].allocate_pools("cuda")
         self.h = [c.handle for c in self.caches]
         self.cache_arr = (ctypes.c_void_p * wl.streams)(*self.h)
         self.ws = torch.empty(pkv.workspace_bytes(self.caches), dtype=torch.uint8, device="cuda")
         self.ring = workload.qkv_ring_cuda(wl, seed, ring)            # [R, B, 3, streams*T, H, D]
         self.out = torch.empty((wl.blocks, wl.streams * wl.T, wl.H, wl.D), dtype=wl.torch_dtype(), device="cuda")
-        row = wl.T * wl.H * wl.D * self.ring.element_size()
         self.ptr = [[[self.ring[r, b, i].data_ptr() for i in range(3)] for b in range(wl.blocks)]
                     for r in range(ring)]
-        self.row = row
         self.optr = [self.out[b].data_ptr() for b in range(wl.blocks)]
         self.ws_ptr, self.ws_bytes = self.ws.data_ptr(), self.ws.numel()
-        self.stats = []
+        self.lkv, self.fused = [], []
         # warm every stream to its age: page state only (metadata appends)
         # (a frame step closes once every block has been appended)
         for h, age in zip(self.h, self.ages):
@@ -306,49 +352,45 @@ class BatchRunner:
         if rc != 0:
             raise self.capi.KVError(rc, what, self.L.kv_last_error().decode())
 
-    def one_pass(self, events=None, host=None):
-        torch, L, wl, sp = self.torch, self.L, self.wl, self.sp
+    def one_pass(self, io=None):
+        L, wl, sp = self.L, self.wl, self.sp
         plan = ctypes.c_void_p()
-        self.stats = []
+        st = self.capi.kv_plan_stats()
+        self.lkv, self.fused = [], []
         launches = 0
+        if io is not None:
+            io.begin_pass(self.stream)
         for f in range(self.steps):
             r = f % self.ring_n
-            if host is not None:
-                hring, hout, dstage = host
-                dstage.copy_(hring[r], non_blocking=True)
-                ptr = [[dstage[b, i].data_ptr() for i in range(3)] for b in range(wl.blocks)]
-            else:
-                ptr = self.ptr[r]
+            ptr, optr = io.inputs(f, r, self.stream) if io is not None else (self.ptr[r], self.optr)
+            for h in self.h:
+                self._chk(L.kv_begin_frame(h), "begin_frame")
+                self._chk(L.kv_evict_frames(h), "evict")
+            if plan.value:
+                L.kv_plan_free(plan)
+            self._chk(L.kv_plan(ctypes.byref(plan), self.cache_arr, wl.streams, 0, self.ws_ptr,
+                                self.ws_bytes, sp), "plan")
+            L.kv_plan_get_stats(plan, ctypes.byref(st))
+            launches += st.upload_launches + wl.blocks * st.run_launches
+            self.lkv.append(st.visible_tokens)
+            self.fused.append(st.fused_merge)
             for b in range(wl.blocks):
                 q, k, v = ptr[b]
-                for si, h in enumerate(self.h):
-                    self._chk(L.kv_append_frame(h, b, k + si * self.row, v + si * self.row, sp), "append")
-                    launches += 1
-                if b == 0:
-                    for h in self.h:
-                        self._chk(L.kv_evict_frames(h), "evict")
-                    if plan.value:
-                        L.kv_plan_free(plan)
-                    self._chk(L.kv_plan(ctypes.byref(plan), self.cache_arr, wl.streams, 0, self.ws_ptr,
-                                        self.ws_bytes, sp), "plan")
-                    st = self.capi.kv_plan_stats()
-                    L.kv_plan_get_stats(plan, ctypes.byref(st))
-                    launches += 1
-                    self.stats.append((st.visible_tokens, st.n_split_units))
-                if events is not None:
-                    e0 = torch.cuda.Event(enable_timing=True)
-                    e1 = torch.cuda.Event(enable_timing=True)
-                    e0.record(self.stream)
-                self._chk(L.kv_run(plan, b, q, self.optr[b], sp), "run")
-                launches += 1 + (1 if self.stats[-1][1] else 0)
-                if events is not None:
-                    e1.record(self.stream)
-                    events.append((e0, e1))
-            if host is not None:
-                hout[r].copy_(self.out, non_blocking=True)
+                self._chk(L.kv_run_append(plan, b, k, v, q, optr[b], sp), "run_append")
+            if io is not None:
+                io.outputs(f, r, self.stream)
         if plan.value:
             L.kv_plan_free(plan)
+        if io is not None:
+            io.end_pass(self.stream)
         return launches
+
+
+def roofline_ms(wl, lkvs, peak_tf, hbm_gbs):
+    """Sum over one pass of each attention call's roofline time
+    max(FLOPs / tensor peak, K/V bytes / HBM bandwidth), in ms."""
+    return sum(max(call_flops(wl.T, l, wl.H, wl.D) / (peak_tf * 1e12),
+                   call_kv_bytes(l, wl.H, wl.D) / (hbm_gbs * 1e9)) for l in lkvs) * wl.blocks * 1e3
 
 
 def run_gpu(args):
@@ -384,8 +426,10 @@ def run_gpu(args):
         runner.one_pass()
     torch.cuda.synchronize()
 
-    # ---- timed region: K passes over the stream, inputs resident in HBM
-    events = []
+    # ---- timed region: K passes over the stream, inputs resident in HBM.
+    # Nothing but the library's kernels runs on the stream inside it (one plan
+    # upload per frame step, one kernel per block), so the region's time is
+    # also the attention kernels' time, launch gaps included.
     barrier()
     torch.cuda.synchronize()
     clocks = ClockSampler(local)
@@ -399,40 +443,25 @@ def run_gpu(args):
         t1.record()
         torch.cuda.synchronize()
     barrier()
-    # One more pass, outside the timed region, with events around every
-    # kv_run (attention + merge): the per-call kernel time for the roofline.
-    # (Events between launches would break the launch overlap of the timed
-    # passes, so they are recorded only here.)
-    runner.one_pass(events=events)
-    torch.cuda.synchronize()
     ms_max = max_over_ranks(t0.elapsed_time(t1), world, "cuda")
-    frames_total = args.steps * runner.frames_per_pass * world
     value = whole_job_rate(args.steps * runner.frames_per_pass, world, ms_max)
+    ms_pass = ms_max / args.steps
 
-    # per-call attention time (run = attention + merge) against the roofline
-    run_ms = [a.elapsed_time(b) for a, b in events]
-    per_pass = len(run_ms)
-    lkvs = [s[0] for s in runner.stats]                 # per frame of the last pass
+    lkvs = list(runner.lkv)                            # per frame step of the last pass
     flops = sum(call_flops(wl.T, l, wl.H, wl.D) for l in lkvs) * wl.blocks
     kvbytes = sum(call_kv_bytes(l, wl.H, wl.D) for l in lkvs) * wl.blocks
-    run_s = sum(run_ms[-per_pass:]) / 1e3
     pk, pk_kind = peaks()
-    tflops = flops / run_s / 1e12
-    gbs = kvbytes / run_s / 1e9
-    # The attention kernel runs inside a seconds-long stream of calls, so the
-    # denominator is the sustained (power-capped) dense bf16 rate.
-    peak_tf = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
-    t_roof = sum(max(call_flops(wl.T, l, wl.H, wl.D) / (peak_tf * 1e12),
-                     call_kv_bytes(l, wl.H, wl.D) / (pk["hbm_gbs"] * 1e9)) for l in lkvs) * wl.blocks
-    roof_frac = t_roof / run_s
+    burst_tf = pk["bf16_tflops"]
+    sust_tf = pk.get("bf16_tflops_sustained", burst_tf)
+    tflops = flops / (ms_pass / 1e3) / 1e12
+    roof_sust = roofline_ms(wl, lkvs, sust_tf, pk["hbm_gbs"])
+    roof_burst = roofline_ms(wl, lkvs, burst_tf, pk["hbm_gbs"])
 
-    # ---- end to end: host (pinned) inputs copied in, outputs copied out, every frame
+    # ---- end to end: host (pinned) inputs copied in, outputs copied out, every frame step
     e2e = None
     if not args.no_e2e:
-        hring = runner.ring.cpu().pin_memory()
-        hout = torch.empty((runner.ring_n,) + tuple(runner.out.shape), dtype=runner.out.dtype).pin_memory()
-        dstage = torch.empty_like(runner.ring[0])
-        runner.one_pass(host=(hring, hout, dstage))
+        io = HostIO(runner)
+        runner.one_pass(io=io)
         torch.cuda.synchronize()
         barrier()
         torch.cuda.synchronize()
@@ -440,54 +469,51 @@ def run_gpu(args):
         b = torch.cuda.Event(enable_timing=True)
         a.record()
         for _ in range(args.steps):
-            runner.one_pass(host=(hring, hout, dstage))
+            runner.one_pass(io=io)
         b.record()
         torch.cuda.synchronize()
         barrier()
         ems = max_over_ranks(a.elapsed_time(b), world, "cuda")
         e2e = {"value": whole_job_rate(args.steps * runner.frames_per_pass, world, ems), "unit": "frames/s",
-               "h2d_bytes_per_step": int(dstage.numel() * dstage.element_size() * runner.steps_per_pass),
-               "d2h_bytes_per_step": int(runner.out.numel() * runner.out.element_size() * runner.steps_per_pass)}
+               "h2d_bytes_per_step": int(io.h2d_bytes * runner.steps_per_pass),
+               "d2h_bytes_per_step": int(io.d2h_bytes * runner.steps_per_pass),
+               "copies": "per frame step: H2D on a copy stream, D2H on another, double-buffered"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and wl.streams == 1:
-        cpu = cpu_baseline(wl, args.seed, budget_s=args.cpu_budget,
-                           frames_sample=tuple(sorted({0, min(71, wl.frames - 1), wl.frames // 2, wl.frames - 1})))
-
-    # steady state: frame steps whose window is full (more than S + W frames)
-    steady = [i for i in range(len(lkvs)) if i >= wl.S + wl.W] if wl.streams == 1 else list(range(len(lkvs)))
-    if steady:
-        st_ms = sum(run_ms[i * wl.blocks + b] for i in steady for b in range(wl.blocks))
-        st_fl = sum(call_flops(wl.T, lkvs[i], wl.H, wl.D) for i in steady) * wl.blocks
-        steady_tflops = st_fl / (st_ms / 1e3) / 1e12
-    else:
-        steady_tflops = None
+        cpu = cpu_baseline(wl, args.seed, budget_s=args.cpu_budget, frames_sample=oracle_sample_frames(wl))
 
     if rank == 0:
         metric = metric_name(args.workload, wl)
         config = arm_config(wl, world, args.seed)
         if wl.streams > 1:
             assert config["stream_ages"] == [int(x) for x in runner.ages]
+        kernel_ms = ms_pass   # per pass: all library kernels of the timed region
         line = {
             "metric": metric,
             "profiling_case_not_a_bench_value": profiling_case or None,
             "value": round(value, 2), "unit": "frames/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 3),
+            "warmup": args.warmup, "ms_per_step": round(ms_pass, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
             "data": f"synthetic (seeded N(0,1) Q/K/V, ring of {runner.ring_n} frame sets in HBM)",
             "config": config,
-            "attention": {"tflops": round(tflops, 2), "kv_gbs": round(gbs, 1),
-                          "roofline_frac": round(roof_frac, 4),
-                          "frac_of_burst_peak": round(tflops / pk["bf16_tflops"], 4),
-                          "steady_state_tflops": round(steady_tflops, 2) if steady_tflops else None,
-                          "roofline_ms_per_pass": round(t_roof * 1e3, 3),
-                          "run_ms_per_pass": round(run_s * 1e3, 3)},
+            "attention": {"tflops": round(tflops, 2), "kv_gbs": round(kvbytes / (kernel_ms / 1e3) / 1e9, 1),
+                          "frac_of_sustained_roofline": round(roof_sust / kernel_ms, 4),
+                          "frac_of_burst_roofline": round(roof_burst / kernel_ms, 4),
+                          "roofline_ms_per_pass_sustained": round(roof_sust, 3),
+                          "roofline_ms_per_pass_burst": round(roof_burst, 3),
+                          "kernel_ms_per_pass": round(kernel_ms, 3),
+                          "fused_merge_steps": int(sum(runner.fused)),
+                          "steps_per_pass": len(lkvs)},
             "roofline": {"bound": "tensor", "achieved": round(tflops, 2),
-                         "peak": peak_tf, "unit": "TFLOP/s",
-                         "frac": round(tflops / peak_tf, 4),
+                         "peak": sust_tf, "unit": "TFLOP/s",
+                         "frac": round(roof_sust / kernel_ms, 4),
+                         "frac_of_burst": round(roof_burst / kernel_ms, 4),
                          "traffic": measured_traffic() if args.workload == 1 else None,
-                         "peak_kind": f"{pk_kind} bf16 dense sustained (kernel timed inside a long step)",
-                         "kernel": "paged_prefill_attn + splitkv_merge (kv_run), event-timed per call in one extra pass"},
+                         "peak_kind": f"{pk_kind} bf16 dense sustained (kernel timed inside a long step); "
+                                      f"burst {burst_tf} in frac_of_burst",
+                         "kernel": "paged_prefill_attn (append + attention + split merge in one launch "
+                                   "per block) and the per-frame plan upload: the whole timed region"},
             "gpu_launches": launches,
             "clocks": clocks.summary(),
             "e2e": e2e,
@@ -539,7 +565,15 @@ def workload_config(wl, world):
             "l2": "inputs larger than L2 (one pool per block, all read every frame step)"}
 
 
-def cpu_baseline(wl, seed, budget_s=20.0, frames_sample=(0, 71, 159, 319), rows=None):
+def oracle_sample_frames(wl):
+    """The frames both arms time the oracle on: the last frame of the
+    window's ramp and the stream's last frame (0-based), all query rows of
+    block 0."""
+    n = max(1, wl.frames)
+    return tuple(sorted({min(wl.S + wl.W, n) - 1, n - 1}))
+
+
+def cpu_baseline(wl, seed, budget_s=20.0, frames_sample=(71, 319), rows=None):
     """Times the CPU oracle (float64 dense attention) on a bounded sample of
     the workload and extrapolates frames/s by FLOPs."""
     sys.path.insert(0, os.path.join(ROOT, "tests"))
@@ -564,7 +598,7 @@ def cpu_baseline(wl, seed, budget_s=20.0, frames_sample=(0, 71, 159, 319), rows=
             t = time.perf_counter()
             so.expected(sel)
             dt = time.perf_counter() - t
-            lkv = len(so.sim.patch_frames()) * wl.P + len(so.sim.visible_specials())
+            lkv = len(so.sim.attended_patch_frames()) * wl.P + len(so.sim.visible_specials())
             t_att += dt
             fl += call_flops(len(sel), lkv, wl.H, wl.D)
             done.append(f)
@@ -594,15 +628,13 @@ def run_reference(args):
         # the oracle runs one stream; a stream as old as the oldest in the batch
         import dataclasses
         wl = dataclasses.replace(wl, streams=1, frames=wl.age_hi)
-    budget = max(5.0, 150.0 / max(1, args.steps + args.warmup))
-    for _ in range(args.warmup):
-        cpu_baseline(wl, args.seed, budget_s=budget / 4, frames_sample=(0,), rows=8)
+    for _ in range(args.warmup):   # untimed: a small call to load and warm the oracle's code
+        cpu_baseline(wl, args.seed, budget_s=1.0, frames_sample=(0,), rows=8)
     t = time.perf_counter()
     vals = []
-    n = max(1, wl.frames)
-    sample = tuple(sorted({min(wl.S + wl.W - 1, n - 1), n - 1}))   # a ramp frame and the last frame
+    sample = oracle_sample_frames(wl)   # the GPU arm's cpu_baseline sample
     for _ in range(args.steps):
-        vals.append(cpu_baseline(wl, args.seed, budget_s=budget, frames_sample=sample, rows=16))
+        vals.append(cpu_baseline(wl, args.seed, budget_s=args.cpu_budget, frames_sample=sample))
     el = time.perf_counter() - t
     v = statistics.median(x["value"] for x in vals)
     line = {
