@@ -836,6 +836,7 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
     uint32_t* cnt = a.groups + 2 * u.group;
     const int n = u.n_chunks;
     if (threadIdx.x == 0) {
+      __threadfence();   // release: every thread's partials (fenced, then the barrier) before the arrival
       atomicAdd(cnt, 1u);
       int ok = 1;
       const uint64_t t0 = globaltimer_ns();

@@ -313,11 +313,12 @@ def test_failed_append_launch_leaves_state_unchanged(pkv):
 
 @pytest.mark.parametrize("H", [2, 4])
 def test_more_than_32_chunks_per_split_unit(pkv, H):
-    """One K/V tile per CTA over 53 visible tiles (48 patch pages of 64 tokens
-    and 5 special pages): 53 chunks per unit, past the merge's first 32-lane
-    pass. H = 2 gives 106 CTAs, which fit on the device at once, so the CTAs
-    merge their own groups; H = 4 gives 212, which do not, so the merge runs
-    as its own launch."""
+    """One K/V tile per CTA over 54 visible tiles (48 patch pages of 64 tokens;
+    300 special tokens on 5 pages, the open step's frame's 6 on a tile of
+    their own): 54 chunks per unit, past the merge's first 32-lane pass.
+    H = 2 gives 108 CTAs, which fit on the device at once, so the CTAs merge
+    their own groups; H = 4 gives 216, which do not, so the merge runs as its
+    own launch."""
     wl = small(64, H=H, S=8, W=40, frames=50)
     fr = Frames(wl, seed=70)
     cache = new_cache(pkv, wl)
@@ -329,7 +330,7 @@ def test_more_than_32_chunks_per_split_unit(pkv, H):
         so.begin_frame(f)
     plan = pkv.Plan([cache], workspace(pkv, [cache]), tiles_per_split=1)
     st = plan.stats()
-    assert st["tiles_per_cta"] == 1 and st["n_kv_tiles"] == 53
+    assert st["tiles_per_cta"] == 1 and st["n_kv_tiles"] == 54
     assert st["fused_merge"] == (1 if H == 2 else 0)
     for rep in range(2):   # the group counters must be back at zero for the second run
         out = plan.run(0, q)
