@@ -103,12 +103,13 @@ def workspace(pkv, caches):
 
 def run_stream(pkv, wl, seed, n_frames, check, rows=None, defer=None, keep=None,
                tiles_per_split=0, patch_pages=0, collect=None, dense=(), cross_special=True,
-               camera_only=False, fused=False):
+               camera_only=False, fused=False, all_rows=()):
     """Append frames 0..n_frames-1 of block 0; at frames in `check`, plan + run
     and compare the chosen query rows with the oracle. defer[f] / keep[f]:
     frame f is appended with eviction deferred and then committed (keep) or
     rolled back. At frames in `dense`, every row is also checked against the
-    fp32 dense gather of the visible pages. fused: each frame goes through
+    fp32 dense gather of the visible pages; at frames in `all_rows` every row
+    is checked against the oracle whatever `rows` says. fused: each frame goes through
     begin_frame + plan + run_append (the append inside the attention launch)
     instead of append_frame + plan + run. Returns {frame: (max_err, mean_err)}."""
     fr = Frames(wl, seed)
@@ -135,8 +136,9 @@ def run_stream(pkv, wl, seed, n_frames, check, rows=None, defer=None, keep=None,
                 plan = pkv.Plan([cache], ws, tiles_per_split=tiles_per_split)
                 out = plan.run(0, q)
             plan.check_device()
-            sel = slice(None) if rows is None else torch.as_tensor(rows)
-            res[f] = assert_close(out[sel], so.expected(rows), f"frame {f}")
+            r = None if f in all_rows else rows
+            sel = slice(None) if r is None else torch.as_tensor(r)
+            res[f] = assert_close(out[sel], so.expected(r), f"frame {f}")
             if f in dense:
                 want = dense_fp32(cache, plan, 0, q, so, patch_pages or wl.patch_pages)
                 assert_close_dense(out, want, f"frame {f} (all rows, fp32 dense)")

@@ -223,9 +223,20 @@ def test_include_scale_frames_off_is_zero_scale_frames(pkv):
 
 
 def test_full_224_stream_block0_sampled(pkv):
+    """Every row of the last frame against the oracle (and the fp32 gather),
+    sampled rows elsewhere."""
     wl = workload.WORKLOADS[1]
     run_stream(pkv, wl, seed=1, n_frames=wl.frames, check={0, 71, 72, 159, 319},
-               rows=sample_rows(wl.T, 1), dense={72, 319})
+               rows=sample_rows(wl.T, 1), dense={72, 319}, all_rows={319})
+
+
+def test_full_224_stream_fused_all_rows(pkv):
+    """The fused frame step (begin_frame + run_append) over the whole stream:
+    every row against the oracle at the end of the window's ramp and at the
+    last frame."""
+    wl = workload.WORKLOADS[1]
+    run_stream(pkv, wl, seed=6, n_frames=wl.frames, check={71, 200, 319}, rows=sample_rows(wl.T, 6),
+               fused=True, all_rows={71, 319})
 
 
 def test_full_224_keyframes_block0_sampled(pkv):
@@ -238,7 +249,7 @@ def test_full_224_keyframes_block0_sampled(pkv):
 def test_full_518x378_stream_block0_sampled(pkv):
     wl = workload.WORKLOADS[3]
     run_stream(pkv, wl, seed=3, n_frames=wl.frames, check={0, 499, 999},
-               rows=sample_rows(wl.T, 3, n=12), dense={999})
+               rows=sample_rows(wl.T, 3, n=12), dense={999}, fused=True)
 
 
 def test_full_batched_ragged_sampled(pkv):
@@ -262,9 +273,12 @@ def test_full_batched_ragged_sampled(pkv):
     out = plan.run(0, torch.cat(qs).cuda())
     plan.check_device()
     rows = sample_rows(wl.T, 4, n=8)
+    full = {int(np.argmax(ages)), int(np.argmin(ages))}   # every row of the oldest and youngest stream
     for s, so in enumerate(oracles):
-        got = out[s * wl.T:(s + 1) * wl.T][torch.as_tensor(rows)]
-        assert_close(got, so.expected(rows), f"stream {s} age {ages[s]}")
+        r = None if s in full else rows
+        got = out[s * wl.T:(s + 1) * wl.T]
+        got = got if r is None else got[torch.as_tensor(r)]
+        assert_close(got, so.expected(r), f"stream {s} age {ages[s]}")
 
 
 def test_failed_append_launch_leaves_state_unchanged(pkv):
