@@ -262,7 +262,11 @@ class StreamRunner:
 
     def one_pass(self, io=None):
         """One pass over the stream; returns the library's kernel launches.
-        io: a HostIO for the end-to-end variant."""
+        io: a HostIO for the end-to-end variant. With self.pages_calls each
+        block runs the pages' two calls, kv_append_frame then kv_run (a
+        scatter launch and an attention launch), instead of kv_run_append."""
+        if getattr(self, "pages_calls", False):
+            return self.one_pass_pages(io)
         L, wl, h, sp = self.L, self.wl, self.h, self.sp
         self._chk(L.kv_reset(h), "kv_reset")
         plan = ctypes.c_void_p()
@@ -288,6 +292,48 @@ class StreamRunner:
             for b in range(wl.blocks):
                 q, k, v = ptr[b]
                 self._chk(L.kv_run_append(plan, b, k, v, q, optr[b], sp), "run_append")
+            if self.defer:
+                if self.keep[f]:
+                    self._chk(L.kv_commit_frame(h), "commit")
+                else:
+                    self._chk(L.kv_rollback_last_frame(h), "rollback")
+            if io is not None:
+                io.outputs(f, r, self.stream)
+        if plan.value:
+            L.kv_plan_free(plan)
+        if io is not None:
+            io.end_pass(self.stream)
+        return launches
+
+
+    def one_pass_pages(self, io=None):
+        L, wl, h, sp = self.L, self.wl, self.h, self.sp
+        self._chk(L.kv_reset(h), "kv_reset")
+        plan = ctypes.c_void_p()
+        st = self.capi.kv_plan_stats()
+        self.lkv, self.fused = [], []
+        launches = 0
+        if io is not None:
+            io.begin_pass(self.stream)
+        for f in range(wl.frames):
+            r = f % self.ring_n
+            ptr, optr = io.inputs(f, r, self.stream) if io is not None else (self.ptr[r], self.optr)
+            if self.defer:
+                self._chk(L.kv_defer_eviction(h, 1), "defer")
+            for b in range(wl.blocks):
+                q, k, v = ptr[b]
+                self._chk(L.kv_append_frame(h, b, k, v, sp), "append")
+                if b == 0:
+                    self._chk(L.kv_evict_frames(h), "evict")
+                    if plan.value:
+                        L.kv_plan_free(plan)
+                    self._chk(L.kv_plan(ctypes.byref(plan), self.cache_arr, 1, 0, self.ws_ptr, self.ws_bytes, sp),
+                              "plan")
+                    L.kv_plan_get_stats(plan, ctypes.byref(st))
+                    launches += st.upload_launches + wl.blocks * (1 + st.run_launches)
+                    self.lkv.append(st.visible_tokens)
+                    self.fused.append(st.fused_merge)
+                self._chk(L.kv_run(plan, b, q, optr[b], sp), "run")
             if self.defer:
                 if self.keep[f]:
                     self._chk(L.kv_commit_frame(h), "commit")
@@ -416,6 +462,7 @@ def run_gpu(args):
                              passes=args.warmup + 2 * args.steps + 3)
     else:
         runner = StreamRunner(wl, seed=replica_seed(args.seed, rank))
+        runner.pages_calls = args.calls == "pages"
     torch.cuda.synchronize()
 
     def barrier():
@@ -486,6 +533,8 @@ def run_gpu(args):
     if rank == 0:
         metric = metric_name(args.workload, wl)
         config = arm_config(wl, world, args.seed)
+        if args.calls != "fused":
+            config["calls"] = "kv_append_frame + kv_run"
         if wl.streams > 1:
             assert config["stream_ages"] == [int(x) for x in runner.ages]
         kernel_ms = ms_pass   # per pass: all library kernels of the timed region
@@ -658,6 +707,8 @@ def main():
     ap.add_argument("--workload", type=int, default=1, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--seed", type=int, default=1)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--calls", default="fused", choices=["fused", "pages"],
+                    help="per block: kv_run_append (fused) or the pages' kv_append_frame + kv_run")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)

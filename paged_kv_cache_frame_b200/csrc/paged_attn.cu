@@ -276,7 +276,9 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
     const long long per_kv = (long long)T * rv, per_req = 2 * per_kv;
     const long long total = per_req * a.n_reqs;
     const long long i0 = total * blockIdx.x / gridDim.x, i1 = total * (blockIdx.x + 1) / gridDim.x;
-    for (long long i = i0 + threadIdx.x; i < i1; i += 256) {
+    // vector i of the flattened [request][K/V][token][row vector] space: its
+    // source in k/v and its destination in the pool
+    auto locate = [&](long long i, const uint4** src, uint4** dst) {
       const int r = (int)(i / per_req);
       const long long rem = i - (long long)r * per_req;
       const int kv = rem >= per_kv;
@@ -293,9 +295,27 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
         page = q.cur_page;
         slot = tok - q.NS;
       }
-      const uint4* src = static_cast<const uint4*>(kv ? a.v : a.k) + (long long)(q.q_row0 + tok) * rv + c;
-      uint4* dst = static_cast<uint4*>(a.pools[r]) + (((long long)page * 2 + kv) * q.page_size + slot) * rv + c;
-      *dst = __ldg(src);
+      *src = static_cast<const uint4*>(kv ? a.v : a.k) + (long long)(q.q_row0 + tok) * rv + c;
+      *dst = static_cast<uint4*>(a.pools[r]) + (((long long)page * 2 + kv) * q.page_size + slot) * rv + c;
+    };
+    // a batch of loads in flight before their stores (the loop would
+    // otherwise wait a full memory round trip per vector)
+    constexpr int kBatch = 4;
+    for (long long i = i0 + threadIdx.x; i < i1; i += kBatch * 256) {
+      uint4 x[kBatch];
+      uint4* dst[kBatch];
+#pragma unroll
+      for (int b = 0; b < kBatch; ++b) {
+        const long long ib = i + (long long)b * 256;
+        if (ib < i1) {
+          const uint4* src;
+          locate(ib, &src, &dst[b]);
+          x[b] = __ldg(src);
+        }
+      }
+#pragma unroll
+      for (int b = 0; b < kBatch; ++b)
+        if (i + (long long)b * 256 < i1) *dst[b] = x[b];
     }
   }
 
