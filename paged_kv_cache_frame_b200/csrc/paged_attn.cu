@@ -15,38 +15,39 @@
 //   warps 0-3, 4-7   softmax warpgroups, one per 128-row query tile. Thread i
 //                    owns query row i == TMEM lane i. Per K/V tile it reads its
 //                    S row in two 64-column halves, keeps the running max/sum
-//                    in the log2 domain, writes P (16-bit) over the S columns
-//                    it has read, and rescales its O row when the running max
-//                    grows by more than 2^8 (lazy rescale: between rescales P
-//                    may exceed 1, which the final division by the same sum
-//                    cancels).
-//   producer         warp 9: TMA loads, the
-//                    query tiles once, then K/V tiles of the page table into a
-//                    STAGES-deep ring. A tile is 128 pool rows of one head, one
-//                    3-D box load per 64 columns; the tile table gives each
-//                    tile's row, so pages need not be contiguous.
-//   MMA issuer       warp 11, also the TMEM allocator (tcgen05 kind::f16,
-//                    fp32 accumulators in TMEM): S = Q_t K^T (M=128, N=128,
-//                    K=D) and O_t += P V (M=128, N=D, K=128, P read from TMEM).
-//   tail             warps 8 and 10: the unit's last query tile
-//                    of at most 16 rows (262 = 2 x 128 + 6 tokens per frame).
-//                    An M = 128 tensor-core tile would be almost all padding,
-//                    so each of these warps computes the tail's scores and
-//                    output for 64 of every K/V tile's 128 rows with warp-level
-//                    mma.sync m16n8k16, transposed so that the tail rows fill
-//                    the N = 8 side, reading K and V straight from the
-//                    shared-memory ring, with its own running max/sum and O in
-//                    registers. The two partial results are merged at the end.
+//                    in the log2 domain, writes P (16-bit) to TMEM, and
+//                    rescales its O row when the running max grows by more
+//                    than 2^8 (lazy rescale: between rescales P may exceed 1,
+//                    which the final division by the same sum cancels).
+//   tail             warps 8 and 9: the unit's last query tile of at most 16
+//                    rows (262 = 2 x 128 + 6 tokens per frame). An M = 128
+//                    tensor-core tile would be almost all padding, so each of
+//                    these warps computes the tail's scores and output for 64
+//                    of every K/V tile's 128 rows with warp-level mma.sync
+//                    m16n8k16, transposed so that the tail rows fill the N = 8
+//                    side, reading K and V straight from the shared-memory
+//                    ring, with its own running max/sum and O in registers.
+//                    The two partial results are merged at the end.
+//   producer         warp 10: TMA loads, the query tiles once, then K/V tiles
+//                    of the page table into a STAGES-deep ring. A tile is 128
+//                    pool rows of one head, one 3-D box load per 64 columns;
+//                    the tile table gives each tile's row, so pages need not be
+//                    contiguous.
+//   MMA issuer       warp 11, also the TMEM allocator (tcgen05 kind::f16, fp32
+//                    accumulators in TMEM): S = Q_t K^T (M=128, N=128, K=D) and
+//                    O_t += P V (M=128, N=D, K=128, P read from TMEM). The
+//                    whole warp runs the loop and one elected lane issues, so
+//                    the descriptors stay warp-uniform.
 //
 // Schedule. Score tiles are numbered n = j * nq + t (K/V tile j, query tile t
 // of nq). S_n goes to TMEM buffer n % NB and its P is written over it. NB is 3
 // for head_dim 64 with two query tiles (3 x 128 columns and two 64-column O
-// tiles fill the 512 columns), else 2. The tensor pipe executes a CTA's MMAs
-// in issue order, so S_n may be issued as soon as PV_{n-NB}, the last reader
-// of its buffer, has been issued: the scores of the next tiles are computed
-// while the softmax works on the current one, and the softmax never waits for
-// a PV before it stores P. Both kinds of MMA are issued in order of n, which
-// gives the two facts the waits below rely on:
+// tiles fill the 512 columns), else 2. The issuer's order is fixed: S_0 ..
+// S_{NB-1}, then PV_n followed by S_{n+NB}. A CTA's MMAs from one thread run
+// in issue order, so S_{n+NB} cannot overwrite P_n before PV_n has read it,
+// the scores of the next tiles are computed while the softmax works on the
+// current one, and the softmax never waits for a PV before it stores P. The
+// order gives the two facts the waits below rely on:
 //   - once S_n has completed, every PV_m with m <= n - NB has completed; as
 //     NB <= 2 nq, the O rescale at K/V tile j (after S_t(j) was read) waits
 //     only for PV_t(j-1), because PV_t(j-2) is complete already;
@@ -70,13 +71,15 @@
 namespace pkv {
 
 constexpr int kMaxSmemTiles = 512;   // tile descriptors cached in shared memory
+constexpr int kL2Ahead = 4;          // K/V tiles prefetched into L2 beyond the shared-memory ring
 
 template <int D>
 struct AttnRoles {
-  // warps 8 and 10 are the tail (with the softmax warpgroups, three warps
-  // per SM sub-partition), 9 the producer, 11 the MMA issuer
-  static constexpr int kTailWarps = 2;   // each takes 64 of a K/V tile's 128 columns
-  static constexpr int kProducer = 9, kMma = 11;
+  // warps 8 and 9 are the tail (with the softmax warpgroups, three warps on
+  // each SM sub-partition), 10 the producer, 11 the MMA issuer and TMEM
+  // allocator
+  static constexpr int kTailWarps = 2, kTail0 = 8;
+  static constexpr int kProducer = 10, kMma = 11;
   static constexpr int kWarps = 12;
   static constexpr int kThreads = 32 * kWarps;
 };
@@ -97,13 +100,15 @@ struct AttnSmem {
   static constexpr int kAlloc = kBytes + 1024;      // slack to align the base to 1 KB
 };
 
-// TMEM columns: the S/P buffers (128 columns each) from column 0, then O_0, O_1.
+// TMEM columns: the score buffers (128 columns each, P written over S) from
+// column 0, then O_0, O_1. head_dim 64: three buffers, O_t at 384 + 64 t;
+// head_dim 128: two, O_t at 256 + 128 t.
 template <int D>
 struct AttnTmem {
   static constexpr int kMaxBufs = D == 64 ? 3 : 2;
-  __host__ __device__ static constexpr uint32_t buf(int b) { return 128u * b; }
-  __host__ __device__ static constexpr uint32_t O(int t) { return 128u * kMaxBufs + (uint32_t)D * t; }
-  static_assert(128 * kMaxBufs + 2 * D <= 512, "TMEM budget");
+  __host__ __device__ static constexpr uint32_t S(int b) { return 128u * b; }
+  __host__ __device__ static constexpr uint32_t O(int t) { return (D == 64 ? 384u : 256u) + (uint32_t)D * t; }
+  static_assert((D == 64 ? 384 : 256) + 2 * D <= 512, "TMEM budget");
 };
 
 constexpr uint32_t kTmemCols = 512;
@@ -187,13 +192,13 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
   const int tail_rows = u.tail_rows;
   const bool has_tail = tail_rows > 0;
   const KvTile* tiles_g = a.tiles + u.tile_begin;
+  // rotating score buffers: three where two query tiles leave room for them
+  const int nb = (TM::kMaxBufs == 3 && nq == 2) ? 3 : 2;
   if (n_tiles <= 0 || nq < 1 || nq > 2 || u.tail_rows < 0 || u.tail_rows > (D == 64 ? kMaxTailRows : 8)) {
     // the planner never emits such a unit
     if (threadIdx.x == 0) atomicOr(a.err, 2u);
     return;
   }
-  // S/P buffers in rotation: 3 where two query tiles leave room for them
-  const int nb = (TM::kMaxBufs == 3 && nq == 2) ? 3 : 2;
 
   // Tile descriptors into shared memory (off the softmax's critical path).
   for (int i = threadIdx.x; i < min(n_tiles, kMaxSmemTiles); i += kThreads) tile_cache[i] = tiles_g[i];
@@ -243,13 +248,29 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
       tma_load_3d(smem + L::kV + s * L::kTileBytes + kb * 16384, mv, &bar_kv_full[s], kb * 64, u.head, rv);
     }
   };
-  int j_loaded = 0;   // K/V tiles whose loads the producer has issued
-  if (warp == R::kProducer && lane == 0) {
-    prefetch_tmap(&maps.q);
-    prefetch_tmap(mkv);
-    if (a.fused_append) {
-      prefetch_tmap(&maps.k);
-      prefetch_tmap(&maps.v);
+  // K/V rows of pool tiles that earlier frames wrote, prefetched into L2
+  // kL2Ahead tiles ahead of the ring: a head's tile is 128 rows of 128
+  // bytes, 2 KB apart in the pool, and its DRAM latency under load is
+  // several ring periods.
+  auto prefetch_l2 = [&](int j) {
+    if (j >= n_tiles) return;
+    const KvTile t = tile_at(j);
+    if (t.krow != kNotCurrent) return;   // the frame's own rows: just written, or read from k, v
+#pragma unroll
+    for (int kb = 0; kb < D / 64; ++kb) {
+      tma_prefetch_l2_3d(mkv, kb * 64, u.head, t.row);
+      tma_prefetch_l2_3d(mkv, kb * 64, u.head, t.row + rq.page_size);
+    }
+  };
+  int j_loaded = 0;   // K/V tiles whose loads the producer has issued (same in every lane)
+  if (warp == R::kProducer) {
+    if (lane == 0) {
+      prefetch_tmap(&maps.q);
+      prefetch_tmap(mkv);
+      if (a.fused_append) {
+        prefetch_tmap(&maps.k);
+        prefetch_tmap(&maps.v);
+      }
     }
     // Earlier frames' pool rows may be read before the previous kernel on
     // the stream has completed: that kernel is the previous block's launch,
@@ -258,8 +279,24 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
     // before). The first ring stages are filled with them now; the frame's
     // own tiles, and q, wait.
     for (; j_loaded < min(n_tiles, STAGES) && tile_at(j_loaded).krow == kNotCurrent; ++j_loaded)
-      load_kv(j_loaded);
+      if (lane == 0) load_kv(j_loaded);
+    if (lane == 0)
+      for (int jj = STAGES; jj < STAGES + kL2Ahead; ++jj) prefetch_l2(jj);
   }
+  auto load_q = [&]() {
+    mbar_arrive_expect_tx(bar_q, nq * L::kTileBytes);
+    for (int t = 0; t < nq; ++t)
+#pragma unroll
+      for (int kb = 0; kb < D / 64; ++kb)
+        tma_load_3d(smem + L::kQ + t * L::kTileBytes + kb * 16384, &maps.q, bar_q, kb * 64, u.head,
+                    rq.q_row0 + (u.qtile + t) * kTile);
+  };
+  // no TMA write may still be in flight when the CTA exits
+  auto drain_loads = [&](int j_end) {
+    mbar_drain_wait(bar_q, 0);
+    for (int jj = (j_end > STAGES ? j_end - STAGES : 0); jj < j_end; ++jj)
+      mbar_drain_wait(&bar_kv_full[jj % STAGES], (jj / STAGES) & 1);
+  };
   // The setup above overlaps the previous kernel (the frame's K/V append);
   // q, k, v and the frame's own rows are read only after it has completed.
   pdl_wait();
@@ -322,26 +359,21 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
   if (warp == R::kProducer) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      mbar_arrive_expect_tx(bar_q, nq * L::kTileBytes);
-      for (int t = 0; t < nq; ++t)
-#pragma unroll
-        for (int kb = 0; kb < D / 64; ++kb)
-          tma_load_3d(smem + L::kQ + t * L::kTileBytes + kb * 16384, &maps.q, bar_q, kb * 64, u.head,
-                      rq.q_row0 + (u.qtile + t) * kTile);
+      load_q();
       int j = j_loaded;
       for (; j < n_tiles; ++j) {
         const int s = j % STAGES;
         if (j >= STAGES && !mbar_wait(&bar_kv_empty[s], ((j / STAGES) - 1) & 1, abort_flag)) break;
         load_kv(j);
+        if (j >= STAGES) prefetch_l2(j + kL2Ahead);
       }
-      // no TMA write may still be in flight when the CTA exits
-      mbar_drain_wait(bar_q, 0);
-      for (int jj = (j > STAGES ? j - STAGES : 0); jj < j; ++jj)
-        mbar_drain_wait(&bar_kv_full[jj % STAGES], (jj / STAGES) & 1);
+      drain_loads(j);
     }
   } else if (warp == R::kMma) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the issuer's loop (waits included); one elected
+    // lane issues each MMA group and its commit.
+    {
       // Descriptors are built once and stepped by constant offsets (the start
       // address field counts 16-byte units; shared-memory offsets stay far
       // below its 2^14 range, so the adds never carry out of it).
@@ -357,73 +389,79 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
       auto issue_s = [&](int t, int j, int b) {   // S_n = Q_t K_j^T into buffer b
         const uint64_t k = dK + (j % STAGES) * kStage;
         const uint64_t q = dQ + t * kStage;
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          umma_f16_ss(tmem + TM::buf(b), q + kofs(kk), k + kofs(kk), idS, kk > 0);
-        umma_commit(&bar_s_full[b]);
+          for (int kk = 0; kk < D / 16; ++kk)
+            umma_f16_ss(tmem + TM::S(b), q + kofs(kk), k + kofs(kk), idS, kk > 0);
+          umma_commit(&bar_s_full[b]);
+        }
+        __syncwarp();
       };
       auto issue_pv = [&](int t, int j, int b) {   // O_t += P_n V_j, P_n in buffer b
         const uint64_t v = dV + (j % STAGES) * kStage;
-        umma_f16_ts(tmem + TM::O(t), tmem + TM::buf(b), v, idO, j > 0 ? 1u : 0u);
+        if (elect_one()) {
+          umma_f16_ts(tmem + TM::O(t), tmem + TM::S(b), v, idO, j > 0 ? 1u : 0u);
 #pragma unroll
-        for (int kk = 1; kk < kTile / 16; ++kk)
-          umma_f16_ts(tmem + TM::O(t), tmem + TM::buf(b) + kk * 8, v + kk * 128, idO, 1u);
-        umma_commit(&bar_pv_done[t]);
+          for (int kk = 1; kk < kTile / 16; ++kk)
+            umma_f16_ts(tmem + TM::O(t), tmem + TM::S(b) + kk * 8, v + kk * 128, idO, 1u);
+          umma_commit(&bar_pv_done[t]);
+        }
+        __syncwarp();
       };
-      // S_n once PV_{n-NB} has been issued and K/V tile j has landed; PV_n
-      // once P_n is written; both in order of n. A K/V stage is released once
-      // every MMA that reads it has been issued (the commit arrives when they
-      // complete). Non-blocking polls under one bounded wait; the scores go
-      // first, since the softmax waits on them.
+      auto commit = [&](uint64_t* bar) {
+        if (elect_one()) umma_commit(bar);
+        __syncwarp();
+      };
+      // a wait whose outcome is the same in every lane
+      auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+        return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+      };
+      int kv_ready = -1;   // highest K/V tile whose load was waited for
+      auto wait_kv = [&](int j) -> bool {
+        if (j <= kv_ready) return true;
+        if (!wait(&bar_kv_full[j % STAGES], (j / STAGES) & 1)) return false;
+        kv_ready = j;
+        return true;
+      };
+      // Score tile n = j * nq + t goes to buffer n % NB, P over S. The order
+      // is fixed: S_0 .. S_{NB-1}, then PV_n followed by S_{n+NB}. S_{n+NB}
+      // reuses the buffer PV_n reads, so it cannot go earlier (the tensor
+      // pipe runs one thread's MMAs in issue order); PV_n needs P_n; and
+      // neither waits for anything later. The issue of an MMA returns about
+      // when the tensor pipe takes it and each barrier wait costs a shared-
+      // memory round trip, so the issuer simply blocks on the next barrier
+      // in that order (polling several candidates only adds latency).
       const int n_all = n_tiles * nq;
-      int ns = 0, np = 0, ne = 0;   // next S, next PV, next K/V stage release
-      int kv_ready = -1;            // highest K/V tile whose load was observed
-      bool ok = mbar_wait(bar_q, 0, abort_flag);
-      uint64_t t0 = globaltimer_ns();
-      for (uint32_t spin = 1; ok && ne < n_tiles; ++spin) {
-        bool progress = false;
-        if (ns < n_all && ns - nb < np) {
-          const int j = ns / nq;
-          bool ready = j <= kv_ready;
-          if (!ready && mbar_test_wait(&bar_kv_full[j % STAGES], (j / STAGES) & 1)) {
-            kv_ready = j;
-            ready = true;
-          }
-          if (ready) {
-            tc_fence_after();
-            issue_s(ns - j * nq, j, ns % nb);
-            ++ns;
-            progress = true;
-          }
+      int ns = 0, sj = 0, st = 0, sb = 0;   // next S: number, K/V tile, query tile, buffer
+      auto next_s = [&]() -> bool {
+        if (!wait_kv(sj)) return false;
+        tc_fence_after();
+        issue_s(st, sj, sb);
+        ++ns;
+        if (++st == nq) { st = 0; ++sj; }
+        if (++sb == nb) sb = 0;
+        return true;
+      };
+      bool ok = wait(bar_q, 0);
+      while (ok && ns < min(nb, n_all)) ok = next_s();
+      int pj = 0, pt = 0, pb = 0;   // next PV: K/V tile, query tile, buffer
+      uint32_t ppar = 0;            // parity of its p_full phase
+      for (int np = 0; ok && np < n_all; ++np) {
+        if (!wait(&bar_p_full[pb], ppar)) { ok = false; break; }
+        tc_fence_after();
+        issue_pv(pt, pj, pb);
+        if (++pt == nq) {   // every MMA of K/V tile pj issued
+          commit(&bar_kv_empty[pj % STAGES]);
+          pt = 0;
+          ++pj;
         }
-        if (np < ns && mbar_test_wait(&bar_p_full[np % nb], (np / nb) & 1)) {
-          const int j = np / nq;
-          tc_fence_after();
-          issue_pv(np - j * nq, j, np % nb);
-          ++np;
-          progress = true;
-        }
-        while (ne < n_tiles && np >= (ne + 1) * nq) {   // every PV of K/V tile ne issued
-          umma_commit(&bar_kv_empty[ne % STAGES]);
-          ++ne;
-          progress = true;
-        }
-        if (progress) {
-          t0 = globaltimer_ns();
-        } else {
-          // back off: this warp shares its SM sub-partition with two
-          // softmax warps, whose issue slots a tight poll would take
-          __nanosleep(32);
-          if ((spin & 15u) == 0 && (*abort_flag || globaltimer_ns() - t0 > kWaitLimitNs)) {
-            *abort_flag = 1;
-            ok = false;
-          }
-        }
+        if (++pb == nb) { pb = 0; ppar ^= 1u; }
+        if (ns < n_all) ok = next_s();
       }
-      umma_commit(bar_o_final);
+      commit(bar_o_final);
       pdl_trigger();   // the merge kernel may be scheduled (it waits for this grid)
-      // every MMA of this CTA must be complete before TMEM is released
-      umma_commit(bar_drain);
+      // every MMA of this warp must be complete before TMEM is released
+      commit(bar_drain);
       mbar_drain_wait(bar_drain, 0);
     }
   } else if (warp < 8) {
@@ -442,120 +480,117 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
       float l_run = 0.f;         // running sum of 2^(s * sl2 - m_run)
       bool ok = true;
       for (int j = 0; j < n_tiles; ++j) {
+        // score tile n = j * nq + t in buffer n % NB, its P written over it
         const int n = j * nq + t;
         const int b = n % nb;
+        const uint32_t tS = tmem + TM::S(b) + lane_base;
         // Every warp waits, rows or not: p_full counts 128 arrivals a phase.
         // The waits are warp-uniform: tcgen05.ld/st are .sync.aligned.
         if (!__all_sync(0xffffffffu, mbar_wait(&bar_s_full[b], (n / nb) & 1, abort_flag))) { ok = false; break; }
         tc_fence_after();
+        const KvTile tl = tile_at(j);
+        const bool masked = tl.lo > 0 || tl.hi < kTile || tl.step > 1;
+        float alpha = 1.f;
+        bool need = false;
+        uint64_t acc[4] = {0, 0, 0, 0};
+        uint32_t pa[32];   // P columns 0-63 of this row (16-bit pairs)
+        uint32_t r[64];    // the scores of the half being worked on
+        auto load_half = [&](int h) {
+          tmem_ld_x64_wait(tS + 64 * h, r);
+          if (masked) {
+            const uint64_t vis = visible_cols(tl, 64 * h);
+#pragma unroll
+            for (int c = 0; c < 64; ++c)
+              if (!((vis >> c) & 1)) r[c] = 0xFF800000u;   // -inf
+          }
+        };
+        auto half_max = [&]() -> float {
+          float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < 64; c += 8) {
+            mx0 = fmax3(mx0, __uint_as_float(r[c + 0]), __uint_as_float(r[c + 1]));
+            mx1 = fmax3(mx1, __uint_as_float(r[c + 2]), __uint_as_float(r[c + 3]));
+            mx2 = fmax3(mx2, __uint_as_float(r[c + 4]), __uint_as_float(r[c + 5]));
+            mx3 = fmax3(mx3, __uint_as_float(r[c + 6]), __uint_as_float(r[c + 7]));
+          }
+          return fmax3(mx0, mx1, fmaxf(mx2, mx3)) * sl2;
+        };
+        // P = 2^(s * sl2 - m_run) in 16-bit pairs into pk, summed in fp32
+        // into acc. A half can be fully masked (a short last tile of a
+        // page), so the first half may leave m_run at -inf.
+        auto exp_half = [&](uint32_t (&pk)[32]) {
+          // m_run is -inf only while every column so far was masked: P is 0
+          const float mu = m_run == -INFINITY ? 0.f : m_run;
+          const uint64_t negm2 = f2_pack(-mu, -mu);
+#pragma unroll
+          for (int c = 0; c < 64; c += 2) {
+            const uint64_t x = f2_fma(f2_pack(__uint_as_float(r[c]), __uint_as_float(r[c + 1])), sl2x2, negm2);
+            uint64_t e;
+            if ((kEmuMask >> ((c >> 1) & 7)) & 1u) {
+              e = exp2_poly2(x);
+            } else {
+              float x0, x1;
+              f2_unpack(x, x0, x1);
+              e = f2_pack(ex2_approx(x0), ex2_approx(x1));
+            }
+            acc[(c >> 1) & 3] = f2_add(acc[(c >> 1) & 3], e);
+            float e0, e1;
+            f2_unpack(e, e0, e1);
+            pk[c >> 1] = pack16<kFP16>(e0, e1);
+          }
+        };
         if (active) {
-          const uint32_t tS = tmem + TM::buf(b) + lane_base;
-          const KvTile tl = tile_at(j);
-          const bool masked = tl.lo > 0 || tl.hi < kTile || tl.step > 1;
-          float alpha = 1.f;
-          bool need = false;
-          uint64_t acc[4] = {0, 0, 0, 0};
-          auto load_half = [&](int h, uint32_t (&r)[64]) {
-            tmem_ld_x64_wait(tS + 64 * h, r);
-            if (masked) {
-              const uint64_t vis = visible_cols(tl, 64 * h);
-#pragma unroll
-              for (int c = 0; c < 64; ++c)
-                if (!((vis >> c) & 1)) r[c] = 0xFF800000u;   // -inf
-            }
-          };
-          auto half_max = [&](const uint32_t (&r)[64]) -> float {
-            float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
-#pragma unroll
-            for (int c = 0; c < 64; c += 8) {
-              mx0 = fmax3(mx0, __uint_as_float(r[c + 0]), __uint_as_float(r[c + 1]));
-              mx1 = fmax3(mx1, __uint_as_float(r[c + 2]), __uint_as_float(r[c + 3]));
-              mx2 = fmax3(mx2, __uint_as_float(r[c + 4]), __uint_as_float(r[c + 5]));
-              mx3 = fmax3(mx3, __uint_as_float(r[c + 6]), __uint_as_float(r[c + 7]));
-            }
-            return fmax3(mx0, mx1, fmaxf(mx2, mx3)) * sl2;
-          };
-          // P = 2^(s * sl2 - m_run) in 16-bit pairs into pk, summed in fp32
-          // into acc. A half can be fully masked (a short last tile of a
-          // page), so the first half may leave m_run at -inf.
-          auto exp_half = [&](const uint32_t (&sv)[64], uint32_t (&pk)[32]) {
-            // m_run is -inf only while every column so far was masked: P is 0
-            const float mu = m_run == -INFINITY ? 0.f : m_run;
-            const uint64_t negm2 = f2_pack(-mu, -mu);
-#pragma unroll
-            for (int c = 0; c < 64; c += 2) {
-              const uint64_t x = f2_fma(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sl2x2, negm2);
-              uint64_t e;
-              if ((kEmuMask >> ((c >> 1) & 7)) & 1u) {
-                e = exp2_poly2(x);
-              } else {
-                float x0, x1;
-                f2_unpack(x, x0, x1);
-                e = f2_pack(ex2_approx(x0), ex2_approx(x1));
-              }
-              acc[(c >> 1) & 3] = f2_add(acc[(c >> 1) & 3], e);
-              float e0, e1;
-              f2_unpack(e, e0, e1);
-              pk[c >> 1] = pack16<kFP16>(e0, e1);
-            }
-          };
-          {
-            uint32_t r[64];
-            load_half(0, r);
-            const float m0 = half_max(r);
-            if (m0 > m_run + kRescaleLog2) {
-              alpha = ex2_approx(m_run - m0);   // 0 on the first tile (m_run = -inf)
-              l_run *= alpha;
-              m_run = m0;
+          load_half(0);
+          const float m0 = half_max();
+          if (m0 > m_run + kRescaleLog2) {
+            alpha = ex2_approx(m_run - m0);   // 0 on the first tile (m_run = -inf)
+            l_run *= alpha;
+            m_run = m0;
+            need = true;
+          }
+          exp_half(pa);
+        }
+        if (active) {
+          tmem_st_x32(tS, pa);   // P columns 0-31 (16-bit pairs) over S columns 0-31, read
+          load_half(1);
+          const float m1 = half_max();
+          const bool rare = m1 > m_run + kRescaleLog2;
+          if (__any_sync(0xffffffffu, rare)) {
+            // Rare: the second half raised the max past the threshold after
+            // the first half's P was stored. Scale that half (and its sum)
+            // down to the new max; the extra rounding stays at the 16-bit
+            // level of P. The TMEM accesses are warp-collective, so the
+            // whole warp takes this branch; other rows scale by 1 (exact).
+            float a2 = 1.f;
+            if (rare) {
+              a2 = ex2_approx(m_run - m1);
+              alpha *= a2;
+              l_run *= a2;
+              m_run = m1;
               need = true;
             }
-            uint32_t pa[32];
-            exp_half(r, pa);
-            tmem_st_x32(tS, pa);   // P columns 0-31 (16-bit pairs) over S columns 0-31, read
-          }
-          {
-            uint32_t r[64];
-            load_half(1, r);
-            const float m1 = half_max(r);
-            const bool rare = m1 > m_run + kRescaleLog2;
-            if (__any_sync(0xffffffffu, rare)) {
-              // Rare: the second half raised the max past the threshold after
-              // the first half's P was stored. Scale that half (and its sum)
-              // down to the new max; the extra rounding stays at the 16-bit
-              // level of P. The TMEM accesses are warp-collective, so the
-              // whole warp takes this branch; other rows scale by 1 (exact).
-              float a2 = 1.f;
-              if (rare) {
-                a2 = ex2_approx(m_run - m1);
-                alpha *= a2;
-                l_run *= a2;
-                m_run = m1;
-                need = true;
-              }
-              const uint64_t a22 = f2_pack(a2, a2);
+            const uint64_t a22 = f2_pack(a2, a2);
 #pragma unroll
-              for (int i = 0; i < 4; ++i) acc[i] = f2_mul(acc[i], a22);
-              uint32_t pa[32];
-              tmem_wait_st();
-              tmem_ld_x32_wait(tS, pa);
+            for (int i = 0; i < 4; ++i) acc[i] = f2_mul(acc[i], a22);
+            tmem_wait_st();
+            tmem_ld_x32_wait(tS, pa);
 #pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                float p0, p1;
-                unpack16<kFP16>(pa[i], p0, p1);
-                pa[i] = pack16<kFP16>(p0 * a2, p1 * a2);
-              }
-              tmem_st_x32(tS, pa);
+            for (int i = 0; i < 32; ++i) {
+              float p0, p1;
+              unpack16<kFP16>(pa[i], p0, p1);
+              pa[i] = pack16<kFP16>(p0 * a2, p1 * a2);
             }
-            uint32_t pb[32];
-            exp_half(r, pb);
-            tmem_st_x32(tS + 32, pb);   // P columns 32-63 over S columns 32-63
+            tmem_st_x32(tS, pa);
           }
+          uint32_t pb[32];
+          exp_half(pb);
+          tmem_st_x32(tS + 32, pb);   // P columns 32-63 over S columns 32-63
           float s0, s1;
           f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), s0, s1);
           l_run += s0 + s1;
           // Rescale O_t if the running max moved. O_t holds PV_t(0..j-1);
-          // PV_t(j-2) completed before S_t(j) did, so the wait for PV_t(j-1)
-          // cannot observe an earlier phase of pv_done.
+          // PV_t(j-2) completed before S_t(j) did (NB <= 2 nq), so the wait
+          // for PV_t(j-1) cannot observe an earlier phase of pv_done.
           if (j > 0 && __any_sync(0xffffffffu, need)) {
             if (!__all_sync(0xffffffffu, mbar_wait(&bar_pv_done[t], (j - 1) & 1, abort_flag))) {
               ok = false;
@@ -592,47 +627,46 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
         const int slot = u.slot[t];
 #pragma unroll
         for (int c = 0; c < D; c += 32) {
-          uint32_t r[32];
-          tmem_ld_x32_wait(tO + c, r);
+          uint32_t o[32];
+          tmem_ld_x32_wait(tO + c, o);
           if (!store) continue;
           if (slot < 0) {
-            uint16_t* o = reinterpret_cast<uint16_t*>(a.out) + ((size_t)grow * a.H + u.head) * D + c;
+            uint16_t* po = reinterpret_cast<uint16_t*>(a.out) + ((size_t)grow * a.H + u.head) * D + c;
 #pragma unroll
             for (int i = 0; i < 32; i += 8) {
               uint4 v;
-              v.x = pack16<kFP16>(__uint_as_float(r[i + 0]) * inv, __uint_as_float(r[i + 1]) * inv);
-              v.y = pack16<kFP16>(__uint_as_float(r[i + 2]) * inv, __uint_as_float(r[i + 3]) * inv);
-              v.z = pack16<kFP16>(__uint_as_float(r[i + 4]) * inv, __uint_as_float(r[i + 5]) * inv);
-              v.w = pack16<kFP16>(__uint_as_float(r[i + 6]) * inv, __uint_as_float(r[i + 7]) * inv);
-              *reinterpret_cast<uint4*>(o + i) = v;
+              v.x = pack16<kFP16>(__uint_as_float(o[i + 0]) * inv, __uint_as_float(o[i + 1]) * inv);
+              v.y = pack16<kFP16>(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+              v.z = pack16<kFP16>(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
+              v.w = pack16<kFP16>(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
+              *reinterpret_cast<uint4*>(po + i) = v;
             }
           } else {
             float* po = a.part_o + ((size_t)slot * kTile + row) * D + c;
 #pragma unroll
             for (int i = 0; i < 32; i += 4)
               *reinterpret_cast<float4*>(po + i) =
-                  make_float4(__uint_as_float(r[i]) * inv, __uint_as_float(r[i + 1]) * inv,
-                              __uint_as_float(r[i + 2]) * inv, __uint_as_float(r[i + 3]) * inv);
+                  make_float4(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv,
+                              __uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
           }
         }
         if (store && slot >= 0) a.part_lse[(size_t)slot * kTile + row] = m_run + log2f(l_run);
       }
     }
-  } else if (has_tail && (warp == 8 || warp == 10)) {
+  } else if (has_tail && warp >= R::kTail0 && warp < R::kTail0 + R::kTailWarps) {
     // ------------------------------------------------------------ tail
     // Tail warp w takes K/V rows [64 w, 64 w + 64) of every tile and works
     // transposed, so the few tail rows sit in the narrow dimension:
-    // S^T = K Q_tail^T as 4 m-tiles (16 K/V rows) x 4 k-steps x NQ n-tiles
-    // (8 query rows each) of m16n8k16, softmax per query column, then
-    // O^T += V^T P^T (4 m-tiles of 16 output columns x 4 k-steps x NQ). P^T
-    // goes from the accumulator layout to the operand layout with movmatrix.
-    // Query rows past the tail are zero and never stored.
+    // S^T = K Q_tail^T as 4 m-tiles (16 K/V rows) x D/16 k-steps x NQ n-tiles
+    // (8 query rows each) of m16n8k16, an online softmax per query column,
+    // then O^T += V^T P^T (D/16 m-tiles of 16 output columns x 4 k-steps x NQ).
+    // P^T goes from the accumulator layout to the operand layout with
+    // movmatrix. Query rows past the tail are zero and never stored.
     auto tail_body = [&](auto nq_tag) {
       constexpr int NQ = decltype(nq_tag)::value;   // 8-row query groups (1 or 2)
-      constexpr int kCW = kTile / R::kTailWarps;     // K/V rows per tail warp (64)
-      constexpr int kMT = kCW / 16;                  // S^T m-tiles
+      constexpr int kMT = 4;                         // S^T m-tiles per 64-row half
       constexpr int kDT = D / 16;                    // O^T m-tiles
-      const int w = (warp - 8) >> 1;
+      const int w = warp - R::kTail0;
       const int g = lane >> 2, q4 = lane & 3;
       const float sl2 = a.scale_log2;
       const int row0 = rq.q_row0 + (u.qtile + nq) * kTile;   // first tail row in q/out
@@ -668,88 +702,110 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
         const KvTile tl = tile_at(j);
         const uint32_t ks = k_base + s * L::kTileBytes;
         const uint32_t vs = v_base + s * L::kTileBytes;
-        const uint64_t vis = visible_cols(tl, kCW * w);   // this warp's 64 K/V rows
-        // S^T: m-tile i = K/V rows kCW w + 16 i .. + 15 (accumulator rows g, g + 8)
-        float sc[kMT][NQ][4];
+        const uint64_t vis = visible_cols(tl, 64 * w);   // K/V rows 64 w .. 64 w + 63
+        if (vis != 0) {                                    // else nothing visible in this half
+          // S^T: m-tile i = K/V rows 64 w + 16 i .. + 15 (accumulator rows g, g + 8).
+          // Every A fragment of a group of m-tiles is loaded before its MMAs,
+          // so the shared-memory loads overlap one another.
+          float sc[kMT][NQ][4];
+          constexpr int kSG = D == 64 ? 4 : 2;   // m-tiles per load group
 #pragma unroll
-        for (int i = 0; i < kMT; ++i) {
+          for (int i0 = 0; i0 < kMT; i0 += kSG) {
+            uint32_t af[kSG][D / 16][4];
 #pragma unroll
-          for (int n = 0; n < NQ; ++n) sc[i][n][0] = sc[i][n][1] = sc[i][n][2] = sc[i][n][3] = 0.f;
-          const int kr = kCW * w + 16 * i + (lane & 7) + 8 * ((lane >> 3) & 1);
+            for (int ii = 0; ii < kSG; ++ii) {
+              const int kr = 64 * w + 16 * (i0 + ii) + (lane & 7) + 8 * ((lane >> 3) & 1);
 #pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const int ch = 2 * k + (lane >> 4);
-            uint32_t af[4];
-            ldsm_x4(ks + (ch >> 3) * 16384 + kr * 128 + (((ch & 7) ^ (kr & 7)) << 4), af);
+              for (int k = 0; k < D / 16; ++k) {
+                const int ch = 2 * k + (lane >> 4);
+                ldsm_x4(ks + (ch >> 3) * 16384 + kr * 128 + (((ch & 7) ^ (kr & 7)) << 4), af[ii][k]);
+              }
+            }
 #pragma unroll
-            for (int n = 0; n < NQ; ++n) mma_16816<kFP16>(sc[i][n], af, qb[n][k][0], qb[n][k][1]);
-          }
-          // mask the K/V rows that are not visible
+            for (int ii = 0; ii < kSG; ++ii) {
+              const int i = i0 + ii;
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            if (!((vis >> (16 * i + g + 8 * h)) & 1))
+              for (int n = 0; n < NQ; ++n) sc[i][n][0] = sc[i][n][1] = sc[i][n][2] = sc[i][n][3] = 0.f;
 #pragma unroll
-              for (int n = 0; n < NQ; ++n) sc[i][n][2 * h] = sc[i][n][2 * h + 1] = -INFINITY;
-          }
-        }
-        // per query column: max over this warp's K/V rows (lane values, then
-        // the eight lanes with the same q4)
+              for (int k = 0; k < D / 16; ++k)
 #pragma unroll
-        for (int n = 0; n < NQ; ++n) {
+                for (int n = 0; n < NQ; ++n) mma_16816<kFP16>(sc[i][n], af[ii][k], qb[n][k][0], qb[n][k][1]);
+              // mask the K/V rows that are not visible
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            float mx = -INFINITY;
+              for (int h = 0; h < 2; ++h) {
+                if (!((vis >> (16 * i + g + 8 * h)) & 1))
 #pragma unroll
-            for (int i = 0; i < kMT; ++i) mx = fmax3(mx, sc[i][n][e], sc[i][n][2 + e]);
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-            mx *= sl2;
-            if (mx > m_q[n][e] + kRescaleLog2) {   // never true while every row was masked (-inf)
-              const float al = ex2_approx(m_q[n][e] - mx);
-              l_q[n][e] *= al;
-#pragma unroll
-              for (int dm = 0; dm < kDT; ++dm) { o[dm][n][e] *= al; o[dm][n][2 + e] *= al; }
-              m_q[n][e] = mx;
+                  for (int n = 0; n < NQ; ++n) sc[i][n][2 * h] = sc[i][n][2 * h + 1] = -INFINITY;
+              }
             }
           }
-        }
-        // P^T as B fragments: k-step i = K/V rows 16 i .. + 15 of this warp's
-        // (while every row so far was masked the max is -inf and P is 0)
-        uint32_t pb[kMT][NQ][2];
+          // per query column: max over these K/V rows (lane values, then
+          // the eight lanes with the same q4)
 #pragma unroll
-        for (int n = 0; n < NQ; ++n) {
-          const float m0 = m_q[n][0] == -INFINITY ? 0.f : m_q[n][0];
-          const float m1 = m_q[n][1] == -INFINITY ? 0.f : m_q[n][1];
+          for (int n = 0; n < NQ; ++n) {
 #pragma unroll
-          for (int i = 0; i < kMT; ++i) {
-            const float p0 = ex2_approx(fmaf(sc[i][n][0], sl2, -m0));
-            const float p1 = ex2_approx(fmaf(sc[i][n][1], sl2, -m1));
-            const float p2 = ex2_approx(fmaf(sc[i][n][2], sl2, -m0));
-            const float p3 = ex2_approx(fmaf(sc[i][n][3], sl2, -m1));
-            l_q[n][0] += p0 + p2;
-            l_q[n][1] += p1 + p3;
-            pb[i][n][0] = movmatrix_t(pack16<kFP16>(p0, p1));
-            pb[i][n][1] = movmatrix_t(pack16<kFP16>(p2, p3));
+            for (int e = 0; e < 2; ++e) {
+              float mx = -INFINITY;
+#pragma unroll
+              for (int i = 0; i < kMT; ++i) mx = fmax3(mx, sc[i][n][e], sc[i][n][2 + e]);
+              mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+              mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+              mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+              mx *= sl2;
+              if (mx > m_q[n][e] + kRescaleLog2) {   // never true while every row was masked (-inf)
+                const float al = ex2_approx(m_q[n][e] - mx);
+                l_q[n][e] *= al;
+#pragma unroll
+                for (int dm = 0; dm < kDT; ++dm) { o[dm][n][e] *= al; o[dm][n][2 + e] *= al; }
+                m_q[n][e] = mx;
+              }
+            }
           }
-        }
-        // O^T += V^T P^T: A fragments by transposed loads of V
+          // P^T as B fragments: k-step i = K/V rows 16 i .. + 15 of the half
+          // (while every row so far was masked the max is -inf and P is 0)
+          uint32_t pb[kMT][NQ][2];
 #pragma unroll
-        for (int dm = 0; dm < kDT; ++dm) {
+          for (int n = 0; n < NQ; ++n) {
+            const float m0 = m_q[n][0] == -INFINITY ? 0.f : m_q[n][0];
+            const float m1 = m_q[n][1] == -INFINITY ? 0.f : m_q[n][1];
 #pragma unroll
-          for (int i = 0; i < kMT; ++i) {
-            const int vr = kCW * w + 16 * i + (lane & 7) + 8 * (lane >> 4);
-            const int ch = 2 * dm + ((lane >> 3) & 1);
-            uint32_t af[4];
-            ldsm_x4_t(vs + (ch >> 3) * 16384 + vr * 128 + (((ch & 7) ^ (vr & 7)) << 4), af);
+            for (int i = 0; i < kMT; ++i) {
+              const float p0 = ex2_approx(fmaf(sc[i][n][0], sl2, -m0));
+              const float p1 = ex2_approx(fmaf(sc[i][n][1], sl2, -m1));
+              const float p2 = ex2_approx(fmaf(sc[i][n][2], sl2, -m0));
+              const float p3 = ex2_approx(fmaf(sc[i][n][3], sl2, -m1));
+              l_q[n][0] += p0 + p2;
+              l_q[n][1] += p1 + p3;
+              pb[i][n][0] = movmatrix_t(pack16<kFP16>(p0, p1));
+              pb[i][n][1] = movmatrix_t(pack16<kFP16>(p2, p3));
+            }
+          }
+          // O^T += V^T P^T: A fragments by transposed loads of V, a group of
+          // output m-tiles loaded before its MMAs
+          constexpr int kPG = D == 64 ? 4 : 2;   // output m-tiles per load group
 #pragma unroll
-            for (int n = 0; n < NQ; ++n) mma_16816<kFP16>(o[dm][n], af, pb[i][n][0], pb[i][n][1]);
+          for (int d0 = 0; d0 < kDT; d0 += kPG) {
+            uint32_t af[kPG][kMT][4];
+#pragma unroll
+            for (int dd = 0; dd < kPG; ++dd)
+#pragma unroll
+              for (int i = 0; i < kMT; ++i) {
+                const int vr = 64 * w + 16 * i + (lane & 7) + 8 * (lane >> 4);
+                const int ch = 2 * (d0 + dd) + ((lane >> 3) & 1);
+                ldsm_x4_t(vs + (ch >> 3) * 16384 + vr * 128 + (((ch & 7) ^ (vr & 7)) << 4), af[dd][i]);
+              }
+#pragma unroll
+            for (int dd = 0; dd < kPG; ++dd)
+#pragma unroll
+              for (int i = 0; i < kMT; ++i)
+#pragma unroll
+                for (int n = 0; n < NQ; ++n) mma_16816<kFP16>(o[d0 + dd][n], af[dd][i], pb[i][n][0], pb[i][n][1]);
           }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar_kv_empty[s]);
       }
-      // this warp's sums per query row
+      // this warp's sums per query row (over the eight lanes that hold it)
 #pragma unroll
       for (int n = 0; n < NQ; ++n)
 #pragma unroll
@@ -783,8 +839,10 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
           }
       }
       named_bar_sync(1, 32 * kTW);
+      // (a failed wait in either warp also sets the abort flag, which marks
+      // the launch's outputs invalid)
       ok = __all_sync(0xffffffffu, ok);
-      // merge: thread i of the tail warps finishes row i / 4, columns 16 (i % 4) .. + 15
+      // merge: thread i of the tail warps finishes row i / 4, columns (i % 4) D / 4 .. + D / 4 - 1
       constexpr int kCols = D / 4;
       const int i = w * 32 + lane;
       const int r = i >> 2, c0 = (i & 3) * kCols;
@@ -873,13 +931,16 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
       const int group_rows = rows_of(0) + (nq > 1 ? rows_of(1) : 0) + tail_rows;
       const int r0 = (int)((long long)u.chunk * group_rows / n);
       const int r1 = (int)((long long)(u.chunk + 1) * group_rows / n);
-      for (int gr = r0 + warp; gr < r1; gr += R::kWarps) {
+      // 8 lanes per row: 48 rows of loads in flight at once
+      merge_rows_grouped<D, kFP16>(a.part_o, a.part_lse, n, r0 + (threadIdx.x >> 3), r1, kThreads / 8,
+                                   threadIdx.x & 7, [&](int gr, int* slot0, int* row, uint16_t** out_row) {
         int t = 0, r = gr;
         while (t < nq && r >= rows_of(t)) r -= rows_of(t++);
         const int orow = rq.q_row0 + (u.qtile + t) * kTile + r;
-        uint16_t* out_row = reinterpret_cast<uint16_t*>(a.out) + ((size_t)orow * a.H + u.head) * D;
-        merge_row_warp<D, kFP16>(a.part_o, a.part_lse, u.slot[t] - u.chunk, n, r, out_row, lane);
-      }
+        *slot0 = u.slot[t] - u.chunk;
+        *row = r;
+        *out_row = reinterpret_cast<uint16_t*>(a.out) + ((size_t)orow * a.H + u.head) * D;
+      });
     }
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -893,8 +954,10 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
   if (threadIdx.x == 0 && *abort_flag) atomicOr(a.err, 1u);
 }
 
-// Exponentials on the FMA pipe: pair positions {6, 7} of every 8 (25 %).
-constexpr uint32_t kEmu = 0xC0u;
+// Exponentials on the FMA pipe: pair position 7 of every 8 (12.5 %). The
+// softmax is bound by instruction issue more than by the MUFU unit here, and
+// the polynomial costs six instructions a pair against two MUFU ones.
+constexpr uint32_t kEmu = 0x80u;
 
 template <int D, bool kFP16, int STAGES>
 static cudaError_t launch_attn_t(const AttnMaps& maps, const AttnArgs& a, int n_units, cudaStream_t stream) {

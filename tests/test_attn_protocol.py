@@ -1,8 +1,8 @@
 """A randomised model of the attention kernel's mbarrier protocol.
 
 The kernel's warps meet only at mbarriers and at the tensor pipe, so the
-protocol can be checked on the CPU: this model runs the MMA issuer's poll
-loop, every softmax warp (with valid rows or not), the TMA producer, the tail
+protocol can be checked on the CPU: this model runs the MMA issuer's fixed
+issue order, every softmax warp (with valid rows or not), the TMA producer, the tail
 warps' stage releases and an in-order tensor pipe whose commit arrives once
 every earlier MMA has run, in random interleavings. It checks:
 
@@ -19,9 +19,10 @@ every earlier MMA has run, in random interleavings. It checks:
 The schedule modelled is the kernel's: score tile n = j * nq + t goes to
 TMEM buffer n % NB (NB = 3 for head_dim 64 with two query tiles, else 2) with
 its P stored over it; per-buffer s_full / p_full barriers; the issuer issues
-S_n once PV_{n-NB} has been issued and PV_n once P_n is written, both in
-order of n; a softmax warp waits for PV_t(j-1) only when it rescales O_t. The
-negative tests drop one rule each and find the failure it prevents.
+S_0 .. S_{NB-1}, then PV_n (once P_n is written) followed by S_{n+NB} (once
+its K/V tile has landed), for n = 0, 1, ...; a softmax warp waits for
+PV_t(j-1) only when it rescales O_t. The negative tests drop one rule each
+and find the failure it prevents.
 
 A model is not the kernel: it checks the protocol's logic only.
 """
@@ -56,8 +57,9 @@ class Bar:
 
 def run(nq, n_tiles, active, tail, seed, nb=None, gate_slack=0, idle_warps_wait=True, rescale_p=0.2):
     """nb: S/P buffers (default: the kernel's choice, 3 for two query tiles
-    else 2). gate_slack: S_n issued once PV_{n-NB+gate_slack} is issued (0 is
-    the kernel's rule, -1 one PV too early). idle_warps_wait: warps without valid rows wait for
+    else 2). gate_slack: NB - gate_slack scores are issued before the first
+    PV, so S_n follows PV_{n-NB+gate_slack} (0 is the kernel's rule, -1 one
+    PV too early). idle_warps_wait: warps without valid rows wait for
     their scores before they arrive (the kernel's rule)."""
     rng = random.Random(seed)
     if nb is None:
@@ -91,37 +93,47 @@ def run(nq, n_tiles, active, tail, seed, nb=None, gate_slack=0, idle_warps_wait=
         ran.add((kind, n))
 
     def issuer():
-        st = {"ns": 0, "np": 0, "ne": 0, "kv": -1, "q": False, "done": False}
+        # the kernel's fixed order: S_0 .. S_{NB-1}, then PV_n and S_{n+NB}
+        # for n = 0, 1, ...; each op blocks on its own barrier
+        prefill = min(nb - gate_slack, n_all)
+        st = {"ns": 0, "np": 0, "kv": -1, "after_pv": False, "done": False}
+
+        def issue_s():
+            ns = st["ns"]
+            j = ns // nq
+            if j > st["kv"]:
+                if not kv_full[j % ST].test(j // ST, "issuer"):
+                    return False
+                st["kv"] = j
+            pipe.append(("S", ns))
+            pipe.append(("commit", s_full[ns % nb]))
+            st["ns"] = ns + 1
+            return True
 
         def step():
             if st["done"]:
                 return None
-            moved = False
-            ns, np_ = st["ns"], st["np"]
-            if ns < n_all and ns - nb + gate_slack < np_:
-                j = ns // nq
-                ready = j <= st["kv"]
-                if not ready and kv_full[j % ST].test(j // ST, "issuer"):
-                    st["kv"], ready = j, True
-                if ready:
-                    pipe.append(("S", ns))
-                    pipe.append(("commit", s_full[ns % nb]))
-                    st["ns"] = ns + 1
-                    moved = True
-            if np_ < st["ns"] and p_full[np_ % nb].test(np_ // nb, "issuer"):
-                pipe.append(("PV", np_))
-                pipe.append(("commit", pv_done[np_ % nq]))
-                st["np"] = np_ + 1
-                moved = True
-            while st["ne"] < n_tiles and st["np"] >= (st["ne"] + 1) * nq:
-                pipe.append(("commit", kv_empty[st["ne"] % ST]))
-                st["ne"] += 1
-                moved = True
-            if st["ne"] >= n_tiles:
+            if st["ns"] < prefill:
+                return issue_s()
+            if st["after_pv"]:
+                if st["ns"] < n_all and not issue_s():
+                    return False
+                st["after_pv"] = False
+                return True
+            np_ = st["np"]
+            if np_ == n_all:
                 pipe.append(("commit", o_final))
                 st["done"] = True
                 return True
-            return moved
+            if not p_full[np_ % nb].test(np_ // nb, "issuer"):
+                return False
+            pipe.append(("PV", np_))
+            pipe.append(("commit", pv_done[np_ % nq]))
+            if np_ % nq == nq - 1:   # every MMA of K/V tile np_ // nq issued
+                pipe.append(("commit", kv_empty[(np_ // nq) % ST]))
+            st["np"] = np_ + 1
+            st["after_pv"] = True
+            return True
         return step
 
     def softmax_warp(t, w):
