@@ -46,7 +46,7 @@ def peaks():
 
 TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "paged_prefill_attn_224x224_dram.txt")
 KERNEL_SOURCES = ("paged_attn.cu", "sm100.cuh", "tmem_access.cuh", "kernels.h", "kv_layout.h", "merge.cuh",
-                  "launch.cuh")
+                  "launch.cuh", "per_device.h")
 
 
 def kernel_source_hash():

@@ -11,6 +11,8 @@
 #include <atomic>
 #include <cstdint>
 
+#include "per_device.h"
+
 namespace pkv {
 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
@@ -39,22 +41,17 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
-constexpr int kMaxDevices = 256;
-
 // cudaFuncSetAttribute(MaxDynamicSharedMemorySize) applies to the current
 // device only, so it is set once per (kernel, device). `done` is the caller's
-// per-kernel array of kMaxDevices flags. Two threads that race on a first
-// launch both set the attribute, which is harmless.
+// per-kernel array of kMaxDevices flags.
 template <typename F>
 cudaError_t ensure_dynamic_smem(F kern, int bytes, std::atomic<uint8_t>* done) {
   int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  const cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess) done[dev].store(1, std::memory_order_release);
-  return e;
+  return once_per_device(dev, done, cudaSuccess, cudaErrorInvalidDevice, [&]() {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  });
 }
 
 }  // namespace pkv
