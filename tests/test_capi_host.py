@@ -337,6 +337,21 @@ def test_kv_tiles_cover_visible_tokens_exactly_once(pkv, ps, n, xs):
     pkv.kv_plan_free(p)
 
 
+def test_unit_beyond_the_shared_tile_cache_host_plan(pkv):
+    """The configuration of the GPU test of a CTA with more K/V tiles than its
+    shared-memory cache of 512 descriptors: 16-token pages, S = 2, W = 600,
+    620 frames, no split."""
+    S, W, ps, frames = 2, 600, 16, 620
+    h = mk(pkv, S, W, ps, (S + W + 1) + -(-6 * frames // ps), H=1)
+    for _ in range(frames):
+        step(pkv, h)
+    p = pkv.kv_plan([h], tiles_per_split=4096)
+    s = pkv.kv_plan_get_stats(p)
+    assert s["n_ctas"] == 1 and s["tiles_per_cta"] == s["n_kv_tiles"] == 836 > 512
+    assert s["visible_tokens"] == (S + W) * ps + 6 * frames
+    pkv.kv_plan_free(p)
+
+
 def test_split_schedule_covers_each_unit(pkv):
     """Host plan for the 224x224 shape at frame 320: 160 tiles per head
     (71 earlier patch pages x 2, the current frame's page x 2, the earlier

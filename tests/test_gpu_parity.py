@@ -86,6 +86,17 @@ def test_split_and_unsplit_agree(pkv):
     assert d.max().item() <= 1e-2
 
 
+def test_unit_with_more_tiles_than_the_shared_tile_cache(pkv):
+    """One unsplit CTA over 836 K/V tiles (16-token pages, one tile per page,
+    and a 600-frame window; the host plan's tile count is checked in
+    test_capi_host). A CTA caches 512 tile descriptors in shared
+    memory and reads the rest from global memory; both kinds of tile are
+    checked against the oracle, through both frame-step forms."""
+    wl = small(16, H=1, S=2, W=600, frames=620)
+    run_stream(pkv, wl, seed=41, n_frames=wl.frames, check={wl.frames - 1}, tiles_per_split=4096)
+    run_stream(pkv, wl, seed=42, n_frames=wl.frames, check={wl.frames - 1}, tiles_per_split=4096, fused=True)
+
+
 @pytest.mark.parametrize("ps", [16, 64, 100, 128, 129, 256, 999])
 def test_page_sizes_with_eviction(pkv, ps):
     wl = small(ps, H=2, S=2, W=3, frames=12)
