@@ -86,6 +86,22 @@ def test_split_and_unsplit_agree(pkv):
     assert d.max().item() <= 1e-2
 
 
+# Frame sizes around the tail limits: T = P + 6 rows make full 128-row query
+# tiles plus a remainder r. r <= 16 (head_dim 64) or r <= 8 (head_dim 128)
+# runs on the tail warps -- one 8-row group for r <= 8, two above -- and a
+# larger remainder is a query tile of its own.
+@pytest.mark.parametrize("ps,D", [(123, 64), (131, 64), (138, 64), (139, 64), (259, 64), (266, 64),
+                                  (130, 128), (131, 128)],
+                         ids=lambda x: str(x))
+def test_tail_sizes(pkv, ps, D):
+    dtype = "fp16" if D == 128 else "bf16"
+    wl = small(ps, H=2, D=D, S=2, W=3, dtype=dtype, frames=7)
+    T = ps + 6
+    run_stream(pkv, wl, seed=50 + ps + D, n_frames=wl.frames, check={0, 6}, rows=np.arange(T))
+    run_stream(pkv, wl, seed=60 + ps + D, n_frames=wl.frames, check={6}, rows=np.arange(T), fused=True)
+    run_stream(pkv, wl, seed=70 + ps + D, n_frames=wl.frames, check={6}, rows=np.arange(T), tiles_per_split=1)
+
+
 def test_unit_with_more_tiles_than_the_shared_tile_cache(pkv):
     """One unsplit CTA over 836 K/V tiles (16-token pages, one tile per page,
     and a 600-frame window; the host plan's tile count is checked in
