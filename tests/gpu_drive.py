@@ -103,7 +103,7 @@ def workspace(pkv, caches):
 
 def run_stream(pkv, wl, seed, n_frames, check, rows=None, defer=None, keep=None,
                tiles_per_split=0, patch_pages=0, collect=None, dense=(), cross_special=True,
-               camera_only=False, fused=False, all_rows=()):
+               camera_only=False, fused=False, all_rows=(), frames=None):
     """Append frames 0..n_frames-1 of block 0; at frames in `check`, plan + run
     and compare the chosen query rows with the oracle. defer[f] / keep[f]:
     frame f is appended with eviction deferred and then committed (keep) or
@@ -111,8 +111,10 @@ def run_stream(pkv, wl, seed, n_frames, check, rows=None, defer=None, keep=None,
     fp32 dense gather of the visible pages; at frames in `all_rows` every row
     is checked against the oracle whatever `rows` says. fused: each frame goes through
     begin_frame + plan + run_append (the append inside the attention launch)
-    instead of append_frame + plan + run. Returns {frame: (max_err, mean_err)}."""
-    fr = Frames(wl, seed)
+    instead of append_frame + plan + run. frames: a Frames-like source of the
+    stream's q, k, v (default: the seeded workload frames). Returns
+    {frame: (max_err, mean_err)}."""
+    fr = frames if frames is not None else Frames(wl, seed)
     cache = new_cache(pkv, wl, patch_pages=patch_pages, cross_special=cross_special, camera_only=camera_only)
     ws = workspace(pkv, [cache])
     so = StreamOracle(wl.S, wl.W, wl.NS, wl.P, wl.dtype, fr.bits, cross_frame_special=cross_special,

@@ -102,6 +102,47 @@ def test_tail_sizes(pkv, ps, D):
     run_stream(pkv, wl, seed=70 + ps + D, n_frames=wl.frames, check={6}, rows=np.arange(T), tiles_per_split=1)
 
 
+class SpikeFrames(Frames):
+    """Every query row near one vector u (per head) and a few keys equal to
+    c * u, so that their scores stand far above the rest: in log2 units a key
+    c * u scores about c * |u|^2 / sqrt(D) * log2(e), about 11.5 c here, while
+    the other keys' maximum is about 6."""
+
+    def __init__(self, wl, seed, spikes):
+        super().__init__(wl, seed)
+        g = torch.Generator().manual_seed(seed)
+        self.u = torch.randn(wl.H, wl.D, generator=g)
+        self.spikes = spikes   # {(frame, patch token): c}
+
+    def get(self, f):
+        if f not in self.cache:
+            q, k, v = (x.float() for x in workload.frame_qkv(self.wl, self.seed, f, 0))
+            q = self.u.unsqueeze(0) + 0.1 * q
+            for (ff, p), c in self.spikes.items():
+                if ff == f:
+                    k[self.wl.NS + p] = c * self.u
+            dt = self.wl.torch_dtype()
+            self.cache[f] = (q.to(dt), k.to(dt), v.to(dt))
+        return self.cache[f]
+
+
+@pytest.mark.parametrize("fused,tps", [(False, 4096), (True, 4096), (False, 0)])
+def test_running_max_jumps_force_both_rescales(pkv, fused, tps):
+    """Spike keys move the running max past the 2^8 lazy threshold. The first
+    sits in the second 64-key half of the stream's first tile, so it raises
+    the max (by 9 in head 0, 14 in head 1, log2 units) after the first half's
+    P was stored, which is then scaled down in TMEM. The second, in a first
+    half four frames later, raises it again by 10 in head 1 (O rescaled after
+    earlier PVs) and by 7 in head 0 (under the threshold: no rescale). The
+    stale terms a rescale scales would otherwise weigh 2^8 times too much.
+    Frames 0 and 1 are scale frames, so the first spike stays visible. Without
+    a split (tiles_per_split 4096) both jumps fall inside one CTA's tiles."""
+    wl = small(256, H=2, S=2, W=3, frames=7)
+    fr = SpikeFrames(wl, 77, {(0, 100): 1.4, (5, 10): 2.13})
+    run_stream(pkv, wl, seed=77, n_frames=wl.frames, check={1, 5, 6}, rows=np.arange(wl.T), frames=fr,
+               fused=fused, tiles_per_split=tps)
+
+
 def test_unit_with_more_tiles_than_the_shared_tile_cache(pkv):
     """One unsplit CTA over 836 K/V tiles (16-token pages, one tile per page,
     and a 600-frame window; the host plan's tile count is checked in
