@@ -27,7 +27,7 @@ struct AttnArgs {
   float* part_lse;     // [slot][128] log2-sum-exp of each partial row
   void* out;           // [sum T, H, D]
   uint32_t* err;       // device error word
-  uint32_t* groups;    // [n_groups][2] arrival / departure counters of split groups
+  uint32_t* groups;    // [n_groups][4] arrivals, merge tickets, departures (and padding) of split groups
   int H;
   int fused_merge;     // the CTAs of a split group merge it themselves
   float scale_log2;    // log2(e) / sqrt(D)

@@ -90,7 +90,7 @@ struct KvPlanHeader {
   int32_t upload_bytes;
   int64_t off_part_o, off_part_lse;                    // byte offsets from the header
   int32_t n_groups;      // split groups
-  int32_t off_groups;    // byte offset of the groups' counters: [n_groups][2] uint32, zero
+  int32_t off_groups;    // byte offset of the groups' counters: [n_groups][4] uint32, zero
   int32_t fused_merge;   // 1: the attention CTAs of a split group merge it themselves
 };
 

@@ -355,7 +355,7 @@ WorkspaceLayout workspace_layout(const std::vector<const PageState*>& st) {
   off += align_up(units_cap * sizeof(KvUnit), 16);
   off += align_up(units_base * sizeof(KvMergeItem), 16);
   off += align_up(tiles_cap * sizeof(KvTile), 16);
-  off += align_up(units_base * 2 * sizeof(uint32_t), 16);   // split groups' counters
+  off += align_up(units_base * 4 * sizeof(uint32_t), 16);   // split groups' counters
   L.table_bytes = align_up(off, 256);
   L.off_part_o = L.table_bytes;
   L.off_part_lse = align_up(L.off_part_o + L.slot_cap * kTile * (size_t)D * 4, 256);
@@ -532,11 +532,16 @@ int build_plan(const std::vector<const PageState*>& st, const PlanInputs& in, Ho
   Hd.off_units = (int)off;  off += align_up(P.units.size() * sizeof(KvUnit), 16);
   Hd.off_merge = (int)off;  off += align_up(P.merges.size() * sizeof(KvMergeItem), 16);
   Hd.off_tiles = (int)off;  off += align_up(P.tiles.size() * sizeof(KvTile), 16);
-  Hd.off_groups = (int)off; off += align_up((size_t)n_groups * 2 * sizeof(uint32_t), 16);
+  Hd.off_groups = (int)off; off += align_up((size_t)n_groups * 4 * sizeof(uint32_t), 16);
   Hd.n_groups = n_groups;
-  // The CTAs of a split group wait for one another before merging it, which
-  // needs every CTA of the launch resident at once: one CTA per SM slot.
-  Hd.fused_merge = (n_groups > 0 && (int)P.units.size() <= target) ? 1 : 0;
+  // The attention CTAs of a split group merge it themselves when the launch
+  // has at most one CTA per SM slot (so the group's CTAs usually run at the
+  // same time and share the merge) and no group has more than 32 chunks (the
+  // kernel marks a group's shares in a 32-bit mask); otherwise a separate
+  // merge launch does.
+  int max_chunks = 0;
+  for (const KvUnit& u : P.units) max_chunks = std::max(max_chunks, (int)u.n_chunks);
+  Hd.fused_merge = (n_groups > 0 && (int)P.units.size() <= target && max_chunks <= 32) ? 1 : 0;
   Hd.upload_bytes = (int)off;
   Hd.off_part_o = (int64_t)WL.off_part_o;
   Hd.off_part_lse = (int64_t)WL.off_part_lse;

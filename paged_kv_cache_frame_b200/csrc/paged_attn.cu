@@ -113,6 +113,9 @@ struct AttnTmem {
 
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
+// How long a CTA of a split group waits for the group's other CTAs before it
+// leaves its share of the merge to the last one to arrive.
+constexpr uint64_t kGroupWaitNs = 50000ull;
 
 // Waits bounded by time only (used to drain in-flight async work on exit).
 __device__ __forceinline__ void mbar_drain_wait(uint64_t* bar, uint32_t parity) {
@@ -180,7 +183,7 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
   uint64_t* bar_drain = bar_s_full + 9;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_s_full + 10);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile int* merge_ok = reinterpret_cast<volatile int*>(tmem_slot + 2);
+  volatile uint32_t* merge_shares = tmem_slot + 2;   // shares of the split merge this CTA takes
   KvTile* tile_cache = reinterpret_cast<KvTile*>(smem + L::kTiles);
 
   const int warp = threadIdx.x >> 5;
@@ -906,49 +909,67 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
   }
   if (fuse) {
     // ---------------------------------------------------------- fused merge
-    // The n CTAs of a split group (all resident: the planner fuses only
-    // launches of at most one CTA per SM slot) each arrive once their
-    // partials are written, wait for the others, and merge rows
-    // [k R / n, (k + 1) R / n) of the group's R query rows. The last to
-    // leave resets the two counters for the next launch of the plan.
-    uint32_t* cnt = a.groups + 2 * u.group;
+    // The n CTAs of a split group (n <= 32) merge it in n shares of its R
+    // query rows, CTA k taking rows [k R / n, (k + 1) R / n), once every
+    // CTA's partials are written. One 64-bit word per group counts the
+    // arrivals (high half) and marks abandoned shares (low half). A CTA that
+    // is not the last to arrive waits a short, bounded time for the rest; if
+    // the time runs out while the group is still incomplete it abandons its
+    // share (a compare-and-swap that fails once the count is n) and leaves.
+    // The last to arrive gets every abandoned share with its arrival and
+    // merges them with its own. So no CTA depends on another being resident
+    // (another kernel may hold SMs), and each share is merged exactly once.
+    // The last CTA to leave resets the counters for the next launch.
+    unsigned long long* word = reinterpret_cast<unsigned long long*>(a.groups + 4 * u.group);
+    uint32_t* departed = a.groups + 4 * u.group + 2;
     const int n = u.n_chunks;
+    constexpr unsigned long long kArrive = 1ull << 32;
     if (threadIdx.x == 0) {
       __threadfence();   // release: every thread's partials (fenced, then the barrier) before the arrival
-      atomicAdd(cnt, 1u);
-      int ok = 1;
-      const uint64_t t0 = globaltimer_ns();
-      while (ld_acquire_gpu(cnt) < (uint32_t)n) {
-        if (globaltimer_ns() - t0 > kWaitLimitNs) { ok = 0; break; }
-        __nanosleep(64);
+      const unsigned long long old = atomicAdd(word, kArrive);
+      uint32_t mine = 1u << u.chunk;
+      if ((old >> 32) == (unsigned long long)(n - 1)) {
+        mine |= (uint32_t)old;   // the last to arrive: its share and every abandoned one
+      } else {
+        const uint64_t t0 = globaltimer_ns();
+        for (;;) {
+          const unsigned long long v = ld_acquire_gpu_u64(word);
+          if ((v >> 32) >= (unsigned long long)n) break;   // complete: merge the own share
+          if (globaltimer_ns() - t0 > kGroupWaitNs) {
+            if (atomicCAS(word, v, v | mine) == v) { mine = 0; break; }   // abandoned
+            continue;   // the word moved meanwhile: look again
+          }
+          __nanosleep(64);
+        }
       }
-      *merge_ok = ok;
+      *merge_shares = mine;
     }
     __syncthreads();
-    if (*merge_ok) {
-      __threadfence();   // order this thread's reads after the arrivals it saw
+    uint32_t mine = *merge_shares;
+    if (mine) {
+      __threadfence();   // order this CTA's reads after the arrivals it saw
       auto rows_of = [&](int t) { return t < nq ? min(kTile, rq.T - (u.qtile + t) * kTile) : tail_rows; };
       const int group_rows = rows_of(0) + (nq > 1 ? rows_of(1) : 0) + tail_rows;
-      const int r0 = (int)((long long)u.chunk * group_rows / n);
-      const int r1 = (int)((long long)(u.chunk + 1) * group_rows / n);
-      // 8 lanes per row: 48 rows of loads in flight at once
-      merge_rows_grouped<D, kFP16>(a.part_o, a.part_lse, n, r0 + (threadIdx.x >> 3), r1, kThreads / 8,
-                                   threadIdx.x & 7, [&](int gr, int* slot0, int* row, uint16_t** out_row) {
-        int t = 0, r = gr;
-        while (t < nq && r >= rows_of(t)) r -= rows_of(t++);
-        const int orow = rq.q_row0 + (u.qtile + t) * kTile + r;
-        *slot0 = u.slot[t] - u.chunk;
-        *row = r;
-        *out_row = reinterpret_cast<uint16_t*>(a.out) + ((size_t)orow * a.H + u.head) * D;
-      });
+      for (; mine; mine &= mine - 1) {
+        const int k = __ffs(mine) - 1;
+        const int r0 = (int)((long long)k * group_rows / n);
+        const int r1 = (int)((long long)(k + 1) * group_rows / n);
+        // 8 lanes per row: 48 rows of loads in flight at once
+        merge_rows_grouped<D, kFP16>(a.part_o, a.part_lse, n, r0 + (threadIdx.x >> 3), r1, kThreads / 8,
+                                     threadIdx.x & 7, [&](int gr, int* slot0, int* row, uint16_t** out_row) {
+          int t = 0, r = gr;
+          while (t < nq && r >= rows_of(t)) r -= rows_of(t++);
+          const int orow = rq.q_row0 + (u.qtile + t) * kTile + r;
+          *slot0 = u.slot[t] - u.chunk;
+          *row = r;
+          *out_row = reinterpret_cast<uint16_t*>(a.out) + ((size_t)orow * a.H + u.head) * D;
+        });
+      }
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-      if (!*merge_ok) atomicOr(a.err, 1u);
-      if (atomicAdd(cnt + 1, 1u) == (uint32_t)(n - 1)) {
-        atomicExch(cnt, 0u);
-        atomicExch(cnt + 1, 0u);
-      }
+    if (threadIdx.x == 0 && atomicAdd(departed, 1u) == (uint32_t)(n - 1)) {
+      atomicExch(word, 0ull);
+      atomicExch(departed, 0u);
     }
   }
   if (threadIdx.x == 0 && *abort_flag) atomicOr(a.err, 1u);

@@ -352,6 +352,24 @@ def test_unit_beyond_the_shared_tile_cache_host_plan(pkv):
     pkv.kv_plan_free(p)
 
 
+def test_in_kernel_merge_takes_at_most_32_chunks(pkv):
+    """The attention CTAs merge a split group themselves only while the
+    launch fits the device and no group has more than 32 chunks (the kernel
+    marks a group's shares in a 32-bit mask): 32 chunks of one tile merge in
+    the kernel, 54 run the merge as its own launch although their 108 CTAs
+    would fit."""
+    for W, frames, tiles, fused in ((20, 30, 32, 1), (40, 50, 54, 0)):
+        h = mk(pkv, 8, W, 64, 200)
+        for _ in range(frames):
+            step(pkv, h)
+        p = pkv.kv_plan([h], tiles_per_split=1)
+        s = pkv.kv_plan_get_stats(p)
+        assert s["n_kv_tiles"] == tiles and s["n_ctas"] == 2 * tiles <= 148
+        assert s["fused_merge"] == fused
+        pkv.kv_plan_free(p)
+        pkv.kv_destroy(h)
+
+
 def test_split_schedule_covers_each_unit(pkv):
     """Host plan for the 224x224 shape at frame 320: 160 tiles per head
     (71 earlier patch pages x 2, the current frame's page x 2, the earlier

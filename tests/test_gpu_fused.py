@@ -258,3 +258,43 @@ def test_group_of_streams_sharing_one_pool(pkv, fused):
             assert_close(out[j * wl.T:(j + 1) * wl.T], sos[i].expected(), f"step {step_i} stream {i}")
         assert np.array_equal(pool_bits(caches[0]), img.bits), f"step {step_i}: shared pool"
         assert caches[0].free_list() == pool.free
+
+
+def test_two_plans_on_two_streams_at_once(pkv):
+    """Two caches whose launches each fill the GPU (about 144 CTAs, split
+    merge in the kernel) run on two CUDA streams at the same time, many
+    times. Their CTAs interleave on the SMs, so the CTAs of a split group are
+    not all resident together: the merge must still complete (the last CTA
+    to arrive takes what the others left), outputs match the oracle and the
+    device error word stays clear."""
+    wl = small(256, H=16, S=2, W=8, frames=12)
+    caches = [new_cache(pkv, wl) for _ in range(2)]
+    frames = [Frames(wl, 300 + i) for i in range(2)]
+    oracles = [StreamOracle(wl.S, wl.W, wl.NS, wl.P, wl.dtype, fr.bits) for fr in frames]
+    wss = [workspace(pkv, [c]) for c in caches]
+    streams = [torch.cuda.Stream() for _ in range(2)]
+    rows = np.arange(0, wl.T, 7)
+    for f in range(wl.frames):
+        qs = []
+        for c, fr, so in zip(caches, frames, oracles):
+            q, k, v = (x.cuda() for x in fr.get(f))
+            c.append_frame(0, k, v)
+            c.evict_frames()
+            so.begin_frame(f, False)
+            qs.append(q)
+        if f == wl.frames - 1:
+            plans = [pkv.Plan([c], ws) for c, ws in zip(caches, wss)]
+            assert all(p.stats()["fused_merge"] for p in plans)
+            assert sum(p.stats()["n_ctas"] for p in plans) > 148
+            torch.cuda.synchronize()
+            outs = [torch.empty_like(q) for q in qs]
+            for _ in range(20):
+                for p, q, o, st in zip(plans, qs, outs, streams):
+                    with torch.cuda.stream(st):
+                        p.run(0, q, o, stream=st)
+            torch.cuda.synchronize()
+            for p, o, so in zip(plans, outs, oracles):
+                p.check_device()
+                assert_close(o[torch.as_tensor(rows)], so.expected(rows), "concurrent plans")
+        for so in oracles:
+            so.end_frame(True)

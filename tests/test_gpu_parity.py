@@ -393,15 +393,17 @@ def test_failed_append_launch_leaves_state_unchanged(pkv):
     assert_close(out, so.expected(), "after failed launches")
 
 
-@pytest.mark.parametrize("H", [2, 4])
-def test_more_than_32_chunks_per_split_unit(pkv, H):
-    """One K/V tile per CTA over 54 visible tiles (48 patch pages of 64 tokens;
-    300 special tokens on 5 pages, the open step's frame's 6 on a tile of
-    their own): 54 chunks per unit, past the merge's first 32-lane pass.
-    H = 2 gives 108 CTAs, which fit on the device at once, so the CTAs merge
-    their own groups; H = 4 gives 216, which do not, so the merge runs as its
-    own launch."""
-    wl = small(64, H=H, S=8, W=40, frames=50)
+@pytest.mark.parametrize("H,W,frames,tiles,fused", [(2, 40, 50, 54, 0), (4, 40, 50, 54, 0), (2, 20, 30, 32, 1)],
+                         ids=["54-chunks-H2", "54-chunks-H4", "32-chunks-H2"])
+def test_many_chunks_per_split_unit(pkv, H, W, frames, tiles, fused):
+    """One K/V tile per CTA, so a unit has as many chunks as visible tiles
+    (64-token pages, one tile each; the special tokens on their own pages,
+    the open step's frame's 6 on a tile of their own). 54 chunks: more than
+    the 32 the in-kernel merge takes (a 32-bit mask of shares), so the merge
+    runs as its own launch, past its first 32-lane pass; with H = 4 the 216
+    CTAs would not fit on the device at once either. 32 chunks with H = 2 (64
+    CTAs): the CTAs merge their groups themselves, the mask full."""
+    wl = small(64, H=H, S=8, W=W, frames=frames)
     fr = Frames(wl, seed=70)
     cache = new_cache(pkv, wl)
     so = StreamOracle(wl.S, wl.W, wl.NS, wl.P, wl.dtype, fr.bits)
@@ -412,13 +414,12 @@ def test_more_than_32_chunks_per_split_unit(pkv, H):
         so.begin_frame(f)
     plan = pkv.Plan([cache], workspace(pkv, [cache]), tiles_per_split=1)
     st = plan.stats()
-    assert st["tiles_per_cta"] == 1 and st["n_kv_tiles"] == 54
-    assert st["fused_merge"] == (1 if H == 2 else 0)
+    assert st["tiles_per_cta"] == 1 and st["n_kv_tiles"] == tiles
+    assert st["fused_merge"] == fused
     for rep in range(2):   # the group counters must be back at zero for the second run
         out = plan.run(0, q)
         plan.check_device()
         assert_close(out, so.expected(), f"H={H} run {rep}")
-
 
 
 @pytest.mark.parametrize("xs", [True, False])
