@@ -107,8 +107,11 @@ typedef struct kv_plan_stats {
   int n_kv_tiles;     /* 128-token K/V tiles summed over streams */
   int tiles_per_cta;  /* largest number of K/V tiles one CTA processes */
   long long visible_tokens; /* visible tokens summed over streams */
-  int fused_merge;    /* 1: split units are merged by their own CTAs (every CTA of
-                         the launch fits on the device at once), 0: by a merge launch */
+  int fused_merge;    /* 1: split units are merged by their own CTAs (the launch
+                         has at most one CTA per SM and no unit more than 32
+                         chunks; a CTA whose partners do not run alongside it,
+                         e.g. because another launch holds SMs, leaves its share
+                         to the last one), 0: by a merge launch */
   int run_launches;   /* kernel launches of one kv_run / kv_run_append (1, or 2 with
                          a merge launch) */
   int upload_launches; /* kernel launches kv_plan made to upload the tables */
@@ -266,8 +269,10 @@ int kv_plan(kv_plan_t** out, kv_cache_t* const* caches, int n_streams, int tiles
  *     out[i, h] = sum_j softmax_j(q[i, h] . k_j[h] / sqrt(D)) v_j[h]
  * over the visible tokens j of block `block`'s pool, no mask. q, out: device
  * [sum T, H, D] in the cache dtype; fp32 accumulation; out rounded to nearest
- * even. Launches the attention kernel and, when the plan splits a unit, the
- * split-KV merge kernel on `stream`.
+ * even. Launches the attention kernel and, when the plan splits a unit and
+ * its CTAs do not merge it themselves (kv_plan_stats.fused_merge), the
+ * split-KV merge kernel on `stream`. Plans may run on several streams at
+ * once.
  * Errors: KV_ERR_ARG, KV_ERR_STALE_PLAN, KV_ERR_NOT_APPENDED, KV_ERR_CUDA. */
 int kv_run(const kv_plan_t* plan, int block, const void* q, void* out, void* stream);
 
