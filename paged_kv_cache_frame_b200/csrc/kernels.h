@@ -16,6 +16,9 @@ struct AttnMaps {
   CUtensorMap q;
   CUtensorMap k, v;    // the frame's own k, v [sum T, H, D] (launches that append it)
   CUtensorMap kv[KV_MAX_STREAMS];
+  // the next block's pools: the first ring of each CTA's tiles is prefetched
+  // into L2 for the next block's launch of the same plan (prefetch_next)
+  CUtensorMap kv_next[KV_MAX_STREAMS];
 };
 
 struct AttnArgs {
@@ -38,6 +41,7 @@ struct AttnArgs {
   int row_vecs;        // 16-byte vectors per token row: H * D * 2 / 16
   const void* k;       // [sum T, H, D]
   const void* v;
+  int prefetch_next;   // kv_next holds the next block's pools
   void* pools[KV_MAX_STREAMS];   // this block's pool of each request
 };
 

@@ -448,6 +448,15 @@ int run_impl(const kv_plan_t* p, int block, const void* q, void* out, const void
     }
     maps.kv[r] = c->dev->maps[block];
   }
+  // Blocks run in order in a frame step, all on this plan: the CTAs prefetch
+  // the first tiles of their units from the next block's pools into L2 once
+  // their own loads are issued, so the next launch starts on L2 hits.
+  a.prefetch_next = block + 1 < B;
+  for (size_t r = 0; r < p->caches.size() && a.prefetch_next; ++r) {
+    const kv_cache* c = p->caches[r];
+    if (!c->dev->bound[block + 1]) a.prefetch_next = 0;
+    else maps.kv_next[r] = c->dev->maps[block + 1];
+  }
   int rc = encode_rows_map(&maps.q, q, p->H, p->D, p->total_T, p->dtype);
   if (rc == KV_OK && append) rc = encode_rows_map(&maps.k, k, p->H, p->D, p->total_T, p->dtype);
   if (rc == KV_OK && append) rc = encode_rows_map(&maps.v, v, p->H, p->D, p->total_T, p->dtype);

@@ -370,6 +370,21 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
         load_kv(j);
         if (j >= STAGES) prefetch_l2(j + kL2Ahead);
       }
+      if (a.prefetch_next) {
+        // The next block's launch of this plan runs the same units: the
+        // first ring of this unit's tiles in its pools (rows of earlier
+        // frames) into L2 now, while this CTA still computes.
+        const CUtensorMap* mn = &maps.kv_next[u.req];
+        for (int jj = 0; jj < min(n_tiles, STAGES + kL2Ahead); ++jj) {
+          const KvTile t = tile_at(jj);
+          if (t.krow != kNotCurrent) continue;
+#pragma unroll
+          for (int kb = 0; kb < D / 64; ++kb) {
+            tma_prefetch_l2_3d(mn, kb * 64, u.head, t.row);
+            tma_prefetch_l2_3d(mn, kb * 64, u.head, t.row + rq.page_size);
+          }
+        }
+      }
       drain_loads(j);
     }
   } else if (warp == R::kMma) {
