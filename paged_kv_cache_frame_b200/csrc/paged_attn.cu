@@ -72,6 +72,7 @@ namespace pkv {
 
 constexpr int kMaxSmemTiles = 512;   // tile descriptors cached in shared memory
 constexpr int kL2Ahead = 4;          // K/V tiles prefetched into L2 beyond the shared-memory ring
+constexpr int kNextAhead = 8;        // first tiles of the unit prefetched for the next block's launch
 
 template <int D>
 struct AttnRoles {
@@ -375,7 +376,7 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
         // first ring of this unit's tiles in its pools (rows of earlier
         // frames) into L2 now, while this CTA still computes.
         const CUtensorMap* mn = &maps.kv_next[u.req];
-        for (int jj = 0; jj < min(n_tiles, STAGES + kL2Ahead); ++jj) {
+        for (int jj = 0; jj < min(n_tiles, kNextAhead); ++jj) {
           const KvTile t = tile_at(jj);
           if (t.krow != kNotCurrent) continue;
 #pragma unroll
