@@ -450,8 +450,11 @@ int run_impl(const kv_plan_t* p, int block, const void* q, void* out, const void
   }
   // Blocks run in order in a frame step, all on this plan: the CTAs prefetch
   // the first tiles of their units from the next block's pools into L2 once
-  // their own loads are issued, so the next launch starts on L2 hits.
-  a.prefetch_next = block + 1 < B;
+  // their own loads are issued, so the next launch starts on L2 hits. Only
+  // while a launch's K/V fits well inside L2 (126 MB): a larger launch evicts
+  // the prefetched tiles before the next one reads them.
+  const double kv_bytes = 2.0 * (double)p->hp.visible * p->H * p->D * 2.0;
+  a.prefetch_next = block + 1 < B && kv_bytes <= 80.0 * (1 << 20);
   for (size_t r = 0; r < p->caches.size() && a.prefetch_next; ++r) {
     const kv_cache* c = p->caches[r];
     if (!c->dev->bound[block + 1]) a.prefetch_next = 0;
