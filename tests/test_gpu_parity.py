@@ -440,6 +440,21 @@ def test_camera_only_page_sizes(pkv, ps):
     run_stream(pkv, wl, seed=92 + ps, n_frames=wl.frames, check={39}, camera_only=True, tiles_per_split=1)
 
 
+@pytest.mark.parametrize("fused", [False, True])
+def test_visibility_options_head_dim_128_fp16(pkv, fused):
+    """camera_only and cross_frame_special = False on the head_dim 128 fp16
+    path (P over S in two rotating buffers, a tail of at most 8 rows): 256
+    patch tokens per frame, so each frame adds two full query tiles and a
+    6-row tail; every row checked, with and without a split."""
+    wl = small(256, H=2, D=128, dtype="fp16", S=2, W=3, frames=14)
+    run_stream(pkv, wl, seed=95, n_frames=wl.frames, check={0, 6, 13}, rows=np.arange(wl.T), camera_only=True,
+               fused=fused)
+    run_stream(pkv, wl, seed=96, n_frames=wl.frames, check={13}, rows=np.arange(wl.T), camera_only=True,
+               tiles_per_split=1, fused=fused)
+    run_stream(pkv, wl, seed=97, n_frames=wl.frames, check={6, 13}, rows=np.arange(wl.T), cross_special=False,
+               fused=fused)
+
+
 def test_camera_only_224_stream(pkv):
     wl = dataclasses.replace(workload.WORKLOADS[1], frames=200)
     run_stream(pkv, wl, seed=93, n_frames=wl.frames, check={0, 100, 199}, rows=sample_rows(wl.T, 93),
