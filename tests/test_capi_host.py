@@ -190,12 +190,11 @@ OPS = st.lists(st.sampled_from(["key", "key", "key", "defer_keep", "defer_drop",
 
 @settings(max_examples=120, deadline=None)
 @given(ops=OPS, S=st.integers(0, 3), W=st.integers(0, 4), ps=st.sampled_from([1, 5, 16, 130]),
-       B=st.integers(1, 3), xs=st.booleans())
-def test_state_machine_bit_exact_vs_oracle(pkv, ops, S, W, ps, B, xs):
-    NS = 6
+       B=st.integers(1, 3), xs=st.booleans(), NS=st.sampled_from([6, 6, 1, 0]))
+def test_state_machine_bit_exact_vs_oracle(pkv, ops, S, W, ps, B, xs, NS):
     max_pages = S + W + 1 + (NS * 60) // ps + 2
     m = PageModel(S, W, ps, max_pages, NS=NS, cross_frame_special=xs)
-    h = mk(pkv, S, W, ps, max_pages, B=B)
+    h = mk(pkv, S, W, ps, max_pages, NS=NS, B=B)
     pkv.kv_set_cross_frame_special(h, xs)
     E = pkv.capi
     try:
@@ -335,6 +334,34 @@ def test_kv_tiles_cover_visible_tokens_exactly_once(pkv, ps, n, xs):
     assert s["visible_tokens"] == m.visible_token_count()
     assert s["n_kv_tiles"] == len(tiles)
     pkv.kv_plan_free(p)
+
+
+@pytest.mark.parametrize("S,W,NS,xs", [(2, 3, 0, True), (8, 64, 0, True), (2, 0, 6, True), (2, 0, 6, False),
+                                        (0, 0, 6, True), (0, 0, 1, True), (1, 0, 1, False)])
+def test_kv_tiles_degenerate_configs(pkv, S, W, NS, xs):
+    """No special tokens, an empty sliding window, or both scale frames and
+    window empty: after every frame the K/V tiles cover exactly the oracle's
+    visible tokens (with W = 0 the frame just appended is already evicted)."""
+    ps, n = 64, 40
+    max_pages = S + W + 1 + math.ceil(NS * n / ps) + 1
+    h = mk(pkv, S, W, ps, max_pages, NS=NS)
+    pkv.kv_set_cross_frame_special(h, xs)
+    m = PageModel(S, W, ps, max_pages, NS=NS, cross_frame_special=xs)
+    try:
+        for f in range(n):
+            step(pkv, h)
+            m.append(f)
+            m.evict()
+            p = pkv.kv_plan([h])
+            try:
+                want = [(pg, t) for _, pg in m.patch_pages_visible() for t in range(ps)]
+                want += [(m.Np + j // ps, j % ps) for j in m.visible_special_index()]
+                assert sorted(tile_cover(pkv.kv_get_kv_tiles(p), ps)) == sorted(want), f"frame {f}"
+                assert pkv.kv_plan_get_stats(p)["visible_tokens"] == m.visible_token_count() == len(want)
+            finally:
+                pkv.kv_plan_free(p)
+    finally:
+        pkv.kv_destroy(h)
 
 
 def test_unit_beyond_the_shared_tile_cache_host_plan(pkv):

@@ -298,3 +298,65 @@ def test_two_plans_on_two_streams_at_once(pkv):
                 assert_close(o[torch.as_tensor(rows)], so.expected(rows), "concurrent plans")
         for so in oracles:
             so.end_frame(True)
+
+
+@pytest.mark.parametrize("fused", [False, True])
+def test_batch_at_the_stream_limit(pkv, fused):
+    """One plan over KV_MAX_STREAMS streams, the most a batch takes, all of one
+    kv_init_group with two blocks (so a block-0 launch also prefetches from
+    every stream's block-1 pool). Streams join at different steps: at the last
+    steps their windows, scale frames and special streams all differ. Both
+    blocks match the oracle for every stream, and each block's shared pool
+    matches the oracle's image after every step."""
+    from oracle import SharedPatchPool
+    n, joins, steps = pkv.KV_MAX_STREAMS, 8, 12
+    wl = small(16, H=2, S=1, W=2, frames=steps)
+    T = wl.T
+    sp_pages = -(-wl.NS * steps // wl.page_size)
+    Np = n * wl.patch_pages
+    caches = pkv.PagedKVCache.group(n, Np + n * sp_pages, wl.page_size, wl.H, wl.D, wl.S, wl.W,
+                                    num_blocks=2, num_special=wl.NS, dtype=wl.dtype,
+                                    patch_pages=Np, special_pages=sp_pages)
+    caches[0].allocate_pools("cuda")
+    pool = SharedPatchPool(Np)
+    ms = [PageModel(wl.S, wl.W, wl.page_size, Np + n * sp_pages, NS=wl.NS, shared=pool,
+                    sp_base=Np + i * sp_pages, sp_pages=sp_pages) for i in range(n)]
+    imgs = [PoolImage(ms[0], wl.H, wl.D) for _ in range(2)]
+    frs = [[Frames(wl, seed=131, stream=i, block=b) for b in range(2)] for i in range(n)]
+    sos = [[StreamOracle(wl.S, wl.W, wl.NS, wl.P, wl.dtype, fr.bits) for fr in pair] for pair in frs]
+    ws = workspace(pkv, caches)
+    ages = [0] * n
+    for step in range(steps):
+        live = [i for i in range(n) if i % joins <= step]
+        qkv = [[frs[i][b].get(ages[i]) for b in range(2)] for i in live]
+        for j, i in enumerate(live):
+            if fused:
+                caches[i].begin_frame()
+            else:
+                caches[i].append_frame(0, qkv[j][0][1].cuda(), qkv[j][0][2].cuda())
+            caches[i].evict_frames()
+            page, sp0 = ms[i].append(ages[i])
+            ms[i].evict()
+            for b in range(2):
+                imgs[b].write(page, sp0, bits16(qkv[j][b][1]), bits16(qkv[j][b][2]), model=ms[i])
+                sos[i][b].begin_frame(ages[i])
+            ages[i] += 1
+        plan = pkv.Plan([caches[i] for i in live], ws)
+        assert plan.stats()["n_streams"] == len(live)
+        for b in range(2):
+            q, k, v = (torch.cat([x[b][t] for x in qkv]).cuda() for t in range(3))
+            if fused:
+                out = plan.run_append(b, k, v, q)
+            else:
+                if b == 1:
+                    for j, i in enumerate(live):
+                        caches[i].append_frame(1, k[j * T:(j + 1) * T], v[j * T:(j + 1) * T])
+                out = plan.run(b, q)
+            plan.check_device()
+            if step >= steps - 2:
+                for j, i in enumerate(live):
+                    assert_close(out[j * T:(j + 1) * T], sos[i][b].expected(),
+                                 f"step {step} block {b} stream {i}")
+            assert np.array_equal(pool_bits(caches[0], b), imgs[b].bits), f"step {step} block {b}: shared pool"
+        assert caches[0].free_list() == pool.free
+    assert sorted(set(ages)) == list(range(steps - joins + 1, steps + 1))

@@ -290,6 +290,32 @@ def test_include_scale_frames_off_is_zero_scale_frames(pkv):
                dense={89})
 
 
+@pytest.mark.parametrize("ps,D", [(128, 64), (130, 64), (64, 128), (136, 128)])
+@pytest.mark.parametrize("fused", [False, True])
+def test_no_special_tokens(pkv, ps, D, fused):
+    """num_special = 0: a frame is its patch tokens alone (T = page size), the
+    special stream stays empty and only patch pages are visible. 128 rows are
+    one full query tile with no tail, 130 and 136 leave a tail of 2 and 8
+    rows, 64 rows a partial tile; every row of every frame is checked."""
+    wl = dataclasses.replace(small(ps, D=D, dtype="fp16" if D == 128 else "bf16", frames=14), NS=0)
+    assert wl.T == ps
+    run_stream(pkv, wl, seed=140 + ps, n_frames=wl.frames, check=set(range(wl.frames)), rows=np.arange(wl.T),
+               fused=fused)
+
+
+@pytest.mark.parametrize("S,xs", [(2, True), (2, False), (0, True)])
+@pytest.mark.parametrize("fused", [False, True])
+def test_empty_window(pkv, S, xs, fused):
+    """sliding_window = 0: once the scale frames are set, a frame's patch
+    tokens are evicted in the step that appends them, so its queries see the
+    scale frames' patches and the special tokens only (with S = 0 the special
+    tokens alone). The frame is still written to its page, which the next
+    frame takes again."""
+    wl = small(64, S=S, W=0, frames=12)
+    run_stream(pkv, wl, seed=150 + S, n_frames=wl.frames, check=set(range(wl.frames)), rows=np.arange(wl.T),
+               cross_special=xs, fused=fused)
+
+
 def test_full_224_stream_block0_sampled(pkv):
     """Every row of the last frame against the oracle (and the fp32 gather),
     sampled rows elsewhere."""
