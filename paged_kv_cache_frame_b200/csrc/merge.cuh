@@ -110,49 +110,68 @@ __device__ __forceinline__ void merge_row_warp(const float* part_o, const float*
 namespace pkv {
 
 // The same merge for many rows at once, 8 lanes per row: lane l of a row's
-// group holds output columns [l D/8, (l + 1) D/8) and chunk weights l, l + 8,
-// ...; the chunks' rows are loaded 8 (4 for D = 128) at a time, all in
-// flight before the first multiply, so a CTA of 384 threads has 48 rows'
-// loads outstanding together. row_of(i) gives the i-th row's (slot0, row,
-// output row pointer); rows i = first, first + stride, ... < end go to the
-// calling group.
+// group holds output columns [l D/8, (l + 1) D/8) and the log2-sum-exps of
+// chunks l, l + 8, l + 16, l + 24 (n <= 32). The lse values and the rows of
+// the first 12 chunks (6 for D = 128) are all requested before the first
+// result is used, so a group of up to 12 chunks costs one L2 round trip; a
+// CTA of 384 threads keeps 48 rows' loads in flight. row_of(i) gives the
+// i-th row's (slot0, row, output row pointer); rows i = first, first +
+// stride, ... < end go to the calling group.
 template <int D, bool kFP16, typename RowOf>
 __device__ __forceinline__ void merge_rows_grouped(const float* part_o, const float* part_lse, int n, int first,
                                                    int end, int stride, int l8, RowOf row_of) {
   constexpr int kCols = D / 8;                 // columns per lane: 8 or 16
   constexpr int kV4 = kCols / 4;               // float4 per lane per chunk
-  constexpr int kBatch = D == 64 ? 8 : 4;      // chunks loaded together
-  const unsigned gmask = 0xFFu << (threadIdx.x & 24);   // this row's 8 lanes
+  constexpr int kBatch = D == 64 ? 12 : 6;     // chunks loaded together
+  const int g0 = threadIdx.x & 24;             // first lane of this row's group
+  const unsigned gmask = 0xFFu << g0;
+  constexpr size_t kStride = (size_t)kTile * D / 4;   // one slot, in float4
   for (int i = first; i < end; i += stride) {
     int slot0, row;
     uint16_t* out_row;
     row_of(i, &slot0, &row, &out_row);
     const float* lse = part_lse + (size_t)slot0 * kTile + row;
-    // max of the chunks' log2-sum-exps over the group
-    float top = -INFINITY;
-    for (int c = l8; c < n; c += 8) top = fmaxf(top, __ldcg(lse + (size_t)c * kTile));
+    const float4* po = reinterpret_cast<const float4*>(part_o + ((size_t)slot0 * kTile + row) * D + l8 * kCols);
+    float lv[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) lv[q] = l8 + 8 * q < n ? __ldcg(lse + (size_t)(l8 + 8 * q) * kTile) : -INFINITY;
+    float4 x[kBatch][kV4];
+#pragma unroll
+    for (int k = 0; k < kBatch; ++k)
+      if (k < n)
+#pragma unroll
+        for (int v = 0; v < kV4; ++v) x[k][v] = __ldcg(po + (size_t)k * kStride + v);
+    // max of the chunks' log2-sum-exps over the group, then each lane's weights
+    float top = fmaxf(fmaxf(lv[0], lv[1]), fmaxf(lv[2], lv[3]));
 #pragma unroll
     for (int o = 1; o < 8; o <<= 1) top = fmaxf(top, __shfl_xor_sync(gmask, top, o));
+    float wl[4];
+    float wsum = 0.f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      wl[q] = l8 + 8 * q < n ? ex2_approx(lv[q] - top) : 0.f;
+      wsum += wl[q];
+    }
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) wsum += __shfl_xor_sync(gmask, wsum, o);
     float acc[kCols];
 #pragma unroll
     for (int k = 0; k < kCols; ++k) acc[k] = 0.f;
-    float wsum = 0.f;
-    const float4* po = reinterpret_cast<const float4*>(part_o + ((size_t)slot0 * kTile + row) * D + l8 * kCols);
-    constexpr size_t kStride = (size_t)kTile * D / 4;   // one slot, in float4
     for (int c0 = 0; c0 < n; c0 += kBatch) {
-      float4 x[kBatch][kV4];
+      if (c0 > 0) {
 #pragma unroll
-      for (int k = 0; k < kBatch; ++k)
-        if (c0 + k < n)
+        for (int k = 0; k < kBatch; ++k)
+          if (c0 + k < n)
 #pragma unroll
-          for (int v = 0; v < kV4; ++v) x[k][v] = __ldcg(po + (size_t)(c0 + k) * kStride + v);
-      // lane l8 < kBatch holds chunk c0 + l8's weight
-      const float lw = (l8 < kBatch && c0 + l8 < n) ? ex2_approx(__ldcg(lse + (size_t)(c0 + l8) * kTile) - top) : 0.f;
-      wsum += lw;
+            for (int v = 0; v < kV4; ++v) x[k][v] = __ldcg(po + (size_t)(c0 + k) * kStride + v);
+      }
 #pragma unroll
       for (int k = 0; k < kBatch; ++k) {
-        const float w = __shfl_sync(gmask, lw, (threadIdx.x & 24) + k);
-        if (c0 + k < n) {
+        const int c = c0 + k;   // uniform over the group: chunk c's weight is wl[c / 8] of lane c % 8
+        const int q = c >> 3;
+        const float sel = q == 0 ? wl[0] : q == 1 ? wl[1] : q == 2 ? wl[2] : wl[3];
+        const float w = __shfl_sync(gmask, sel, g0 + (c & 7));
+        if (c < n) {
 #pragma unroll
           for (int v = 0; v < kV4; ++v) {
             acc[4 * v + 0] = fmaf(w, x[k][v].x, acc[4 * v + 0]);
@@ -163,8 +182,6 @@ __device__ __forceinline__ void merge_rows_grouped(const float* part_o, const fl
         }
       }
     }
-#pragma unroll
-    for (int o = 1; o < 8; o <<= 1) wsum += __shfl_xor_sync(gmask, wsum, o);
     const float inv = 1.f / wsum;
     uint32_t pk[kCols / 2];
 #pragma unroll

@@ -915,7 +915,6 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
   }
 
   const bool fuse = a.fused_merge && u.n_chunks > 1;
-  if (fuse) __threadfence();   // this CTA's partials, before its arrival below
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -941,10 +940,13 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
     const int n = u.n_chunks;
     constexpr unsigned long long kArrive = 1ull << 32;
     if (threadIdx.x == 0) {
-      __threadfence();   // release: every thread's partials (fenced, then the barrier) before the arrival
+      // release: every thread's partials (ordered before this thread by the
+      // barrier above) before the arrival
+      fence_acq_rel_gpu();
       const unsigned long long old = atomicAdd(word, kArrive);
       uint32_t mine = 1u << u.chunk;
       if ((old >> 32) == (unsigned long long)(n - 1)) {
+        fence_acq_rel_gpu();     // acquire: the other CTAs' partials, released by their arrivals
         mine |= (uint32_t)old;   // the last to arrive: its share and every abandoned one
       } else {
         const uint64_t t0 = globaltimer_ns();
@@ -960,10 +962,9 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
       }
       *merge_shares = mine;
     }
-    __syncthreads();
+    __syncthreads();   // the acquire above, then this barrier, orders every thread's reads below
     uint32_t mine = *merge_shares;
     if (mine) {
-      __threadfence();   // order this CTA's reads after the arrivals it saw
       auto rows_of = [&](int t) { return t < nq ? min(kTile, rq.T - (u.qtile + t) * kTile) : tail_rows; };
       const int group_rows = rows_of(0) + (nq > 1 ? rows_of(1) : 0) + tail_rows;
       for (; mine; mine &= mine - 1) {

@@ -98,6 +98,12 @@ __device__ __forceinline__ unsigned long long ld_acquire_gpu_u64(const unsigned 
   return v;
 }
 
+// A fence that, after a barrier of the CTA, makes its relaxed atomic that
+// follows a release of every write the CTA made before the barrier, and
+// that, after a relaxed atomic read, makes it an acquire (PTX memory model:
+// release and acquire patterns at GPU scope).
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
                                             int y, int z) {
