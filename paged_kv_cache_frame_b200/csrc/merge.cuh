@@ -109,39 +109,35 @@ __device__ __forceinline__ void merge_row_warp(const float* part_o, const float*
 
 namespace pkv {
 
-// The same merge for many rows at once, 8 lanes per row: lane l of a row's
-// group holds output columns [l D/8, (l + 1) D/8) and the log2-sum-exps of
-// chunks l, l + 8, l + 16, l + 24 (n <= 32). The lse values and the rows of
-// the first 12 chunks (6 for D = 128) are all requested before the first
-// result is used, so a group of up to 12 chunks costs one L2 round trip; a
-// CTA of 384 threads keeps 48 rows' loads in flight. row_of(i) gives the
-// i-th row's (slot0, row, output row pointer); rows i = first, first +
-// stride, ... < end go to the calling group.
-template <int D, bool kFP16, typename RowOf>
-__device__ __forceinline__ void merge_rows_grouped(const float* part_o, const float* part_lse, int n, int first,
-                                                   int end, int stride, int l8, RowOf row_of) {
-  constexpr int kCols = D / 8;                 // columns per lane: 8 or 16
-  constexpr int kV4 = kCols / 4;               // float4 per lane per chunk
-  constexpr int kBatch = D == 64 ? 12 : 6;     // chunks loaded together
+// The same merge for the S rows of one share, their chunks' partial rows
+// already requested into shared memory (`stage`, [n][S][D] fp32): 8 lanes
+// per row, lane l holding output columns 4 (l + 8 v) .. 4 (l + 8 v) + 3 (v <
+// D/32, so a row's 8 lanes read 128 contiguous bytes at a time) and the
+// log2-sum-exps of chunks l, l + 8, l + 16, l + 24 (n <= 32). Each row's lse
+// values are loaded before `wait()` (the stage's completion) is called.
+// row_of(i) gives share row i's (slot0, row, output row pointer); rows i =
+// first, first + stride, ... < S go to the calling group. Returns false if
+// wait() failed (nothing was read from the stage then).
+template <int D, bool kFP16, typename Wait, typename RowOf>
+__device__ __forceinline__ bool merge_rows_staged(const float* stage, int S, const float* part_lse, int n, int first,
+                                                  int stride, int l8, Wait wait, RowOf row_of) {
+  constexpr int kV4 = D / 32;                  // float4 per lane per chunk
   const int g0 = threadIdx.x & 24;             // first lane of this row's group
   const unsigned gmask = 0xFFu << g0;
-  constexpr size_t kStride = (size_t)kTile * D / 4;   // one slot, in float4
-  for (int i = first; i < end; i += stride) {
+  const size_t chunk4 = (size_t)S * D / 4;     // one chunk's rows in the stage, in float4
+  bool waited = false;
+  for (int i = first; i < S; i += stride) {
     int slot0, row;
     uint16_t* out_row;
     row_of(i, &slot0, &row, &out_row);
     const float* lse = part_lse + (size_t)slot0 * kTile + row;
-    const float4* po = reinterpret_cast<const float4*>(part_o + ((size_t)slot0 * kTile + row) * D + l8 * kCols);
     float lv[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) lv[q] = l8 + 8 * q < n ? __ldcg(lse + (size_t)(l8 + 8 * q) * kTile) : -INFINITY;
-    float4 x[kBatch][kV4];
-#pragma unroll
-    for (int k = 0; k < kBatch; ++k)
-      if (k < n)
-#pragma unroll
-        for (int v = 0; v < kV4; ++v) x[k][v] = __ldcg(po + (size_t)k * kStride + v);
-    // max of the chunks' log2-sum-exps over the group, then each lane's weights
+    if (!waited) {
+      if (!wait()) return false;
+      waited = true;
+    }
     float top = fmaxf(fmaxf(lv[0], lv[1]), fmaxf(lv[2], lv[3]));
 #pragma unroll
     for (int o = 1; o < 8; o <<= 1) top = fmaxf(top, __shfl_xor_sync(gmask, top, o));
@@ -154,43 +150,35 @@ __device__ __forceinline__ void merge_rows_grouped(const float* part_o, const fl
     }
 #pragma unroll
     for (int o = 1; o < 8; o <<= 1) wsum += __shfl_xor_sync(gmask, wsum, o);
-    float acc[kCols];
+    float acc[kV4][4];
 #pragma unroll
-    for (int k = 0; k < kCols; ++k) acc[k] = 0.f;
-    for (int c0 = 0; c0 < n; c0 += kBatch) {
-      if (c0 > 0) {
+    for (int v = 0; v < kV4; ++v) acc[v][0] = acc[v][1] = acc[v][2] = acc[v][3] = 0.f;
+    const float4* xs = reinterpret_cast<const float4*>(stage + (size_t)i * D) + l8;
+    for (int c = 0; c < n; ++c) {
+      // chunk c's weight is wl[c / 8] of lane c % 8 (c is uniform over the group)
+      const int q = c >> 3;
+      const float sel = q == 0 ? wl[0] : q == 1 ? wl[1] : q == 2 ? wl[2] : wl[3];
+      const float w = __shfl_sync(gmask, sel, g0 + (c & 7));
 #pragma unroll
-        for (int k = 0; k < kBatch; ++k)
-          if (c0 + k < n)
-#pragma unroll
-            for (int v = 0; v < kV4; ++v) x[k][v] = __ldcg(po + (size_t)(c0 + k) * kStride + v);
-      }
-#pragma unroll
-      for (int k = 0; k < kBatch; ++k) {
-        const int c = c0 + k;   // uniform over the group: chunk c's weight is wl[c / 8] of lane c % 8
-        const int q = c >> 3;
-        const float sel = q == 0 ? wl[0] : q == 1 ? wl[1] : q == 2 ? wl[2] : wl[3];
-        const float w = __shfl_sync(gmask, sel, g0 + (c & 7));
-        if (c < n) {
-#pragma unroll
-          for (int v = 0; v < kV4; ++v) {
-            acc[4 * v + 0] = fmaf(w, x[k][v].x, acc[4 * v + 0]);
-            acc[4 * v + 1] = fmaf(w, x[k][v].y, acc[4 * v + 1]);
-            acc[4 * v + 2] = fmaf(w, x[k][v].z, acc[4 * v + 2]);
-            acc[4 * v + 3] = fmaf(w, x[k][v].w, acc[4 * v + 3]);
-          }
-        }
+      for (int v = 0; v < kV4; ++v) {
+        const float4 y = xs[(size_t)c * chunk4 + 8 * v];
+        acc[v][0] = fmaf(w, y.x, acc[v][0]);
+        acc[v][1] = fmaf(w, y.y, acc[v][1]);
+        acc[v][2] = fmaf(w, y.z, acc[v][2]);
+        acc[v][3] = fmaf(w, y.w, acc[v][3]);
       }
     }
     const float inv = 1.f / wsum;
-    uint32_t pk[kCols / 2];
 #pragma unroll
-    for (int k = 0; k < kCols; k += 2)
-      pk[k / 2] = kFP16 ? cvt_pack_f16(acc[k] * inv, acc[k + 1] * inv) : cvt_pack_bf16(acc[k] * inv, acc[k + 1] * inv);
-    uint4* o = reinterpret_cast<uint4*>(out_row + l8 * kCols);
-#pragma unroll
-    for (int k = 0; k < kCols / 8; ++k) o[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+    for (int v = 0; v < kV4; ++v) {
+      const uint32_t p0 = kFP16 ? cvt_pack_f16(acc[v][0] * inv, acc[v][1] * inv)
+                                : cvt_pack_bf16(acc[v][0] * inv, acc[v][1] * inv);
+      const uint32_t p1 = kFP16 ? cvt_pack_f16(acc[v][2] * inv, acc[v][3] * inv)
+                                : cvt_pack_bf16(acc[v][2] * inv, acc[v][3] * inv);
+      *reinterpret_cast<uint2*>(out_row + 4 * (l8 + 8 * v)) = make_uint2(p0, p1);
+    }
   }
+  return true;
 }
 
 }  // namespace pkv

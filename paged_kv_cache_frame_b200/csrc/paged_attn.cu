@@ -967,20 +967,46 @@ __global__ void __launch_bounds__(AttnRoles<D>::kThreads, 1)
     if (mine) {
       auto rows_of = [&](int t) { return t < nq ? min(kTile, rq.T - (u.qtile + t) * kTile) : tail_rows; };
       const int group_rows = rows_of(0) + (nq > 1 ? rows_of(1) : 0) + tail_rows;
+      // A share's rows of every chunk's partials are staged in shared memory
+      // (the Q and K/V stages, idle now) by bulk copies that complete on
+      // bar_q, whose phase 0 was the Q load. A share of a group of R <= 272
+      // rows in n <= 32 chunks has S <= ceil(R / n) rows: S n < R + n rows.
+      float* stage = reinterpret_cast<float*>(smem);
+      static_assert((2 * kTile + kMaxTailRows + 31) * D * 4 <= L::kTailO, "merge stage fits the Q and K/V stages");
+      uint32_t phase = 1;
       for (; mine; mine &= mine - 1) {
         const int k = __ffs(mine) - 1;
         const int r0 = (int)((long long)k * group_rows / n);
         const int r1 = (int)((long long)(k + 1) * group_rows / n);
-        // 8 lanes per row: 48 rows of loads in flight at once
-        merge_rows_grouped<D, kFP16>(a.part_o, a.part_lse, n, r0 + (threadIdx.x >> 3), r1, kThreads / 8,
-                                     threadIdx.x & 7, [&](int gr, int* slot0, int* row, uint16_t** out_row) {
-          int t = 0, r = gr;
-          while (t < nq && r >= rows_of(t)) r -= rows_of(t++);
-          const int orow = rq.q_row0 + (u.qtile + t) * kTile + r;
-          *slot0 = u.slot[t] - u.chunk;
-          *row = r;
-          *out_row = reinterpret_cast<uint16_t*>(a.out) + ((size_t)orow * a.H + u.head) * D;
-        });
+        const int S = r1 - r0;
+        if (threadIdx.x == 0) {
+          fence_proxy_async_global();   // the partials acquired above, before the copies read them
+          fence_async_smem();           // the stage's earlier reads (before the barrier), before the copies write it
+          mbar_arrive_expect_tx(bar_q, (uint32_t)(S * n * D * 4));
+          // [r0, r1) by query tile (index nq: the tail), one copy per chunk
+          for (int t = 0, gr = 0; t <= nq; gr += rows_of(t), ++t) {
+            const int a0 = max(r0, gr), a1 = min(r1, gr + rows_of(t));
+            if (a1 <= a0) continue;
+            const float* src = a.part_o + ((size_t)(u.slot[t] - u.chunk) * kTile + (a0 - gr)) * D;
+            for (int c = 0; c < n; ++c)
+              bulk_g2s(stage + ((size_t)c * S + (a0 - r0)) * D, src + (size_t)c * kTile * D,
+                       (uint32_t)((a1 - a0) * D * 4), bar_q);
+          }
+        }
+        const bool got = merge_rows_staged<D, kFP16>(
+            stage, S, a.part_lse, n, threadIdx.x >> 3, kThreads / 8, threadIdx.x & 7,
+            [&]() { return mbar_wait(bar_q, phase & 1u, abort_flag); },
+            [&](int i, int* slot0, int* row, uint16_t** out_row) {
+              int t = 0, r = r0 + i;
+              while (t < nq && r >= rows_of(t)) r -= rows_of(t++);
+              const int orow = rq.q_row0 + (u.qtile + t) * kTile + r;
+              *slot0 = u.slot[t] - u.chunk;
+              *row = r;
+              *out_row = reinterpret_cast<uint16_t*>(a.out) + ((size_t)orow * a.H + u.head) * D;
+            });
+        if (!got) mbar_drain_wait(bar_q, phase & 1u);   // no copy may land after the stage is reused
+        __syncthreads();   // the stage is free for the next share's copies
+        phase ^= 1u;
       }
     }
     __syncthreads();
